@@ -1,0 +1,285 @@
+"""Pins for the CPU oracle: each check holds it to something other than itself.
+
+* brute force over every mask on tiny inputs, in exact rational arithmetic;
+* special cases that reduce to a plain matrix-product chain (numpy): top-K with
+  K = d_ff is the dense SwiGLU FFN, a threshold below every gate value is an
+  affine-gated (bilinear) FFN, LoPA's two stages equal x (A B);
+* the closed-form active count of a Gaussian gate;
+* the sparse == dense invariant behind gate-first evaluation ("Model Casting
+  and Low-Parameter Gating", abstract);
+* the empty cases (tau = +inf, K = 0);
+* the page's 3x FLOP cap for a full-size gate and its lifting by LoPA.
+"""
+import itertools
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _np64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _silu_np(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def _tiny_weights(d, d_ff, n, seed, dtype="bf16", r=0):
+    gate = "both" if r else "dense"
+    w = workloads.ffn_weights(d, d_ff, dtype, seed=seed, gate=gate, r=r)
+    x = workloads.tokens(n, d, dtype, seed=seed)
+    return w, x
+
+
+# --------------------------------------------------------------------------
+# brute force
+
+def _exact(t):
+    return [[Fraction(float(v)) for v in row] for row in t.to(torch.float64).tolist()]
+
+
+@pytest.mark.parametrize("seed,d,d_ff,n", [(1, 3, 8, 2), (2, 5, 10, 2), (3, 8, 12, 1)])
+def test_threshold_set_and_y_by_brute_force(seed, d, d_ff, n):
+    w, x = _tiny_weights(d, d_ff, n, seed)
+    tau = 0.1234567
+    X, WG, WU, WD = _exact(x), _exact(w["w_gate"]), _exact(w["w_up"]), _exact(w["w_down"])
+    T = Fraction(tau)
+    res = oracle.forward(x, w, "dense", "threshold", tau=tau)
+    for t in range(n):
+        z = [sum(X[t][j] * WG[j][k] for j in range(d)) for k in range(d_ff)]
+        assert all(zk != T for zk in z)
+        best, best_mask = None, None
+        for mask in itertools.product((0, 1), repeat=d_ff):
+            s = sum((z[k] - T) for k in range(d_ff) if mask[k])
+            if best is None or s > best:
+                best, best_mask = s, mask
+        S = [k for k in range(d_ff) if best_mask[k]]
+        assert list(res.sets[t]) == S
+        u = [sum(X[t][j] * WU[j][k] for j in range(d)) for k in range(d_ff)]
+        for j in range(d):
+            terms = [(z[k] - T) * u[k] * WD[k][j] for k in S]
+            exact = sum(terms, Fraction(0))
+            scale = float(sum(abs(v) for v in terms)) + 1e-300
+            assert abs(res.y[t, j] - float(exact)) <= 1e-13 * scale
+
+
+@pytest.mark.parametrize("seed,d,d_ff,K", [(4, 4, 10, 3), (5, 6, 12, 5), (6, 3, 9, 8)])
+def test_topk_set_by_brute_force(seed, d, d_ff, K):
+    n = 2
+    w, x = _tiny_weights(d, d_ff, n, seed)
+    res = oracle.forward(x, w, "dense", "topk", k=K)
+    X, WG = _exact(x), _exact(w["w_gate"])
+    for t in range(n):
+        z = [float(sum(X[t][j] * WG[j][k] for j in range(d))) for k in range(d_ff)]
+        g = [zk / (1.0 + math.exp(-zk)) for zk in z]
+        best, best_set = None, None
+        for S in itertools.combinations(range(d_ff), K):   # lexicographic order
+            s = math.fsum(g[k] for k in S)
+            if best is None or s > best:
+                best, best_set = s, S
+        assert tuple(res.sets[t]) == best_set
+        for k in range(d_ff):
+            expect = g[k] if k in best_set else 0.0
+            assert res.g[t, k] == pytest.approx(expect, rel=1e-13, abs=1e-300)
+
+
+def test_topk_ties_go_to_lower_index():
+    z = np.array([[0.5, 2.0, 1.0, 2.0, 1.0, 1.0, -3.0]])
+    sets, g = oracle.select_topk(z, 4)
+    assert list(sets[0]) == [1, 2, 3, 4]
+    sets, _ = oracle.select_topk(z, 3)
+    assert list(sets[0]) == [1, 2, 3]
+
+
+def test_topk_ranks_by_silu_not_by_z():
+    # SiLU is not monotone below its minimum near z = -1.278: -6 outranks -1.3.
+    z = np.array([[-1.3, -6.0, 0.2]])
+    sets, _ = oracle.select_topk(z, 2)
+    assert list(sets[0]) == [1, 2]
+
+
+# --------------------------------------------------------------------------
+# special cases against an independent numpy product chain
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_topk_all_channels_is_dense_swiglu(dtype):
+    d, d_ff, n = 48, 80, 3
+    w, x = _tiny_weights(d, d_ff, n, 7, dtype)
+    res = oracle.forward(x, w, "dense", "topk", k=d_ff)
+    X, WG, WU, WD = (_np64(t) for t in (x, w["w_gate"], w["w_up"], w["w_down"]))
+    y_ref = (_silu_np(X @ WG) * (X @ WU)) @ WD
+    np.testing.assert_allclose(res.y, y_ref, rtol=1e-11, atol=1e-12 * np.abs(y_ref).max())
+    assert all(len(s) == d_ff for s in res.sets)
+
+
+def test_threshold_below_all_gates_is_affine_glu():
+    d, d_ff, n = 40, 72, 2
+    w, x = _tiny_weights(d, d_ff, n, 8)
+    tau = -50.0
+    res = oracle.forward(x, w, "dense", "threshold", tau=tau)
+    X, WG, WU, WD = (_np64(t) for t in (x, w["w_gate"], w["w_up"], w["w_down"]))
+    y_ref = ((X @ WG - tau) * (X @ WU)) @ WD
+    np.testing.assert_allclose(res.y, y_ref, rtol=1e-11, atol=1e-12 * np.abs(y_ref).max())
+
+
+def test_lopa_gate_equals_product_gate():
+    d, d_ff, r, n = 64, 96, 16, 3
+    w, x = _tiny_weights(d, d_ff, n, 9, r=r)
+    u, z = oracle.gate_lopa(x, w["A"], w["B"])
+    X, A, B = _np64(x), _np64(w["A"]), _np64(w["B"])
+    np.testing.assert_allclose(u, X @ A, rtol=1e-12, atol=1e-13)
+    zr = X @ (A @ B)
+    assert np.abs(z - zr).max() <= 1e-12 * np.abs(zr).max()
+
+
+def test_dense_gate_against_matmul():
+    d, d_ff, n = 33, 70, 4
+    w, x = _tiny_weights(d, d_ff, n, 10, "f32")
+    z = oracle.gate_dense(x, w["w_gate"])
+    np.testing.assert_allclose(z, _np64(x) @ _np64(w["w_gate"]), rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# invariants
+
+@pytest.mark.parametrize("select", ["threshold", "topk"])
+def test_sparse_equals_dense_bitwise(select):
+    wl = workloads.tiny()
+    w, x = wl.weights(), wl.x()
+    kw = dict(tau=wl.tau) if select == "threshold" else dict(k=wl.d_ff // 8)
+    sp = oracle.forward(x, w, "dense", select, **kw)
+    de = oracle.forward(x, w, "dense", select, dense=True, **kw)
+    assert np.array_equal(sp.y, de.y)      # == treats -0.0 and +0.0 as equal
+
+
+def test_empty_selection_gives_zero():
+    d, d_ff, n = 16, 24, 3
+    w, x = _tiny_weights(d, d_ff, n, 11)
+    for kw in (dict(select="threshold", tau=float("inf")), dict(select="topk", k=0)):
+        res = oracle.forward(x, w, "dense", **kw)
+        assert all(len(s) == 0 for s in res.sets)
+        assert not res.y.any()
+        assert not res.g.any()
+
+
+def test_gate_values_on_given_sets():
+    z = np.array([[0.3, 2.0, -1.0], [1.5, 0.0, 4.0]])
+    g = oracle.gate_values(z, [np.array([1]), np.array([0, 2])], "threshold", 1.0)
+    np.testing.assert_array_equal(g, [[0.0, 1.0, 0.0], [0.5, 0.0, 3.0]])
+    g = oracle.gate_values(z, [np.array([0]), np.array([])], "topk")
+    assert g[0, 0] == pytest.approx(0.3 / (1 + math.exp(-0.3)), rel=1e-15) and g.sum() == g[0, 0]
+
+
+# --------------------------------------------------------------------------
+# closed forms
+
+def _phi(v):
+    return 0.5 * math.erfc(-v / math.sqrt(2.0))
+
+
+@pytest.mark.parametrize("s", [0.5, 0.8, 0.9, 0.99])
+def test_active_count_matches_gaussian_closed_form(s):
+    d, d_ff, n = 256, 4096, 4
+    w, x = _tiny_weights(d, d_ff, n, 12, "f32")
+    tau = workloads.tau_for_sparsity(s)
+    res = oracle.forward(x, w, "dense", "threshold", tau=tau)
+    X = _np64(x)
+    var_w = float(_np64(w["w_gate"]).var())
+    for t in range(n):
+        sigma = math.sqrt(float(X[t] @ X[t]) * var_w)
+        p = 1.0 - _phi(tau / sigma)
+        m = len(res.sets[t])
+        assert abs(m - d_ff * p) <= 4.0 * math.sqrt(d_ff * p * (1 - p)) + 1, (t, m, d_ff * p)
+
+
+def test_lopa_active_count_matches_gaussian_closed_form():
+    d, d_ff, r, n = 512, 4096, 32, 3
+    w, x = _tiny_weights(d, d_ff, n, 13, "f32", r=r)
+    tau = workloads.tau_for_sparsity(0.9)
+    res = oracle.forward(x, w, "lopa", "threshold", tau=tau)
+    U = _np64(x) @ _np64(w["A"])
+    var_b = float(_np64(w["B"]).var())
+    for t in range(n):
+        sigma = math.sqrt(float(U[t] @ U[t]) * var_b)
+        p = 1.0 - _phi(tau / sigma)
+        m = len(res.sets[t])
+        assert abs(m - d_ff * p) <= 4.0 * math.sqrt(d_ff * p * (1 - p)) + 1
+
+
+def test_topk_count_is_exactly_k():
+    wl = workloads.moc_topk(n=3)
+    w = workloads.ffn_weights(256, 704, "bf16", seed=3)
+    x = workloads.tokens(3, 256, "bf16", seed=3)
+    res = oracle.forward(x, w, "dense", "topk", k=88)
+    for t in range(3):
+        S = res.sets[t]
+        assert len(S) == 88 and np.all(np.diff(S) > 0)
+        sil = _silu_np(res.z[t])
+        chosen = np.zeros(704, bool)
+        chosen[S] = True
+        assert sil[chosen].min() >= sil[~chosen].max()
+    assert wl.k == wl.d_ff // 8
+
+
+def _claims():
+    out = {}
+    with open(os.path.join(GOLDEN, "page_claims.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, value, pinned, _src = [p.strip() for p in line.split("|", 3)]
+            out[name] = (float(value), pinned == "yes")
+    return out
+
+
+def test_flop_ratio_closed_form_and_page_cap():
+    claims = _claims()
+    cap, pinned = claims["dense_gate_flop_cap"]
+    assert pinned
+    d, d_ff, n = 4096, 11008, 1
+    for m in (0, 1, 110, 1101, 5504, 11008):
+        rho = Fraction(m, n * d_ff)
+        ratio = Fraction(oracle.dense_flops(n, d, d_ff), oracle.flops(n, d, d_ff, m))
+        assert ratio == 3 / (1 + 2 * rho)
+        assert ratio <= cap
+    assert Fraction(oracle.dense_flops(n, d, d_ff), oracle.flops(n, d, d_ff, 0)) == cap
+    # LoPA r = 256 at 90 % sparsity: 3 d d_ff / (r (d + d_ff) + 2 rho d d_ff)
+    lifts, pinned = claims["lopa_lifts_cap"]
+    assert pinned and lifts == 1
+    m, r = 1101, 256
+    ratio = Fraction(oracle.dense_flops(n, d, d_ff), oracle.flops(n, d, d_ff, m, r=r))
+    assert ratio == Fraction(3 * d * d_ff, r * (d + d_ff) + 2 * m * d)
+    assert ratio > cap
+
+
+def test_byte_counter_matches_layout_arithmetic():
+    # the dense gate, two bf16 rows of 8 KB per union channel, x in and y out
+    assert oracle.bytes_moved(1, 4096, 11008, 1101, 2, 2) == \
+        4096 * 11008 * 2 + 2 * 1101 * 8192 + 2 * 8192
+    assert oracle.bytes_moved(1, 4096, 11008, 1101, 2, 2, r=256) == \
+        256 * (4096 + 11008) * 2 + 2 * 1101 * 8192 + 2 * 8192
+    assert oracle.dense_bytes(1, 4096, 11008, 2, 2) == 3 * 4096 * 11008 * 2 + 2 * 8192
+    assert oracle.union_size([np.array([1, 5]), np.array([5, 7])]) == 3
+
+
+def test_thread_count_does_not_change_results():
+    wl = workloads.tiny()
+    w, x = wl.weights(), wl.x()
+    n0 = oracle.num_threads()
+    try:
+        oracle.set_threads(1)
+        a = oracle.forward(x, w, "dense", "threshold", tau=wl.tau)
+        oracle.set_threads(max(2, n0))
+        b = oracle.forward(x, w, "dense", "threshold", tau=wl.tau)
+    finally:
+        oracle.set_threads(n0)
+    assert np.array_equal(a.y, b.y) and np.array_equal(a.z, b.z)
