@@ -1,0 +1,524 @@
+// C ABI of the activation-sparse gated FFN (declared in include/sffn.h).
+//
+// Host-side orchestration only: argument checks, the device workspace plan,
+// weight repacking, and the kernel sequence of one forward:
+//   threshold:  [LoPA x A] -> gate+select+up -> down
+//   top-K:      [LoPA x A] -> gate (z) -> top-K -> preselected up -> down
+// Every kernel is launched with programmatic dependent launch so its launch
+// latency overlaps the previous kernel's tail; each kernel waits on its
+// predecessor before touching shared buffers.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "sffn.h"
+
+using namespace sffn;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    const int code = e == cudaErrorMemoryAllocation ? SFFN_ERR_OOM : SFFN_ERR_CUDA;
+    return fail(code, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define SFFN_CUDA(call, what)                              \
+    do {                                                   \
+        cudaError_t e_ = (call);                           \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+struct DeviceGuard {
+    int prev = -1, dev;
+    cudaError_t err = cudaSuccess;
+    explicit DeviceGuard(int d) : dev(d) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) err = cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        if (prev >= 0 && prev != dev) cudaSetDevice(prev);
+    }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Plan {
+    int g1 = 0, cpb = 0, mw = 0;                          // gate grid
+    int lopa_rows = 0, lopa_cols = 0, lopa_splits = 0, lopa_groups = 0;
+    int down_slices = 0, down_chunks = 0, down_min_rows = 0, down_max_rows = 0;
+};
+
+}  // namespace
+
+struct sffn_ctx {
+    sffn_config cfg{};
+    int sms = 0;
+    size_t esz = 0;
+    void* wg = nullptr;
+    void* a = nullptr;
+    void* bcm = nullptr;
+    void* wup = nullptr;
+    void* wdn = nullptr;
+    bool has_dense = false, has_lopa = false, ready = false;
+    void* ws = nullptr;
+    float* zbuf = nullptr;
+    float* gbuf = nullptr;
+    uint8_t* sel = nullptr;
+    int* lst_idx = nullptr;
+    float* lst_h = nullptr;
+    uint32_t* lst_mask = nullptr;
+    int* seg_count = nullptr;
+    float* upart = nullptr;
+    float* u = nullptr;
+    float* dpart = nullptr;
+    unsigned* tickets = nullptr;
+    int* status = nullptr;
+    void* xdev = nullptr;
+    void* ydev = nullptr;
+    Plan plan;
+    int last_n = -1;
+    cudaStream_t last_stream = nullptr;
+    int last_launches = 0;
+    std::vector<cudaEvent_t> events;
+};
+
+namespace {
+
+constexpr size_t kGateSmemCap = 110 * 1024;   // keeps two gate CTAs per SM
+
+int pick_nt(int n) { return n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : 8; }
+
+int gate_nt(const sffn_ctx* h, int n, int gate_kind) {
+    int nt = pick_nt(n);
+    const int r = gate_kind == kGateLopa ? h->cfg.lopa_rank : 0;
+    while (nt > 1 &&
+           gate_smem_bytes(h->cfg.wdtype, nt, h->cfg.d, r, gate_kind, h->plan.cpb, h->plan.mw) > kGateSmemCap)
+        nt /= 2;
+    return nt;
+}
+
+int gate_rw(const sffn_ctx* h, int gate_kind) {
+    const int v = h->cfg.wdtype == SFFN_BF16 ? 8 : 4;
+    if (gate_kind == kGatePreselected) return 1;
+    const int cpr = (gate_kind == kGateLopa ? h->cfg.lopa_rank : h->cfg.d) / v;
+    return cpr <= 64 ? 4 : 1;
+}
+
+// Stage events are recorded as external event nodes under stream capture so
+// that a replayed graph still timestamps them.
+void record(sffn_ctx* h, int i, cudaStream_t s) {
+    if (i >= (int)h->events.size()) return;
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &st) == cudaSuccess && st == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(h->events[i], s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(h->events[i], s);
+}
+
+int check_select(const sffn_ctx* h, const sffn_select* sel) {
+    if (!sel) return fail(SFFN_ERR_INVALID_ARG, "sel is NULL");
+    if (sel->kind == SFFN_SELECT_THRESHOLD) {
+        if (std::isnan(sel->tau) || (std::isinf(sel->tau) && sel->tau < 0))
+            return fail(SFFN_ERR_INVALID_ARG, "threshold tau must be a number or +inf");
+    } else if (sel->kind == SFFN_SELECT_TOPK) {
+        if (sel->k < 0 || sel->k > h->cfg.d_ff)
+            return fail(SFFN_ERR_INVALID_ARG, "top-K k=%d outside [0, d_ff=%d]", sel->k, h->cfg.d_ff);
+    } else {
+        return fail(SFFN_ERR_INVALID_ARG, "unknown select kind %d", sel->kind);
+    }
+    return SFFN_OK;
+}
+
+int check_forward(const sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_select* sel,
+                  const void* out, bool device_ptrs) {
+    if (!h) return fail(SFFN_ERR_INVALID_ARG, "handle is NULL");
+    if (n < 0 || n > h->cfg.max_tokens)
+        return fail(SFFN_ERR_INVALID_ARG, "n_tokens=%d outside [0, max_tokens=%d]", n, h->cfg.max_tokens);
+    if (gate_mode != SFFN_GATE_DENSE && gate_mode != SFFN_GATE_LOPA)
+        return fail(SFFN_ERR_INVALID_ARG, "unknown gate mode %d", gate_mode);
+    const int rc = check_select(h, sel);
+    if (rc) return rc;
+    if (n > 0) {
+        if (!x || !out) return fail(SFFN_ERR_INVALID_ARG, "x or out is NULL");
+        if (device_ptrs && (!aligned16(x) || !aligned16(out)))
+            return fail(SFFN_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
+    }
+    if (!h->ready) return fail(SFFN_ERR_NOT_READY, "sffn_set_weights has not been called");
+    if (gate_mode == SFFN_GATE_DENSE && !h->has_dense)
+        return fail(SFFN_ERR_UNSUPPORTED, "dense gate requested but no W_gate was set");
+    if (gate_mode == SFFN_GATE_LOPA && !h->has_lopa)
+        return fail(SFFN_ERR_UNSUPPORTED, "LoPA gate requested but A and B were not set");
+    return SFFN_OK;
+}
+
+int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_select* sel, void* out,
+                cudaStream_t s, bool dense) {
+    const sffn_config& c = h->cfg;
+    const Plan& P = h->plan;
+    const bool lopa = gate_mode == SFFN_GATE_LOPA;
+    const int gk = lopa ? kGateLopa : kGateDense;
+    const bool pdl = true;
+    int launches = 0;
+    record(h, 0, s);
+
+    if (lopa) {
+        LopaUParams lp{};
+        lp.x = x; lp.a = h->a; lp.n = n; lp.d = c.d; lp.r = c.lopa_rank;
+        lp.rows_per_cta = P.lopa_rows; lp.cols_per_cta = P.lopa_cols;
+        lp.part = h->upart; lp.u = h->u; lp.tickets = h->tickets;
+        SFFN_CUDA(launch_lopa_u(c.wdtype, lp, pick_nt(n), dim3(P.lopa_splits, P.lopa_groups), s, pdl),
+                  "LoPA x*A launch");
+        record(h, ++launches, s);
+    }
+
+    GateParams gp{};
+    gp.x = x; gp.n = n; gp.d = c.d; gp.d_ff = c.d_ff; gp.r = c.lopa_rank;
+    gp.wg = h->wg; gp.bcm = h->bcm; gp.u = h->u; gp.wup = h->wup;
+    gp.force_all = dense ? 1 : 0;
+    gp.tau = sel->tau;
+    gp.zbuf = h->zbuf; gp.gbuf = h->gbuf; gp.sel = h->sel;
+    gp.cpb = P.cpb; gp.mw = P.mw;
+    gp.lst_idx = h->lst_idx; gp.lst_h = h->lst_h; gp.lst_mask = h->lst_mask; gp.seg_count = h->seg_count;
+
+    if (sel->kind == SFFN_SELECT_THRESHOLD) {
+        gp.out = kOutSelectUp;
+        const int nt = gate_nt(h, n, gk);
+        SFFN_CUDA(launch_gate(c.wdtype, gp, nt, gate_rw(h, gk), gk, P.g1,
+                              gate_smem_bytes(c.wdtype, nt, c.d, c.lopa_rank, gk, P.cpb, P.mw), s, pdl),
+                  "gate/select/up launch");
+        record(h, ++launches, s);
+    } else {
+        gp.out = kOutWriteZ;
+        int nt = gate_nt(h, n, gk);
+        SFFN_CUDA(launch_gate(c.wdtype, gp, nt, gate_rw(h, gk), gk, P.g1,
+                              gate_smem_bytes(c.wdtype, nt, c.d, c.lopa_rank, gk, P.cpb, P.mw), s, pdl),
+                  "gate launch");
+        record(h, ++launches, s);
+        TopkParams tp{};
+        tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
+        SFFN_CUDA(launch_topk(tp, s, pdl), "top-K launch");
+        record(h, ++launches, s);
+        gp.out = kOutSelectUp;
+        nt = gate_nt(h, n, kGatePreselected);
+        SFFN_CUDA(launch_gate(c.wdtype, gp, nt, 1, kGatePreselected, P.g1,
+                              gate_smem_bytes(c.wdtype, nt, c.d, 0, kGatePreselected, P.cpb, P.mw), s, pdl),
+                  "selected up launch");
+        record(h, ++launches, s);
+    }
+
+    DownParams dp{};
+    dp.wdn = h->wdn; dp.n = n; dp.d = c.d; dp.d_ff = c.d_ff;
+    dp.seg_count = h->seg_count; dp.g1 = P.g1; dp.cpb = P.cpb;
+    dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.part = h->dpart;
+    dp.tickets = h->tickets + P.lopa_groups; dp.y = out;
+    dp.chunks = P.down_chunks; dp.min_rows = P.down_min_rows; dp.max_rows = P.down_max_rows;
+    dp.status = h->status;
+    const int dnt = pick_nt(n);
+    SFFN_CUDA(launch_down(c.wdtype, dp, dnt, P.down_slices,
+                          down_smem_bytes(c.wdtype, dnt, P.g1, P.down_max_rows), s, pdl),
+              "down launch");
+    record(h, ++launches, s);
+
+    h->last_n = n;
+    h->last_stream = s;
+    h->last_launches = launches;
+    return SFFN_OK;
+}
+
+int forward_common(sffn_handle h, const void* x, int n, int gate_mode, const sffn_select* sel, void* out,
+                   void* stream, bool dense) {
+    int rc = check_forward(h, x, n, gate_mode, sel, out, true);
+    if (rc) return rc;
+    if (n == 0) return SFFN_OK;
+    DeviceGuard g(h->cfg.device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    return run_forward(h, x, n, gate_mode, sel, out, static_cast<cudaStream_t>(stream), dense);
+}
+
+void free_weights(sffn_ctx* h) {
+    for (void** p : {&h->wg, &h->a, &h->bcm, &h->wup, &h->wdn}) {
+        if (*p) cudaFree(*p);
+        *p = nullptr;
+    }
+    h->has_dense = h->has_lopa = h->ready = false;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sffn_strerror(int code) {
+    switch (code) {
+        case SFFN_OK: return "ok";
+        case SFFN_ERR_INVALID_ARG: return "invalid argument";
+        case SFFN_ERR_NOT_READY: return "weights not set";
+        case SFFN_ERR_UNSUPPORTED: return "unsupported mode for this handle";
+        case SFFN_ERR_CUDA: return "CUDA error";
+        case SFFN_ERR_OOM: return "out of device memory";
+        case SFFN_ERR_TIMEOUT: return "device wait timed out";
+        case SFFN_ERR_DEVICE_CHECK: return "a kernel's own bounds check failed";
+        default: return "unknown status";
+    }
+}
+
+const char* sffn_last_error(void) { return g_err; }
+
+int sffn_create(sffn_handle* out, const sffn_config* cfg) {
+    if (!out || !cfg) return fail(SFFN_ERR_INVALID_ARG, "out or cfg is NULL");
+    *out = nullptr;
+    const sffn_config c = *cfg;
+    if (c.d <= 0 || c.d % 8 || c.d_ff <= 0 || c.lopa_rank < 0 || c.lopa_rank % 8 ||
+        c.max_tokens < 1 || c.max_tokens > kMaxTokens || (c.wdtype != SFFN_BF16 && c.wdtype != SFFN_F32))
+        return fail(SFFN_ERR_INVALID_ARG,
+                    "bad config d=%d d_ff=%d r=%d max_tokens=%d wdtype=%d (d, r multiples of 8; "
+                    "1 <= max_tokens <= %d)", c.d, c.d_ff, c.lopa_rank, c.max_tokens, c.wdtype, kMaxTokens);
+    if ((long long)c.d * c.d_ff > (1LL << 31) - 1 || c.lopa_rank > 4096)
+        return fail(SFFN_ERR_INVALID_ARG, "shape too large");
+    int ndev = 0;
+    SFFN_CUDA(cudaGetDeviceCount(&ndev), "cudaGetDeviceCount");
+    if (c.device < 0 || c.device >= ndev) return fail(SFFN_ERR_INVALID_ARG, "no CUDA device %d", c.device);
+    DeviceGuard g(c.device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+
+    sffn_ctx* h = new (std::nothrow) sffn_ctx();
+    if (!h) return fail(SFFN_ERR_OOM, "host allocation failed");
+    h->cfg = c;
+    h->esz = c.wdtype == SFFN_BF16 ? 2 : 4;
+    cudaError_t e = cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, c.device);
+    if (e != cudaSuccess) { delete h; return cuda_fail(e, "device attribute"); }
+
+    Plan& P = h->plan;
+    const int target = 2 * h->sms;
+    P.cpb = (c.d_ff + target - 1) / target;
+    P.g1 = (c.d_ff + P.cpb - 1) / P.cpb;
+    P.mw = (c.max_tokens + 31) / 32;
+    if (c.lopa_rank > 0) {
+        P.lopa_rows = 128;
+        P.lopa_cols = 64;
+        P.lopa_splits = (c.d + P.lopa_rows - 1) / P.lopa_rows;
+        P.lopa_groups = (c.lopa_rank + P.lopa_cols - 1) / P.lopa_cols;
+    }
+    P.down_slices = (c.d + down_slice_cols(c.wdtype) - 1) / down_slice_cols(c.wdtype);
+    P.down_chunks = target / P.down_slices > 1 ? target / P.down_slices : 1;
+    P.down_min_rows = 16;
+    P.down_max_rows = down_max_rows(c.d_ff, P.down_chunks, P.down_min_rows);
+
+    const size_t T = c.max_tokens, F = c.d_ff, D = c.d, R = c.lopa_rank;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t o = off; off = round_up(off + bytes, 256); return o; };
+    const size_t o_z = take(T * F * 4), o_g = take(T * F * 4), o_sel = take(T * F);
+    const size_t o_idx = take(F * 4), o_h = take(F * T * 4), o_mask = take(F * P.mw * 4);
+    const size_t o_seg = take((size_t)P.g1 * 4);
+    const size_t o_up = take((size_t)P.lopa_splits * T * R * 4), o_u = take(T * R * 4);
+    const size_t o_dp = take((size_t)P.down_chunks * T * D * 4);
+    const size_t o_tk = take((size_t)(P.lopa_groups + P.down_slices) * 4), o_st = take(4);
+    const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
+    e = cudaMalloc(&h->ws, off);
+    if (e != cudaSuccess) { delete h; return cuda_fail(e, "workspace allocation"); }
+    char* b = static_cast<char*>(h->ws);
+    h->zbuf = reinterpret_cast<float*>(b + o_z);
+    h->gbuf = reinterpret_cast<float*>(b + o_g);
+    h->sel = reinterpret_cast<uint8_t*>(b + o_sel);
+    h->lst_idx = reinterpret_cast<int*>(b + o_idx);
+    h->lst_h = reinterpret_cast<float*>(b + o_h);
+    h->lst_mask = reinterpret_cast<uint32_t*>(b + o_mask);
+    h->seg_count = reinterpret_cast<int*>(b + o_seg);
+    h->upart = reinterpret_cast<float*>(b + o_up);
+    h->u = reinterpret_cast<float*>(b + o_u);
+    h->dpart = reinterpret_cast<float*>(b + o_dp);
+    h->tickets = reinterpret_cast<unsigned*>(b + o_tk);
+    h->status = reinterpret_cast<int*>(b + o_st);
+    h->xdev = b + o_x;
+    h->ydev = b + o_y;
+    e = cudaMemset(h->ws, 0, off);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(e, "workspace init"); }
+    *out = h;
+    return SFFN_OK;
+}
+
+int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const void* B, const void* w_up,
+                     const void* w_down, int src_is_device, void* stream) {
+    if (!h) return fail(SFFN_ERR_INVALID_ARG, "handle is NULL");
+    const sffn_config& c = h->cfg;
+    if (!w_up || !w_down) return fail(SFFN_ERR_INVALID_ARG, "w_up and w_down are required");
+    if (!w_gate && !(A && B)) return fail(SFFN_ERR_INVALID_ARG, "need w_gate or both A and B");
+    if ((A != nullptr) != (B != nullptr)) return fail(SFFN_ERR_INVALID_ARG, "A and B go together");
+    if (A && c.lopa_rank <= 0) return fail(SFFN_ERR_INVALID_ARG, "A and B need lopa_rank > 0");
+    if (src_is_device)
+        for (const void* p : {w_gate, A, B, w_up, w_down})
+            if (p && !aligned16(p)) return fail(SFFN_ERR_INVALID_ARG, "device weights must be 16-byte aligned");
+    DeviceGuard g(c.device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SFFN_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    free_weights(h);
+
+    const size_t big = (size_t)c.d * c.d_ff * h->esz;
+    const size_t r_d = (size_t)c.lopa_rank * c.d * h->esz, r_ff = (size_t)c.lopa_rank * c.d_ff * h->esz;
+    void* staging = nullptr;
+    int rc = SFFN_OK;
+    auto stage = [&](const void* src, size_t bytes) -> const void* {
+        if (src_is_device) return src;
+        if (cudaMemcpyAsync(staging, src, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return nullptr;
+        return staging;
+    };
+    auto alloc = [&](void** p, size_t bytes) { return cudaMalloc(p, bytes); };
+    cudaError_t e = cudaSuccess;
+    do {
+        if (!src_is_device && (e = alloc(&staging, big > r_ff ? big : r_ff)) != cudaSuccess) break;
+        if ((e = alloc(&h->wup, big)) != cudaSuccess) break;
+        if ((e = alloc(&h->wdn, big)) != cudaSuccess) break;
+        const void* src = stage(w_up, big);
+        if (!src) { e = cudaGetLastError(); break; }
+        if ((e = launch_transpose(c.wdtype, src, h->wup, c.d, c.d_ff, s)) != cudaSuccess) break;
+        if ((e = cudaStreamSynchronize(s)) != cudaSuccess) break;
+        if ((e = cudaMemcpyAsync(h->wdn, w_down, big, src_is_device ? cudaMemcpyDeviceToDevice
+                                                                     : cudaMemcpyHostToDevice, s)) != cudaSuccess)
+            break;
+        if (w_gate) {
+            if ((e = alloc(&h->wg, big)) != cudaSuccess) break;
+            src = stage(w_gate, big);
+            if (!src) { e = cudaGetLastError(); break; }
+            if ((e = launch_transpose(c.wdtype, src, h->wg, c.d, c.d_ff, s)) != cudaSuccess) break;
+            if ((e = cudaStreamSynchronize(s)) != cudaSuccess) break;
+        }
+        if (A) {
+            if ((e = alloc(&h->a, r_d)) != cudaSuccess) break;
+            if ((e = alloc(&h->bcm, r_ff)) != cudaSuccess) break;
+            if ((e = cudaMemcpyAsync(h->a, A, r_d, src_is_device ? cudaMemcpyDeviceToDevice
+                                                                 : cudaMemcpyHostToDevice, s)) != cudaSuccess)
+                break;
+            src = stage(B, r_ff);
+            if (!src) { e = cudaGetLastError(); break; }
+            if ((e = launch_transpose(c.wdtype, src, h->bcm, c.lopa_rank, c.d_ff, s)) != cudaSuccess) break;
+        }
+        e = cudaStreamSynchronize(s);
+    } while (0);
+    if (staging) cudaFree(staging);
+    if (e != cudaSuccess) {
+        rc = cuda_fail(e, "sffn_set_weights");
+        free_weights(h);
+        return rc;
+    }
+    h->has_dense = w_gate != nullptr;
+    h->has_lopa = A != nullptr;
+    h->ready = true;
+    return SFFN_OK;
+}
+
+int sffn_forward(sffn_handle h, const void* x, int n_tokens, int gate_mode, const sffn_select* sel, void* out,
+                 void* stream) {
+    return forward_common(h, x, n_tokens, gate_mode, sel, out, stream, false);
+}
+
+int sffn_forward_dense(sffn_handle h, const void* x, int n_tokens, int gate_mode, const sffn_select* sel,
+                       void* out, void* stream) {
+    return forward_common(h, x, n_tokens, gate_mode, sel, out, stream, true);
+}
+
+int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_mode, const sffn_select* sel,
+                      void* out_host, void* stream) {
+    int rc = check_forward(h, x_host, n_tokens, gate_mode, sel, out_host, false);
+    if (rc) return rc;
+    if (n_tokens == 0) return SFFN_OK;
+    DeviceGuard g(h->cfg.device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)n_tokens * h->cfg.d * h->esz;
+    SFFN_CUDA(cudaMemcpyAsync(h->xdev, x_host, bytes, cudaMemcpyHostToDevice, s), "x host-to-device copy");
+    rc = run_forward(h, h->xdev, n_tokens, gate_mode, sel, h->ydev, s, false);
+    if (rc) return rc;
+    SFFN_CUDA(cudaMemcpyAsync(out_host, h->ydev, bytes, cudaMemcpyDeviceToHost, s), "y device-to-host copy");
+    SFFN_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    return SFFN_OK;
+}
+
+int sffn_check_status(sffn_handle h) {
+    if (!h) return fail(SFFN_ERR_INVALID_ARG, "handle is NULL");
+    DeviceGuard g(h->cfg.device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    SFFN_CUDA(cudaDeviceSynchronize(), "device synchronize");
+    int st = 0;
+    SFFN_CUDA(cudaMemcpy(&st, h->status, sizeof st, cudaMemcpyDeviceToHost), "status read");
+    if (st) return fail(SFFN_ERR_DEVICE_CHECK, "device status word 0x%x", st);
+    return SFFN_OK;
+}
+
+int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union_size) {
+    if (!h || !idx || !counts) return fail(SFFN_ERR_INVALID_ARG, "handle, idx or counts is NULL");
+    if (h->last_n < 0) return fail(SFFN_ERR_NOT_READY, "no forward has run");
+    DeviceGuard g(h->cfg.device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    SFFN_CUDA(cudaStreamSynchronize(h->last_stream), "stream synchronize");
+    int rc = sffn_check_status(h);
+    if (rc) return rc;
+    const Plan& P = h->plan;
+    const int n = h->last_n, F = h->cfg.d_ff;
+    std::vector<int> seg(P.g1), lidx(F);
+    std::vector<uint32_t> mask((size_t)F * P.mw);
+    SFFN_CUDA(cudaMemcpy(seg.data(), h->seg_count, seg.size() * 4, cudaMemcpyDeviceToHost), "list copy");
+    SFFN_CUDA(cudaMemcpy(lidx.data(), h->lst_idx, lidx.size() * 4, cudaMemcpyDeviceToHost), "list copy");
+    SFFN_CUDA(cudaMemcpy(mask.data(), h->lst_mask, mask.size() * 4, cudaMemcpyDeviceToHost), "list copy");
+    for (int t = 0; t < n; ++t) counts[t] = 0;
+    int uni = 0;
+    for (int b = 0; b < P.g1; ++b) {
+        if (seg[b] < 0 || seg[b] > P.cpb || (long long)b * P.cpb + seg[b] > F)
+            return fail(SFFN_ERR_DEVICE_CHECK, "segment %d count %d", b, seg[b]);
+        for (int i = 0; i < seg[b]; ++i) {
+            const int k = lidx[(size_t)b * P.cpb + i];
+            if (k < b * P.cpb || k >= F) return fail(SFFN_ERR_DEVICE_CHECK, "listed channel %d out of range", k);
+            bool any = false;
+            for (int t = 0; t < n; ++t)
+                if ((mask[(size_t)k * P.mw + (t >> 5)] >> (t & 31)) & 1u) {
+                    idx[(size_t)t * F + counts[t]++] = k;
+                    any = true;
+                }
+            uni += any;
+        }
+    }
+    if (union_size) *union_size = uni;
+    return SFFN_OK;
+}
+
+int sffn_set_stage_events(sffn_handle h, void* const* events, int n_events) {
+    if (!h || n_events < 0 || (n_events > 0 && !events)) return fail(SFFN_ERR_INVALID_ARG, "bad events");
+    h->events.clear();
+    for (int i = 0; i < n_events; ++i) h->events.push_back(static_cast<cudaEvent_t>(events[i]));
+    return SFFN_OK;
+}
+
+int sffn_last_launches(sffn_handle h, int32_t* launches) {
+    if (!h || !launches) return fail(SFFN_ERR_INVALID_ARG, "handle or launches is NULL");
+    *launches = h->last_launches;
+    return SFFN_OK;
+}
+
+int sffn_destroy(sffn_handle h) {
+    if (!h) return SFFN_OK;
+    {
+        DeviceGuard g(h->cfg.device);
+        free_weights(h);
+        if (h->ws) cudaFree(h->ws);
+    }
+    delete h;
+    return SFFN_OK;
+}
+
+}  // extern "C"

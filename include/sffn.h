@@ -1,0 +1,152 @@
+/*
+ * sffn -- activation-sparse gated FFN inference on one B200 (sm_100a).
+ *
+ * Computes, for n tokens x (n x d),
+ *
+ *     z = x W_gate                       (dense gate, d x d_ff)
+ *       or  z = (x A) B                  (LoPA low-rank gate, A d x r, B r x d_ff)
+ *     S_t = { k : z[t,k] > tau }         threshold select, g = z - tau on S_t
+ *       or  the K largest SiLU(z[t,k])   per-token top-K select, g = SiLU(z) on S_t
+ *     y[t,:] = sum_{k in S_t} g[t,k] <x[t,:], W_up[:,k]> W_down[k,:]
+ *
+ * "Model Casting and Low-Parameter Gating: Towards More Sparsely Activated
+ * FFNs" (abstract): compute the gating matrix's output first and, because its
+ * activation is highly sparse, skip the two other matrices for the inactive
+ * channels; LoPA gives the gate fewer parameters and FLOPs than the other two
+ * matrices.  "Mixture-of-Channels" (sections "Dentro il mixture", "Dentro
+ * MoC"): keep per token only the top-K channels ranked by the SwiGLU gate and
+ * load only those channels' weight rows.
+ *
+ * Conventions for every entry point:
+ *  - Return 0 (SFFN_OK) or a positive sffn_status code; nothing aborts.
+ *  - A `stream` argument is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  Calls that take a stream are asynchronous on it unless
+ *    stated otherwise.
+ *  - Device pointers must be 16-byte aligned and on the handle's device.
+ *  - A handle is not thread-safe: one host thread at a time, and forwards on
+ *    one handle must be ordered (same stream, or the caller orders them),
+ *    because they share the handle's workspace.
+ */
+#ifndef SFFN_H
+#define SFFN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sffn_ctx* sffn_handle;
+
+typedef enum {
+    SFFN_OK = 0,
+    SFFN_ERR_INVALID_ARG = 1,  /* NULL or misaligned pointer, bad size, NaN tau, ... */
+    SFFN_ERR_NOT_READY = 2,    /* forward before sffn_set_weights */
+    SFFN_ERR_UNSUPPORTED = 3,  /* e.g. LoPA forward on a handle without A and B */
+    SFFN_ERR_CUDA = 4,         /* a CUDA runtime call or a launch failed */
+    SFFN_ERR_OOM = 5,          /* device allocation failed */
+    SFFN_ERR_TIMEOUT = 6,      /* reserved for bounded device-side waits */
+    SFFN_ERR_DEVICE_CHECK = 7  /* a kernel's own bounds check failed (sticky) */
+} sffn_status;
+
+typedef enum { SFFN_BF16 = 0, SFFN_F32 = 1 } sffn_dtype;
+typedef enum { SFFN_GATE_DENSE = 0, SFFN_GATE_LOPA = 1 } sffn_gate_mode;
+typedef enum { SFFN_SELECT_THRESHOLD = 0, SFFN_SELECT_TOPK = 1 } sffn_select_kind;
+
+/* Model shape.  d and lopa_rank must be multiples of 8 (16-byte weight rows);
+ * lopa_rank = 0 means no LoPA gate; 1 <= max_tokens <= 1024; wdtype is the
+ * storage type of weights, x and y (bf16, or fp32 for small exact checks);
+ * device is the CUDA ordinal. */
+typedef struct {
+    int32_t d;
+    int32_t d_ff;
+    int32_t lopa_rank;
+    int32_t max_tokens;
+    int32_t wdtype;      /* sffn_dtype */
+    int32_t device;
+} sffn_config;
+
+/* Channel selection.  THRESHOLD: active iff z > tau, activation z - tau (a
+ * shifted ReLU); tau = +inf selects nothing, NaN or -inf is rejected.
+ * TOPK: per token the k channels with the largest SiLU(z) (ties to the lower
+ * channel index), activation SiLU(z); 0 <= k <= d_ff. */
+typedef struct {
+    int32_t kind;        /* sffn_select_kind */
+    float tau;
+    int32_t k;
+} sffn_select;
+
+/* Allocate a handle and its device workspace, sized for cfg->max_tokens.
+ * The library owns all device memory it allocates; sffn_destroy frees it.
+ * Errors: INVALID_ARG (bad shape), CUDA (bad device), OOM. */
+int sffn_create(sffn_handle* out, const sffn_config* cfg);
+
+/* Copy the weights in (host or device memory, src_is_device says which) and
+ * repack them channel-major into library-owned buffers, so that channel k of
+ * W_gate, W_up and B, and row k of W_down, are each one contiguous row.
+ * Inputs are row-major in the handle's wdtype:
+ *   w_gate d x d_ff,  A d x r,  B r x d_ff,  w_up d x d_ff,  w_down d_ff x d.
+ * w_gate may be NULL when A and B are given and vice versa (not all three
+ * NULL); A and B need lopa_rank > 0.  The caller keeps ownership of its
+ * buffers.  Synchronises `stream` before returning.
+ * Errors: INVALID_ARG, CUDA, OOM. */
+int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const void* B,
+                     const void* w_up, const void* w_down, int src_is_device, void* stream);
+
+/* Sparse forward.  x: n_tokens x d device buffer, out: n_tokens x d device
+ * buffer, both in wdtype and caller-owned.  gate_mode: sffn_gate_mode.
+ * Asynchronous on `stream`, no host synchronisation; n_tokens = 0 is a no-op.
+ * The output is deterministic: the same inputs give bitwise the same y.
+ * Errors: INVALID_ARG, NOT_READY, UNSUPPORTED, CUDA. */
+int sffn_forward(sffn_handle h, const void* x, int n_tokens, int gate_mode,
+                 const sffn_select* sel, void* out, void* stream);
+
+/* The same library's dense FFN: every channel's W_gate, W_up and W_down row is
+ * read and multiplied; the activation (and top-K mask) is the same, so y
+ * equals the sparse forward's up to rounding.  Same arguments and errors. */
+int sffn_forward_dense(sffn_handle h, const void* x, int n_tokens, int gate_mode,
+                       const sffn_select* sel, void* out, void* stream);
+
+/* sffn_forward with HOST buffers: copies x_host to the device, runs the
+ * forward and copies the result into out_host, all on `stream`, then
+ * synchronises it.  Pinned host memory gives asynchronous copies.
+ * Errors: as sffn_forward. */
+int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_mode,
+                      const sffn_select* sel, void* out_host, void* stream);
+
+/* The last forward's active channels per token, for checking: idx (host,
+ * n_tokens x d_ff int32) receives token t's ascending channel list at row t,
+ * counts (host, n_tokens) its length, *union_size (host, may be NULL) the
+ * number of distinct channels over all tokens.  Synchronises the last
+ * forward's stream.  Errors: INVALID_ARG, NOT_READY (no forward yet), CUDA. */
+int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union_size);
+
+/* Record timing events around each kernel of later forwards (profiling):
+ * events[0] before the first launch and events[i] after launch i; at most
+ * n_events events are recorded (cudaEvent_t passed as void*, created by the
+ * caller and kept alive while set).  n_events = 0 switches recording off.
+ * sffn_last_launches stores in *launches the number of kernels the last
+ * forward launched.  Errors: INVALID_ARG. */
+int sffn_set_stage_events(sffn_handle h, void* const* events, int n_events);
+int sffn_last_launches(sffn_handle h, int32_t* launches);
+
+/* Synchronise the device and read the handle's sticky device status word,
+ * which kernels set when one of their own bounds checks fails (they then skip
+ * the access instead of faulting).  Returns SFFN_OK or SFFN_ERR_DEVICE_CHECK
+ * (the word stays set); also INVALID_ARG, CUDA. */
+int sffn_check_status(sffn_handle h);
+
+/* Free the handle and everything it owns.  NULL is accepted. */
+int sffn_destroy(sffn_handle h);
+
+/* Static description of a status code (never NULL). */
+const char* sffn_strerror(int code);
+
+/* Detail of the calling thread's most recent failure (never NULL; "" if none). */
+const char* sffn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFFN_H */

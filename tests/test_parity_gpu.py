@@ -1,0 +1,269 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on the pages' workload
+shapes (seeded synthetic stand-ins), small ragged shapes and edge cases."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import EXEMPT, YTOL, assert_sets, assert_y, check_forward, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sffn(cuda_device):
+    from activation_sparse_gated_gemv_b200 import build
+    build.build()
+    import activation_sparse_gated_gemv_b200 as m
+    return m
+
+
+def _ffn(sffn, wl, max_tokens=None, weights=None, device_src=False):
+    w = weights if weights is not None else wl.weights()
+    ffn = sffn.SparseFFN(wl.d, wl.d_ff, wl.r, max_tokens or wl.n, wl.dtype)
+    if device_src:
+        ffn.set_weights(**{k: v.cuda() for k, v in w.items()})
+    else:
+        ffn.set_weights(**w)
+    return ffn, w
+
+
+# --------------------------------------------------------------------------
+# the pages' workload shapes
+
+def test_tiny_relu_fp32(sffn):
+    wl = workloads.tiny()
+    ffn, w = _ffn(sffn, wl)
+    x = wl.x()
+    y, sets, union = check_forward(ffn, w, x, "dense", "threshold", tau=wl.tau)
+    # fp32 weights and accumulation: far inside the bf16 bar
+    ref = oracle.forward_on_sets(x, w, "dense", "threshold", sets, tau=wl.tau)
+    assert_y(to_np(y), ref, 1e-4, "fp32")
+    assert union == oracle.union_size(sets)
+    ffn.close()
+
+
+def test_llama7b_decode_dense_gate_90(sffn):
+    wl = workloads.llama7b_decode(0.9)
+    ffn, w = _ffn(sffn, wl)
+    x = wl.x()
+    _, sets, _ = check_forward(ffn, w, x, "dense", "threshold", tau=wl.tau)
+    frac = len(sets[0]) / wl.d_ff
+    assert 0.05 < frac < 0.15
+    ffn.close()
+
+
+@pytest.fixture(scope="module")
+def lopa7b_model(sffn):
+    wl = workloads.lopa7b(0.9)
+    w = workloads.ffn_weights(wl.d, wl.d_ff, wl.dtype, seed=wl.seed, gate="both", r=wl.r)
+    ffn = sffn.SparseFFN(wl.d, wl.d_ff, wl.r, 8, wl.dtype)
+    ffn.set_weights(**w)
+    yield wl, ffn, w
+    ffn.close()
+
+
+@pytest.mark.parametrize("sparsity", workloads.LOPA_SPARSITIES)
+def test_lopa7b_sweep(lopa7b_model, sparsity):
+    wl, ffn, w = lopa7b_model
+    tau = workloads.tau_for_sparsity(sparsity)
+    x = wl.x()
+    _, sets, _ = check_forward(ffn, w, x, "lopa", "threshold", tau=tau)
+    assert abs(len(sets[0]) / wl.d_ff - (1 - sparsity)) < 0.05
+
+
+def test_lopa7b_dense_gate_on_same_handle(lopa7b_model):
+    wl, ffn, w = lopa7b_model
+    check_forward(ffn, w, wl.x(n=3, tag="b"), "dense", "threshold", tau=wl.tau)
+
+
+def test_moc_topk_16_tokens(sffn):
+    wl = workloads.moc_topk()
+    ffn, w = _ffn(sffn, wl)
+    x = wl.x()
+    _, sets, union = check_forward(ffn, w, x, "dense", "topk", k=wl.k)
+    assert all(len(s) == wl.k for s in sets)
+    assert union == oracle.union_size(sets)
+    ffn.close()
+
+
+@pytest.fixture(scope="module")
+def llama70b_model(sffn):
+    wl = workloads.llama70b(64, "dense", 0.9)
+    w = workloads.ffn_weights(wl.d, wl.d_ff, wl.dtype, seed=wl.seed, gate="both", r=512)
+    ffn = sffn.SparseFFN(wl.d, wl.d_ff, 512, 64, wl.dtype)
+    ffn.set_weights(**w)
+    yield wl, ffn, w
+    ffn.close()
+
+
+@pytest.mark.parametrize("gate", ["dense", "lopa"])
+@pytest.mark.parametrize("n", workloads.SWEEP_70B_BATCHES)
+def test_llama70b_batches(llama70b_model, gate, n):
+    wl, ffn, w = llama70b_model
+    x = wl.x(n=n)
+    tokens = range(n) if n <= 4 else [0, n // 2, n - 1]       # oracle on sampled tokens
+    _, sets, union = check_forward(ffn, w, x, gate, "threshold", tau=wl.tau, tokens=tokens)
+    assert union == len(set(np.concatenate(sets).tolist()))
+
+
+@pytest.mark.parametrize("sparsity", workloads.SWEEP_70B_SPARSITIES)
+def test_llama70b_sparsity_sweep_lopa(llama70b_model, sparsity):
+    wl, ffn, w = llama70b_model
+    check_forward(ffn, w, wl.x(n=1, tag="s"), "lopa", "threshold", tau=workloads.tau_for_sparsity(sparsity))
+
+
+# --------------------------------------------------------------------------
+# small ragged shapes: several gate CTAs, ragged tails, token tiles
+
+SMALL = [
+    # d, d_ff, r, n, dtype, gate, select
+    (64, 1000, 0, 1, "bf16", "dense", "threshold"),
+    (64, 777, 0, 3, "f32", "dense", "threshold"),
+    (136, 4100, 0, 5, "bf16", "dense", "threshold"),
+    (136, 4100, 16, 5, "bf16", "lopa", "threshold"),
+    (256, 2048, 24, 17, "bf16", "lopa", "threshold"),
+    (512, 3000, 0, 9, "f32", "dense", "topk"),
+    (64, 1000, 8, 2, "bf16", "lopa", "topk"),
+    (1032, 1536, 0, 4, "bf16", "dense", "topk"),
+    (8, 300, 8, 1, "f32", "lopa", "threshold"),
+    (64, 256, 0, 1024, "bf16", "dense", "threshold"),    # the largest token count
+]
+
+
+@pytest.mark.parametrize("d,d_ff,r,n,dtype,gate,select", SMALL)
+def test_small_ragged(sffn, d, d_ff, r, n, dtype, gate, select):
+    w = workloads.ffn_weights(d, d_ff, dtype, seed=d + d_ff + n, gate="both" if r else "dense", r=r)
+    x = workloads.tokens(n, d, dtype, seed=d_ff)
+    ffn = sffn.SparseFFN(d, d_ff, r, n, dtype)
+    ffn.set_weights(**w)
+    tau = workloads.tau_for_sparsity(0.85)
+    k = max(1, d_ff // 8)
+    tokens = None if n <= 32 else [0, 1, 511, 1023]
+    check_forward(ffn, w, x, gate, select, tau=tau, k=k, tokens=tokens)
+    ffn.close()
+
+
+@pytest.mark.parametrize("select", ["threshold", "topk"])
+@pytest.mark.parametrize("gate", ["dense", "lopa"])
+def test_dense_path_matches_oracle_and_sparse(sffn, gate, select):
+    d, d_ff, r, n = 128, 1500, 16, 3
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=5, gate="both", r=r)
+    x = workloads.tokens(n, d, "bf16", seed=5)
+    ffn = sffn.SparseFFN(d, d_ff, r, n, "bf16")
+    ffn.set_weights(**w)
+    tau, k = workloads.tau_for_sparsity(0.9), d_ff // 8
+    yd, _, union = check_forward(ffn, w, x, gate, select, tau=tau, k=k, dense=True)
+    ys, _, _ = check_forward(ffn, w, x, gate, select, tau=tau, k=k)
+    assert_y(to_np(yd), to_np(ys), 1e-2, "dense vs sparse")
+    ffn.close()
+
+
+# --------------------------------------------------------------------------
+# edge cases
+
+def _small(sffn, n=4, r=8, dtype="bf16", d=64, d_ff=500):
+    w = workloads.ffn_weights(d, d_ff, dtype, seed=77, gate="both", r=r)
+    ffn = sffn.SparseFFN(d, d_ff, r, max(n, 1), dtype)
+    ffn.set_weights(**w)
+    return ffn, w, workloads.tokens(n, d, dtype, seed=78)
+
+
+def test_tau_inf_and_k_zero_give_zero(sffn):
+    ffn, w, x = _small(sffn)
+    for gate in ("dense", "lopa"):
+        y = ffn.forward(x.cuda(), gate=gate, select="threshold", tau=math.inf)
+        assert not to_np(y).any()
+        sets, union = ffn.active(4)
+        assert union == 0 and all(len(s) == 0 for s in sets)
+        y = ffn.forward(x.cuda(), gate=gate, select="topk", k=0)
+        assert not to_np(y).any()
+    ffn.close()
+
+
+def test_k_equals_d_ff_is_dense_swiglu(sffn):
+    ffn, w, x = _small(sffn, d_ff=300)
+    y = ffn.forward(x.cuda(), gate="dense", select="topk", k=300)
+    X, WG, WU, WD = (t.to(torch.float64).numpy() for t in (x, w["w_gate"], w["w_up"], w["w_down"]))
+    z = X @ WG
+    ref = (z / (1 + np.exp(-z)) * (X @ WU)) @ WD
+    assert_y(to_np(y), ref, YTOL, "K = d_ff")
+    ffn.close()
+
+
+def test_all_channels_active(sffn):
+    ffn, w, x = _small(sffn)
+    check_forward(ffn, w, x, "dense", "threshold", tau=-40.0)
+    sets, union = ffn.active(4)
+    assert union == 500
+    ffn.close()
+
+
+def test_zero_tokens_is_a_noop(sffn):
+    ffn, w, _ = _small(sffn)
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    y = ffn.forward(x)
+    assert y.shape == (0, 64)
+    ffn.close()
+
+
+def test_deterministic_bitwise(sffn):
+    wl = workloads.moc_topk(n=5)
+    ffn, w = _ffn(sffn, wl)
+    x = wl.x().cuda()
+    a = ffn.forward(x, select="topk", k=wl.k).clone()
+    b = ffn.forward(x, select="topk", k=wl.k).clone()
+    assert torch.equal(a, b)
+    tau = workloads.tau_for_sparsity(0.9)
+    a = ffn.forward(x, select="threshold", tau=tau).clone()
+    b = ffn.forward(x, select="threshold", tau=tau).clone()
+    assert torch.equal(a, b)
+    ffn.close()
+
+
+def test_forward_host_matches_device_forward(sffn):
+    ffn, w, x = _small(sffn)
+    tau = workloads.tau_for_sparsity(0.8)
+    yd = ffn.forward(x.cuda(), gate="lopa", tau=tau).cpu()
+    yh = ffn.forward_host(x.pin_memory(), gate="lopa", tau=tau)
+    assert torch.equal(yd, yh)
+    ffn.close()
+
+
+def test_device_source_weights(sffn):
+    wl = workloads.tiny()
+    ffn, w = _ffn(sffn, wl, device_src=True)
+    check_forward(ffn, w, wl.x(), "dense", "threshold", tau=wl.tau)
+    ffn.close()
+
+
+def test_errors(sffn):
+    import ctypes
+    ffn = sffn.SparseFFN(64, 128, 0, 2, "bf16")
+    x = torch.zeros((2, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sffn.SFFNError) as e:
+        ffn.forward(x)
+    assert e.value.code == sffn.SFFN_ERR_NOT_READY
+    w = workloads.ffn_weights(64, 128, "bf16", seed=1)
+    ffn.set_weights(**w)
+    with pytest.raises(sffn.SFFNError) as e:
+        ffn.forward(x, gate="lopa")
+    assert e.value.code == sffn.SFFN_ERR_UNSUPPORTED
+    for kw in (dict(select="threshold", tau=float("nan")), dict(select="threshold", tau=-math.inf),
+               dict(select="topk", k=-1), dict(select="topk", k=129)):
+        with pytest.raises(sffn.SFFNError) as e:
+            ffn.forward(x, **kw)
+        assert e.value.code == sffn.SFFN_ERR_INVALID_ARG
+    with pytest.raises(sffn.SFFNError) as e:
+        ffn.forward(torch.zeros((3, 64), dtype=torch.bfloat16, device="cuda"))
+    assert e.value.code == sffn.SFFN_ERR_INVALID_ARG
+    # misaligned device pointer
+    buf = torch.zeros(2 * 64 + 1, dtype=torch.bfloat16, device="cuda")
+    sel = sffn.make_select("threshold", 1.0)
+    out = torch.zeros((2, 64), dtype=torch.bfloat16, device="cuda")
+    rc = sffn.sffn_forward(ffn.handle, buf.data_ptr() + 2, 2, 0, ctypes.byref(sel), out.data_ptr(), None)
+    assert rc == sffn.SFFN_ERR_INVALID_ARG
+    ffn.close()
