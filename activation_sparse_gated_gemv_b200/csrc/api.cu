@@ -60,8 +60,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Plan {
     int g1 = 0, cpb = 0, mw = 0;                          // gate grid
-    int lopa_rows = 0, lopa_cols = 0, lopa_splits = 0, lopa_groups = 0;
-    int down_slices = 0, down_chunks = 0, down_min_rows = 0, down_max_rows = 0;
+    int down_slices = 0, down_chunks = 0;
 };
 
 }  // namespace
@@ -84,7 +83,6 @@ struct sffn_ctx {
     float* lst_h = nullptr;
     uint32_t* lst_mask = nullptr;
     int* seg_count = nullptr;
-    float* upart = nullptr;
     float* u = nullptr;
     float* dpart = nullptr;
     unsigned* tickets = nullptr;
@@ -100,24 +98,47 @@ struct sffn_ctx {
 
 namespace {
 
-constexpr size_t kGateSmemCap = 110 * 1024;   // keeps two gate CTAs per SM
+constexpr size_t kPreselSmemCap = 110 * 1024;  // keeps two up-pass CTAs per SM
+constexpr size_t kStreamSmemCap = 110 * 1024;  // two streaming gate CTAs per SM
 
 int pick_nt(int n) { return n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : 8; }
 
-int gate_nt(const sffn_ctx* h, int n, int gate_kind) {
+int presel_nt(const sffn_ctx* h, int n) {
     int nt = pick_nt(n);
-    const int r = gate_kind == kGateLopa ? h->cfg.lopa_rank : 0;
-    while (nt > 1 &&
-           gate_smem_bytes(h->cfg.wdtype, nt, h->cfg.d, r, gate_kind, h->plan.cpb, h->plan.mw) > kGateSmemCap)
+    while (nt > 1 && gate_smem_bytes(h->cfg.wdtype, nt, h->cfg.d, 0, kGatePreselected, h->plan.cpb,
+                                     h->plan.mw) > kPreselSmemCap)
         nt /= 2;
     return nt;
 }
 
-int gate_rw(const sffn_ctx* h, int gate_kind) {
-    const int v = h->cfg.wdtype == SFFN_BF16 ? 8 : 4;
-    if (gate_kind == kGatePreselected) return 1;
-    const int cpr = (gate_kind == kGateLopa ? h->cfg.lopa_rank : h->cfg.d) / v;
-    return cpr <= 64 ? 4 : 1;
+// Token tile and streaming geometry (piece bytes sb, pieces in flight per
+// warp nb) of the streaming gate kernel: the largest tile whose shared memory
+// fits with at least two pieces of 4 KB in flight per warp, then the deepest
+// ring of 8 KB (else 4 KB) pieces, at most 4.
+struct StreamGeom {
+    int nt, sb, nb;
+    size_t smem;
+};
+StreamGeom stream_geom(const sffn_ctx* h, int n, int gate_kind) {
+    const sffn_config& c = h->cfg;
+    const int r = gate_kind == kGateLopa ? c.lopa_rank : 0;
+    auto bytes = [&](int nt, int sb, int nb) {
+        return gate_stream_smem_bytes(nt, c.d, r, gate_kind, h->plan.cpb, h->plan.mw, sb, nb);
+    };
+    int nt = pick_nt(n);
+    while (nt > 1 && bytes(nt, 4096, 2) > kStreamSmemCap) nt /= 2;
+    StreamGeom g{nt, 4096, 1, 0};
+    for (int sb : {8192, 4096}) {
+        int nb = 4;
+        while (nb > 1 && bytes(nt, sb, nb) > kStreamSmemCap) --nb;
+        if (nb >= 2 || sb == 4096) {
+            g.sb = sb;
+            g.nb = nb;
+            break;
+        }
+    }
+    g.smem = bytes(g.nt, g.sb, g.nb);
+    return g;
 }
 
 // Stage events are recorded as external event nodes under stream capture so
@@ -179,11 +200,8 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
 
     if (lopa) {
         LopaUParams lp{};
-        lp.x = x; lp.a = h->a; lp.n = n; lp.d = c.d; lp.r = c.lopa_rank;
-        lp.rows_per_cta = P.lopa_rows; lp.cols_per_cta = P.lopa_cols;
-        lp.part = h->upart; lp.u = h->u; lp.tickets = h->tickets;
-        SFFN_CUDA(launch_lopa_u(c.wdtype, lp, pick_nt(n), dim3(P.lopa_splits, P.lopa_groups), s, pdl),
-                  "LoPA x*A launch");
+        lp.x = x; lp.at = h->a; lp.n = n; lp.d = c.d; lp.r = c.lopa_rank; lp.u = h->u;
+        SFFN_CUDA(launch_lopa_u(c.wdtype, lp, pick_nt(n), s, pdl), "LoPA x*A launch");
         record(h, ++launches, s);
     }
 
@@ -196,26 +214,24 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     gp.cpb = P.cpb; gp.mw = P.mw;
     gp.lst_idx = h->lst_idx; gp.lst_h = h->lst_h; gp.lst_mask = h->lst_mask; gp.seg_count = h->seg_count;
 
+    const StreamGeom sg = stream_geom(h, n, gk);
+    gp.sb = sg.sb;
+    gp.nb = sg.nb;
+    gp.status = h->status;
     if (sel->kind == SFFN_SELECT_THRESHOLD) {
         gp.out = kOutSelectUp;
-        const int nt = gate_nt(h, n, gk);
-        SFFN_CUDA(launch_gate(c.wdtype, gp, nt, gate_rw(h, gk), gk, P.g1,
-                              gate_smem_bytes(c.wdtype, nt, c.d, c.lopa_rank, gk, P.cpb, P.mw), s, pdl),
-                  "gate/select/up launch");
+        SFFN_CUDA(launch_gate_stream(c.wdtype, gp, sg.nt, gk, P.g1, sg.smem, s, pdl), "gate/select/up launch");
         record(h, ++launches, s);
     } else {
         gp.out = kOutWriteZ;
-        int nt = gate_nt(h, n, gk);
-        SFFN_CUDA(launch_gate(c.wdtype, gp, nt, gate_rw(h, gk), gk, P.g1,
-                              gate_smem_bytes(c.wdtype, nt, c.d, c.lopa_rank, gk, P.cpb, P.mw), s, pdl),
-                  "gate launch");
+        SFFN_CUDA(launch_gate_stream(c.wdtype, gp, sg.nt, gk, P.g1, sg.smem, s, pdl), "gate launch");
         record(h, ++launches, s);
         TopkParams tp{};
         tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
         SFFN_CUDA(launch_topk(tp, s, pdl), "top-K launch");
         record(h, ++launches, s);
         gp.out = kOutSelectUp;
-        nt = gate_nt(h, n, kGatePreselected);
+        const int nt = presel_nt(h, n);
         SFFN_CUDA(launch_gate(c.wdtype, gp, nt, 1, kGatePreselected, P.g1,
                               gate_smem_bytes(c.wdtype, nt, c.d, 0, kGatePreselected, P.cpb, P.mw), s, pdl),
                   "selected up launch");
@@ -226,12 +242,12 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     dp.wdn = h->wdn; dp.n = n; dp.d = c.d; dp.d_ff = c.d_ff;
     dp.seg_count = h->seg_count; dp.g1 = P.g1; dp.cpb = P.cpb;
     dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.part = h->dpart;
-    dp.tickets = h->tickets + P.lopa_groups; dp.y = out;
-    dp.chunks = P.down_chunks; dp.min_rows = P.down_min_rows; dp.max_rows = P.down_max_rows;
+    dp.tickets = h->tickets; dp.y = out;
+    dp.chunks = P.down_chunks;
     dp.status = h->status;
     const int dnt = pick_nt(n);
-    SFFN_CUDA(launch_down(c.wdtype, dp, dnt, P.down_slices,
-                          down_smem_bytes(c.wdtype, dnt, P.g1, P.down_max_rows), s, pdl),
+    const int nseg = (P.g1 + P.down_chunks - 1) / P.down_chunks;
+    SFFN_CUDA(launch_down(c.wdtype, dp, dnt, P.down_slices, down_smem_bytes(c.wdtype, dnt, nseg, P.cpb), s, pdl),
               "down launch");
     record(h, ++launches, s);
 
@@ -304,20 +320,13 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "device attribute"); }
 
     Plan& P = h->plan;
-    const int target = 2 * h->sms;
-    P.cpb = (c.d_ff + target - 1) / target;
+    P.cpb = (c.d_ff + 2 * h->sms - 1) / (2 * h->sms);   // two gate CTAs per SM
     P.g1 = (c.d_ff + P.cpb - 1) / P.cpb;
     P.mw = (c.max_tokens + 31) / 32;
-    if (c.lopa_rank > 0) {
-        P.lopa_rows = 128;
-        P.lopa_cols = 64;
-        P.lopa_splits = (c.d + P.lopa_rows - 1) / P.lopa_rows;
-        P.lopa_groups = (c.lopa_rank + P.lopa_cols - 1) / P.lopa_cols;
-    }
     P.down_slices = (c.d + down_slice_cols(c.wdtype) - 1) / down_slice_cols(c.wdtype);
-    P.down_chunks = target / P.down_slices > 1 ? target / P.down_slices : 1;
-    P.down_min_rows = 16;
-    P.down_max_rows = down_max_rows(c.d_ff, P.down_chunks, P.down_min_rows);
+    P.down_chunks = h->sms / P.down_slices;                 // about one down CTA per SM
+    if (P.down_chunks < 1) P.down_chunks = 1;
+    if (P.down_chunks > P.g1) P.down_chunks = P.g1;
 
     const size_t T = c.max_tokens, F = c.d_ff, D = c.d, R = c.lopa_rank;
     size_t off = 0;
@@ -325,9 +334,9 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_z = take(T * F * 4), o_g = take(T * F * 4), o_sel = take(T * F);
     const size_t o_idx = take(F * 4), o_h = take(F * T * 4), o_mask = take(F * P.mw * 4);
     const size_t o_seg = take((size_t)P.g1 * 4);
-    const size_t o_up = take((size_t)P.lopa_splits * T * R * 4), o_u = take(T * R * 4);
+    const size_t o_u = take(T * R * 4);
     const size_t o_dp = take((size_t)P.down_chunks * T * D * 4);
-    const size_t o_tk = take((size_t)(P.lopa_groups + P.down_slices) * 4), o_st = take(4);
+    const size_t o_tk = take((size_t)P.down_slices * 4), o_st = take(4);
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
     e = cudaMalloc(&h->ws, off);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "workspace allocation"); }
@@ -339,7 +348,6 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->lst_h = reinterpret_cast<float*>(b + o_h);
     h->lst_mask = reinterpret_cast<uint32_t*>(b + o_mask);
     h->seg_count = reinterpret_cast<int*>(b + o_seg);
-    h->upart = reinterpret_cast<float*>(b + o_up);
     h->u = reinterpret_cast<float*>(b + o_u);
     h->dpart = reinterpret_cast<float*>(b + o_dp);
     h->tickets = reinterpret_cast<unsigned*>(b + o_tk);
@@ -402,9 +410,10 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
         if (A) {
             if ((e = alloc(&h->a, r_d)) != cudaSuccess) break;
             if ((e = alloc(&h->bcm, r_ff)) != cudaSuccess) break;
-            if ((e = cudaMemcpyAsync(h->a, A, r_d, src_is_device ? cudaMemcpyDeviceToDevice
-                                                                 : cudaMemcpyHostToDevice, s)) != cudaSuccess)
-                break;
+            src = stage(A, r_d);
+            if (!src) { e = cudaGetLastError(); break; }
+            if ((e = launch_transpose(c.wdtype, src, h->a, c.d, c.lopa_rank, s)) != cudaSuccess) break;
+            if ((e = cudaStreamSynchronize(s)) != cudaSuccess) break;
             src = stage(B, r_ff);
             if (!src) { e = cudaGetLastError(); break; }
             if ((e = launch_transpose(c.wdtype, src, h->bcm, c.lopa_rank, c.d_ff, s)) != cudaSuccess) break;

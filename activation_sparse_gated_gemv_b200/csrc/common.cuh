@@ -52,6 +52,74 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
     return v;
 }
 
+// ---------------------------------------------------------------------------
+// Bulk asynchronous copies (TMA engine, 1-D form) completing on an mbarrier.
+// No cluster multicast anywhere: every copy lands in the issuing CTA.
+
+constexpr unsigned long long kWaitLimitNs = 500ull * 1000ull * 1000ull;   // 0.5 s
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+// Global -> this CTA's shared memory, `bytes` a multiple of 16, both ends 16-byte aligned.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+// Ask the TMA engine to bring `bytes` (multiple of 16) at `src` into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+// L2 policy for data read once per forward (weights): evict first.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Every lane of the warp waits for the phase with `parity` to complete.  The
+// decision is warp-uniform; false after kWaitLimitNs (the caller records it).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+    bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (;;) {
+        if (!done) done = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        const bool late = globaltimer_ns() - t0 > kWaitLimitNs;
+        if (__shfl_sync(0xffffffffu, late ? 1 : 0, 0)) return false;
+    }
+}
+
 // bf16 is the upper half of an IEEE binary32: widening is a 16-bit shift.
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -137,17 +205,16 @@ struct GateParams {
     float* lst_h;
     uint32_t* lst_mask;
     int* seg_count;
+    int sb;                 // streamed piece bytes (multiple of 16)
+    int nb;                 // pieces in flight per warp
+    int* status;            // sticky device status word
 };
 
 struct LopaUParams {
     const void* x;          // [n][d] T
-    const void* a;          // [d][r] T
+    const void* at;         // [r][d] T   A transposed: column j of A is row j
     int n, d, r;
-    int rows_per_cta;       // d split
-    int cols_per_cta;       // r split (multiple of the vector width)
-    float* part;            // [splits][n][r]
     float* u;               // [n][r]
-    unsigned* tickets;      // [r column groups]
 };
 
 struct TopkParams {
@@ -167,14 +234,12 @@ struct DownParams {
     float* part;            // [chunks][n][d]
     unsigned* tickets;      // [column slices]
     void* y;                // [n][d] T
-    int chunks;             // chunk CTAs per column slice (grid.y)
-    int min_rows;           // fewest rows worth a chunk
-    int max_rows;           // rows one chunk can hold (shared-memory bound)
+    int chunks;             // chunk CTAs per column slice (grid.y), each a run of gate segments
     int* status;            // sticky device status word (bit set on a failed check)
 };
 
 // Bits of the device status word.
-enum StatusBits { kStatusDownRows = 1 };
+enum StatusBits { kStatusWaitTimeout = 2 };
 
 // Raise a kernel's dynamic shared-memory limit once per device (so a forward
 // inside stream capture issues launches only).  `cache` is per kernel.
@@ -214,13 +279,15 @@ inline cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaS
 cudaError_t launch_gate(int wdtype, const GateParams& p, int nt, int rw, int gate_kind, int grid,
                         size_t smem, cudaStream_t s, bool pdl);
 size_t gate_smem_bytes(int wdtype, int nt, int d, int r, int gate_kind, int cpb, int mw);
-cudaError_t launch_lopa_u(int wdtype, const LopaUParams& p, int nt, dim3 grid, cudaStream_t s,
-                          bool pdl);
+cudaError_t launch_gate_stream(int wdtype, const GateParams& p, int nt, int gate_kind, int grid, size_t smem,
+                               cudaStream_t s, bool pdl);
+size_t gate_stream_smem_bytes(int nt, int d, int r, int gate_kind, int cpb, int mw, int sb, int nb);
+cudaError_t launch_lopa_u(int wdtype, const LopaUParams& p, int nt, cudaStream_t s, bool pdl);
+constexpr int kLopaRowsPerCta = 2;
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_down(int wdtype, const DownParams& p, int nt, int slices, size_t smem,
                         cudaStream_t s, bool pdl);
-size_t down_smem_bytes(int wdtype, int nt, int g1, int max_rows);
-int down_max_rows(int d_ff, int chunks, int min_rows);
+size_t down_smem_bytes(int wdtype, int nt, int nseg, int cpb);
 int down_slice_cols(int wdtype);
 cudaError_t launch_transpose(int wdtype, const void* src, void* dst, int rows, int cols,
                              cudaStream_t s);

@@ -4,14 +4,16 @@
 // the K active channels are multiplied and accumulated, so only their W_down
 // rows are read.)
 //
-// Grid = (column slices of 512 outputs) x (chunks of the active list).  Every
-// CTA rebuilds the list's prefix over the gate CTAs' segments, takes an equal
-// share of the M listed channels, streams the 512-column piece of each of its
-// rows (16-byte L1-bypassing loads, four rows in flight per thread) and writes
-// an fp32 partial.  The last CTA to finish a column slice (ticket counter)
-// adds the partials in chunk order and stores y.  The chunk count shrinks on
-// the device with M, so a short list does not pay for many partials; the
-// result depends only on M, never on timing.
+// Grid = (column slices of 512 outputs) x (chunks).  Chunk c takes the list
+// segments of gate CTAs [c*g1/CH, (c+1)*g1/CH): their counts and (speculatively)
+// their whole slot ranges of channel ids are read in one round trip, then
+// compacted in shared memory.  Each thread reads a 16-byte piece of the
+// 512-column slice of its row group's listed W_down rows, up to 16 rows in
+// flight per thread (L1-bypassing loads), multiplies by h and accumulates in
+// fp32; row groups are added in a fixed order and the CTA's partial goes to
+// global memory.  The last CTA of each column slice
+// (ticket counter) adds the chunk partials in chunk order and stores y, so y is
+// bitwise reproducible.
 #include "common.cuh"
 
 namespace sffn {
@@ -19,72 +21,80 @@ namespace sffn {
 constexpr int kSliceCols = 512;
 
 struct DownSmem {
-    size_t prefix, rows, red, total;
+    size_t cnt, idx, rowk, red, total;
 };
-__host__ __device__ inline DownSmem down_smem_layout(int nt, int g1, int max_rows, int rg) {
+__host__ __device__ inline DownSmem down_smem_layout(int nt, int nseg, int cpb, int rg) {
     DownSmem L;
     size_t o = 0;
-    L.prefix = o; o += (((size_t)g1 + 1) * sizeof(int) + 15) & ~(size_t)15;
-    L.rows = o;   o += ((size_t)max_rows * sizeof(int) + 15) & ~(size_t)15;
-    L.red = o;    o += (size_t)rg * nt * kSliceCols * sizeof(float);
+    const size_t cap = (size_t)nseg * cpb;
+    L.cnt = o;   o += (((size_t)nseg + 1) * 2 * sizeof(int) + 15) & ~(size_t)15;   // counts, prefix
+    L.idx = o;   o += (cap * sizeof(int) + 15) & ~(size_t)15;
+    L.rowk = o;  o += (cap * sizeof(int) + 15) & ~(size_t)15;
+    L.red = o;   o += (size_t)rg * nt * kSliceCols * sizeof(float);
     L.total = o;
     return L;
 }
 
 template <class T, int NT>
-__global__ void __launch_bounds__(kThreads) k_down(const DownParams p) {
+__global__ void __launch_bounds__(kThreads, 2) k_down(const DownParams p) {
     constexpr int V = Elem<T>::kVec;
-    constexpr int TPR = kSliceCols / V;      // threads per row
-    constexpr int RG = kThreads / TPR;       // row groups
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int sh[40];
+    constexpr int TPR = kSliceCols / V;             // threads per row
+    constexpr int RG = kThreads / TPR;              // row groups
+    constexpr int UB = NT == 1 ? 16 : NT == 2 ? 8 : 4;   // rows in flight per thread
+    extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int s_last;
-    const DownSmem L = down_smem_layout(NT, p.g1, p.max_rows, RG);
-    int* prefix = reinterpret_cast<int*>(smem + L.prefix);
-    int* rows_k = reinterpret_cast<int*>(smem + L.rows);
+    const int nseg_max = (p.g1 + p.chunks - 1) / p.chunks;
+    const DownSmem L = down_smem_layout(NT, nseg_max, p.cpb, RG);
+    int* cnt = reinterpret_cast<int*>(smem + L.cnt);
+    int* pre = cnt + nseg_max + 1;
+    int* idx = reinterpret_cast<int*>(smem + L.idx);
+    int* rowk = reinterpret_cast<int*>(smem + L.rowk);
     float* red = reinterpret_cast<float*>(smem + L.red);
+
+    const int seg0 = (int)((long long)blockIdx.y * p.g1 / p.chunks);
+    const int seg1 = (int)((long long)(blockIdx.y + 1) * p.g1 / p.chunks);
+    const int nseg = seg1 - seg0;
+    const int col0 = blockIdx.x * kSliceCols;
+    const int ncols = min(kSliceCols, p.d - col0);
+    const T* wdn = static_cast<const T*>(p.wdn);
 
     griddep_wait();
     griddep_launch_dependents();
 
-    int carry = 0;
-    for (int b0 = 0; b0 < p.g1; b0 += kThreads) {
-        const int b = b0 + threadIdx.x;
-        const int c = b < p.g1 ? p.seg_count[b] : 0;
-        int tot = 0;
-        const int ex = block_exclusive_scan(c, &tot, sh);
-        if (b < p.g1) prefix[b] = carry + ex;
-        carry += tot;
-    }
-    if (threadIdx.x == 0) prefix[p.g1] = carry;
-    const int M = carry;
-    const int chunks_eff = max(1, min(p.chunks, (M + p.min_rows - 1) / p.min_rows));
-    if ((int)blockIdx.y >= chunks_eff) return;
-    const int q0 = (int)((long long)M * blockIdx.y / chunks_eff);
-    const int q1 = (int)((long long)M * (blockIdx.y + 1) / chunks_eff);
-    int rows = q1 - q0;
-    // rows <= max(min_rows, ceil(d_ff / chunks)) by construction; guard anyway
-    // (record it and contribute nothing, so the ticket protocol still completes).
-    if (rows > p.max_rows) {
-        if (threadIdx.x == 0) atomicOr(p.status, (int)kStatusDownRows);
-        rows = 0;
+    // Counts and the segments' whole slot ranges, in one round trip.
+    for (int i = threadIdx.x; i < nseg; i += kThreads) cnt[i] = p.seg_count[seg0 + i];
+    for (int i = threadIdx.x; i < nseg * p.cpb; i += kThreads) {
+        const int slot = seg0 * p.cpb + i;
+        idx[i] = slot < p.d_ff ? p.lst_idx[slot] : 0;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < rows; i += kThreads) {
-        const int q = q0 + i;
-        int lo = 0, hi = p.g1;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (prefix[mid] <= q) lo = mid; else hi = mid;
+    if (threadIdx.x < 32) {
+        int carry = 0;
+        for (int b0 = 0; b0 < nseg; b0 += 32) {
+            const int b = b0 + threadIdx.x;
+            const int c = b < nseg ? cnt[b] : 0;
+            int x = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if ((int)threadIdx.x >= o) x += y;
+            }
+            if (b < nseg) pre[b] = carry + x - c;
+            carry += __shfl_sync(0xffffffffu, x, 31);
         }
-        rows_k[i] = p.lst_idx[lo * p.cpb + (q - prefix[lo])];
+        if (threadIdx.x == 0) pre[nseg] = carry;
+    }
+    __syncthreads();
+    const int rows = pre[nseg];
+    for (int i = threadIdx.x; i < nseg * p.cpb; i += kThreads) {
+        const int j = i / p.cpb, o = i - j * p.cpb;
+        if (o < cnt[j]) rowk[pre[j] + o] = idx[i];
     }
     __syncthreads();
 
-    const T* wdn = static_cast<const T*>(p.wdn);
     const int rg = threadIdx.x / TPR, tc = threadIdx.x - rg * TPR;
-    const int col = blockIdx.x * kSliceCols + tc * V;
-    const bool colok = col < p.d;
+    const bool colok = tc * V < ncols;
+    const T* wcol = wdn + col0 + tc * V;
     for (int t0 = 0; t0 < p.n; t0 += NT) {
         const int nt = min(NT, p.n - t0);
         float acc[NT][V];
@@ -92,37 +102,26 @@ __global__ void __launch_bounds__(kThreads) k_down(const DownParams p) {
         for (int t = 0; t < NT; ++t)
 #pragma unroll
             for (int e = 0; e < V; ++e) acc[t][e] = 0.f;
-        int i = rg;
-        for (; i + 3 * RG < rows; i += 4 * RG) {
-            int kk[4];
-            uint4 w[4];
+        for (int i0 = rg; i0 < rows; i0 += UB * RG) {
+            uint4 w[UB];
+            float h[UB][NT];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) kk[u] = rows_k[i + u * RG];
+            for (int u = 0; u < UB; ++u) {
+                const int i = i0 + u * RG;
+                const bool in = i < rows;
+                const int k = in ? rowk[i] : 0;
+                w[u] = (in && colok) ? ld_stream(wcol + (size_t)k * p.d) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                w[u] = colok ? ld_stream(wdn + (size_t)kk[u] * p.d + col) : make_uint4(0u, 0u, 0u, 0u);
+                for (int t = 0; t < NT; ++t) h[u][t] = (in && t < nt) ? p.lst_h[(size_t)k * p.n + t0 + t] : 0.f;
+            }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < UB; ++u) {
                 float wf[V];
                 unpack<T>(w[u], wf);
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    const float hv = t < nt ? p.lst_h[(size_t)kk[u] * p.n + t0 + t] : 0.f;
+                for (int t = 0; t < NT; ++t)
 #pragma unroll
-                    for (int e = 0; e < V; ++e) acc[t][e] = fmaf(hv, wf[e], acc[t][e]);
-                }
-            }
-        }
-        for (; i < rows; i += RG) {
-            const int k = rows_k[i];
-            const uint4 w = colok ? ld_stream(wdn + (size_t)k * p.d + col) : make_uint4(0u, 0u, 0u, 0u);
-            float wf[V];
-            unpack<T>(w, wf);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const float hv = t < nt ? p.lst_h[(size_t)k * p.n + t0 + t] : 0.f;
-#pragma unroll
-                for (int e = 0; e < V; ++e) acc[t][e] = fmaf(hv, wf[e], acc[t][e]);
+                    for (int e = 0; e < V; ++e) acc[t][e] = fmaf(h[u][t], wf[e], acc[t][e]);
             }
         }
         __syncthreads();
@@ -131,32 +130,77 @@ __global__ void __launch_bounds__(kThreads) k_down(const DownParams p) {
 #pragma unroll
             for (int e = 0; e < V; ++e) red[((size_t)rg * NT + t) * kSliceCols + tc * V + e] = acc[t][e];
         __syncthreads();
-        for (int idx = threadIdx.x; idx < NT * kSliceCols; idx += kThreads) {
-            const int t = idx / kSliceCols, c = idx - t * kSliceCols;
-            const int gc = blockIdx.x * kSliceCols + c;
-            if (t < nt && gc < p.d) {
-                float s = 0.f;
+        for (int i = threadIdx.x; i < NT * (kSliceCols / 4); i += kThreads) {
+            const int t = i / (kSliceCols / 4), c = (i - t * (kSliceCols / 4)) * 4;
+            if (t < nt && c < ncols) {
+                float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int g = 0; g < RG; ++g) s += red[((size_t)g * NT + t) * kSliceCols + c];
-                p.part[((size_t)blockIdx.y * p.n + t0 + t) * p.d + gc] = s;
+                for (int r = 0; r < RG; ++r) {
+                    const float4 v = *reinterpret_cast<const float4*>(red + ((size_t)r * NT + t) * kSliceCols + c);
+                    s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+                }
+                *reinterpret_cast<float4*>(p.part + ((size_t)blockIdx.y * p.n + t0 + t) * p.d + col0 + c) = s;
             }
         }
     }
 
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&p.tickets[blockIdx.x], 1u) == (unsigned)chunks_eff - 1u;
+    if (threadIdx.x == 0) s_last = atomicAdd(&p.tickets[blockIdx.x], 1u) == (unsigned)p.chunks - 1u;
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+
+    // Sum the chunk partials in chunk order.  Item = (token, 4 columns); when
+    // there are fewer items than threads, G thread groups take interleaved
+    // chunks and their sums are added in group order.
     T* y = static_cast<T*>(p.y);
-    for (int idx = threadIdx.x; idx < p.n * kSliceCols; idx += kThreads) {
-        const int t = idx / kSliceCols;
-        const int gc = blockIdx.x * kSliceCols + (idx - t * kSliceCols);
-        if (gc < p.d) {
-            float s = 0.f;
-            for (int ch = 0; ch < chunks_eff; ++ch) s += __ldcg(&p.part[((size_t)ch * p.n + t) * p.d + gc]);
-            y[(size_t)t * p.d + gc] = from_f32<T>(s);
+    constexpr int C4 = kSliceCols / 4;
+    const int items = p.n * C4;
+    const int G = items >= kThreads ? 1 : kThreads / items;
+    const int per_round = kThreads / G;
+    float4* gsum = reinterpret_cast<float4*>(red);                // [G][per_round]
+    const size_t stride = (size_t)p.n * p.d / 4;
+    for (int base = 0; base < items; base += per_round) {
+        const int item = base + (int)threadIdx.x % per_round;
+        const int grp = (int)threadIdx.x / per_round;
+        const int t = item / C4, c = (item - t * C4) * 4;
+        const bool ok = item < items && c < ncols && grp < G;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ok) {
+            const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)t * p.d + col0 + c);
+            int ch = grp;
+            for (; ch + 15 * G < p.chunks; ch += 16 * G) {
+                float4 v[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) v[q] = __ldcg(src + (size_t)(ch + q * G) * stride);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    s.x += v[q].x; s.y += v[q].y; s.z += v[q].z; s.w += v[q].w;
+                }
+            }
+            for (; ch < p.chunks; ch += G) {
+                const float4 v = __ldcg(src + (size_t)ch * stride);
+                s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+            }
+        }
+        if (G > 1) {
+            __syncthreads();
+            if (grp < G) gsum[grp * per_round + (int)threadIdx.x % per_round] = s;
+            __syncthreads();
+            if (grp == 0 && ok) {
+                for (int q = 1; q < G; ++q) {
+                    const float4 v = gsum[q * per_round + (int)threadIdx.x % per_round];
+                    s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+                }
+            }
+        }
+        if (grp == 0 && ok) {
+            T* dst = y + (size_t)t * p.d + col0 + c;
+            dst[0] = from_f32<T>(s.x);
+            dst[1] = from_f32<T>(s.y);
+            dst[2] = from_f32<T>(s.z);
+            dst[3] = from_f32<T>(s.w);
         }
     }
     if (threadIdx.x == 0) p.tickets[blockIdx.x] = 0u;
@@ -164,16 +208,10 @@ __global__ void __launch_bounds__(kThreads) k_down(const DownParams p) {
 
 int down_slice_cols(int /*wdtype*/) { return kSliceCols; }
 
-int down_max_rows(int d_ff, int chunks, int min_rows) {
-    const int c = chunks > 0 ? chunks : 1;
-    const int per = (d_ff + c - 1) / c;
-    return per > min_rows ? per : min_rows;
-}
-
-size_t down_smem_bytes(int wdtype, int nt, int g1, int max_rows) {
+size_t down_smem_bytes(int wdtype, int nt, int nseg, int cpb) {
     const int V = wdtype == 0 ? 8 : 4;
     const int rg = kThreads / (kSliceCols / V);
-    return down_smem_layout(nt, g1, max_rows, rg).total;
+    return down_smem_layout(nt, nseg, cpb, rg).total;
 }
 
 template <class T, int NT>
@@ -187,8 +225,8 @@ static cudaError_t launch_down_t(const DownParams& p, int slices, size_t smem, c
 
 cudaError_t launch_down(int wdtype, const DownParams& p, int nt, int slices, size_t smem, cudaStream_t s,
                         bool pdl) {
-    if (p.max_rows < down_max_rows(p.d_ff, p.chunks, p.min_rows) ||
-        smem < down_smem_bytes(wdtype, nt, p.g1, p.max_rows))
+    const int nseg = (p.g1 + p.chunks - 1) / p.chunks;
+    if (p.chunks < 1 || p.chunks > p.g1 || smem < down_smem_bytes(wdtype, nt, nseg, p.cpb))
         return cudaErrorInvalidValue;
     if (wdtype == 0) {
         switch (nt) {
