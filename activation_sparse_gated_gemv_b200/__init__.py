@@ -69,6 +69,7 @@ _sigs = {
     "sffn_destroy": ([_P], _I),
     "sffn_strerror": ([_I], ctypes.c_char_p),
     "sffn_last_error": ([], ctypes.c_char_p),
+    "sffn_forward_noalloc": ([_P, _P, _P, _I, _I, _I, _P, _I, ctypes.c_float, _P, _P], _I),
 }
 for _name, (_args, _res) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -88,6 +89,7 @@ sffn_check_status = _lib.sffn_check_status
 sffn_destroy = _lib.sffn_destroy
 sffn_strerror = _lib.sffn_strerror
 sffn_last_error = _lib.sffn_last_error
+sffn_forward_noalloc = _lib.sffn_forward_noalloc
 
 EXPORTED = tuple(_sigs)
 

@@ -136,6 +136,37 @@ int sffn_last_launches(sffn_handle h, int32_t* launches);
  * (the word stays set); also INVALID_ARG, CUDA. */
 int sffn_check_status(sffn_handle h);
 
+/* Sparse forward that allocates no device memory, for callers that cannot
+ * call cudaMalloc while they run: a host runtime that owns all device memory
+ * through its own pool, or latency-critical code where an allocation (which
+ * can synchronise the device) is not allowed after start-up.  No handle is
+ * used (creating one allocates); the weights come from the caller.  The
+ * pages describe no such interface: this entry point has no counterpart in
+ * them.
+ *
+ * Computes the dense-gate, threshold-select forward of sffn_forward:
+ * y[t,:] = sum_{k: z[t,k] > tau} (z[t,k] - tau) <x[t,:], W_up[:,k]> W_down[k,:].
+ * Inputs are device buffers in `wdtype` (SFFN_BF16 or SFFN_F32), 16-byte
+ * aligned, on the current device, owned by the caller:
+ *   w_gate_cm  d_ff x d   row k is column k of W_gate
+ *   w_up_cm    d_ff x d   row k is column k of W_up
+ *   w_down     d_ff x d   W_down as is
+ *   x          n_tokens x d;   out  n_tokens x d
+ * Limits: d a multiple of 8 and <= 8192, 1 <= d_ff <= 32768,
+ * 0 <= n_tokens <= 8; beyond them the call returns SFFN_ERR_INVALID_ARG and
+ * prints why.  tau: a number or +inf.
+ * Scratch: one file-scope device array of about 3.9 MiB, reserved on every GPU
+ * that loads the library until the process exits.  Every call shares it and
+ * it keeps the last call's contents (the call clears what must start at
+ * zero), so calls whose kernels overlap on the GPU -- on two streams, or from
+ * two threads -- race and give wrong results: order them.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress, once per
+ * device); make that first call before any stream capture.
+ * Asynchronous on `stream` (cudaStream_t as void*, NULL = legacy default).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+int sffn_forward_noalloc(const void* w_gate_cm, const void* w_up_cm, const void* w_down, int d, int d_ff,
+                         int wdtype, const void* x, int n_tokens, float tau, void* out, void* stream);
+
 /* Free the handle and everything it owns.  NULL is accepted. */
 int sffn_destroy(sffn_handle h);
 
