@@ -70,6 +70,7 @@ _sigs = {
     "sffn_strerror": ([_I], ctypes.c_char_p),
     "sffn_last_error": ([], ctypes.c_char_p),
     "sffn_forward_noalloc": ([_P, _P, _P, _I, _I, _I, _P, _I, ctypes.c_float, _P, _P], _I),
+    "sffn_last_kernel_name": ([_P, _I], ctypes.c_char_p),
 }
 for _name, (_args, _res) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -90,6 +91,7 @@ sffn_destroy = _lib.sffn_destroy
 sffn_strerror = _lib.sffn_strerror
 sffn_last_error = _lib.sffn_last_error
 sffn_forward_noalloc = _lib.sffn_forward_noalloc
+sffn_last_kernel_name = _lib.sffn_last_kernel_name
 
 EXPORTED = tuple(_sigs)
 
@@ -210,6 +212,9 @@ class SparseFFN:
         v = ctypes.c_int32(0)
         check(sffn_last_launches(self._h, ctypes.byref(v)), "sffn_last_launches")
         return int(v.value)
+
+    def last_kernel_names(self) -> List[str]:
+        return [sffn_last_kernel_name(self._h, i).decode() for i in range(self.last_launches())]
 
     def check_status(self) -> None:
         check(sffn_check_status(self._h), "sffn_check_status")

@@ -85,6 +85,7 @@ struct sffn_ctx {
     int* seg_count = nullptr;
     float* u = nullptr;
     float* dpart = nullptr;
+    float* fpart = nullptr;
     unsigned* tickets = nullptr;
     int* status = nullptr;
     void* xdev = nullptr;
@@ -93,13 +94,13 @@ struct sffn_ctx {
     int last_n = -1;
     cudaStream_t last_stream = nullptr;
     int last_launches = 0;
+    const char* last_names[8] = {};
     std::vector<cudaEvent_t> events;
 };
 
 namespace {
 
 constexpr size_t kPreselSmemCap = 110 * 1024;  // keeps two up-pass CTAs per SM
-constexpr size_t kStreamSmemCap = 110 * 1024;  // two streaming gate CTAs per SM
 
 int pick_nt(int n) { return n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : 8; }
 
@@ -111,10 +112,9 @@ int presel_nt(const sffn_ctx* h, int n) {
     return nt;
 }
 
-// Token tile and streaming geometry (piece bytes sb, pieces in flight per
-// warp nb) of the streaming gate kernel: the largest tile whose shared memory
-// fits with at least two pieces of 4 KB in flight per warp, then the deepest
-// ring of 8 KB (else 4 KB) pieces, at most 4.
+// Token tile and streaming geometry of the streaming gate kernel: the largest
+// tile (at most the batch) for which some geometry fits; see
+// gate_stream_geometry for the piece size and depth.
 struct StreamGeom {
     int nt, sb, nb;
     size_t smem;
@@ -122,22 +122,10 @@ struct StreamGeom {
 StreamGeom stream_geom(const sffn_ctx* h, int n, int gate_kind) {
     const sffn_config& c = h->cfg;
     const int r = gate_kind == kGateLopa ? c.lopa_rank : 0;
-    auto bytes = [&](int nt, int sb, int nb) {
-        return gate_stream_smem_bytes(nt, c.d, r, gate_kind, h->plan.cpb, h->plan.mw, sb, nb);
-    };
-    int nt = pick_nt(n);
-    while (nt > 1 && bytes(nt, 4096, 2) > kStreamSmemCap) nt /= 2;
-    StreamGeom g{nt, 4096, 1, 0};
-    for (int sb : {8192, 4096}) {
-        int nb = 4;
-        while (nb > 1 && bytes(nt, sb, nb) > kStreamSmemCap) --nb;
-        if (nb >= 2 || sb == 4096) {
-            g.sb = sb;
-            g.nb = nb;
-            break;
-        }
-    }
-    g.smem = bytes(g.nt, g.sb, g.nb);
+    StreamGeom g{pick_nt(n), 0, 0, 0};
+    while (!gate_stream_geometry(g.nt, c.d, r, gate_kind, h->plan.cpb, h->plan.mw, &g.sb, &g.nb, &g.smem) &&
+           g.nt > 1)
+        g.nt /= 2;
     return g;
 }
 
@@ -197,17 +185,46 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     const bool pdl = true;
     int launches = 0;
     record(h, 0, s);
+    for (auto& nm : h->last_names) nm = nullptr;
+
+    // Fused decode path: threshold selection, a few tokens, sparse forward.
+    int dec_sb = 0, dec_nb = 0;
+    size_t dec_smem = 0;
+    const int dec_nt = pick_nt(n);
+    const bool fused = sel->kind == SFFN_SELECT_THRESHOLD && !dense && n <= kDecodeMaxTokens &&
+                       decode_geometry(dec_nt, c.d, lopa ? c.lopa_rank : 0, gk, P.cpb, P.mw, &dec_sb, &dec_nb,
+                                       &dec_smem);
 
     if (lopa) {
         LopaUParams lp{};
         lp.x = x; lp.at = h->a; lp.n = n; lp.d = c.d; lp.r = c.lopa_rank; lp.u = h->u;
         SFFN_CUDA(launch_lopa_u(c.wdtype, lp, pick_nt(n), s, pdl), "LoPA x*A launch");
+        h->last_names[launches] = "lopa_u";
         record(h, ++launches, s);
+    }
+
+    if (fused) {
+        DecodeParams dp{};
+        dp.x = x; dp.n = n; dp.d = c.d; dp.d_ff = c.d_ff; dp.r = c.lopa_rank;
+        dp.wg = h->wg; dp.bcm = h->bcm; dp.u = h->u; dp.wup = h->wup; dp.wdn = h->wdn;
+        dp.tau = sel->tau; dp.cpb = P.cpb; dp.mw = P.mw;
+        dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
+        dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.part = h->fpart;
+        dp.tickets = h->tickets; dp.y = out;
+        dp.reducers = 32;
+        while (dp.reducers > 1 && (c.d % (4 * dp.reducers) || dp.reducers > P.g1)) dp.reducers /= 2;
+        SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
+        h->last_names[launches] = "decode_fused";
+        record(h, ++launches, s);
+        h->last_n = n;
+        h->last_stream = s;
+        h->last_launches = launches;
+        return SFFN_OK;
     }
 
     GateParams gp{};
     gp.x = x; gp.n = n; gp.d = c.d; gp.d_ff = c.d_ff; gp.r = c.lopa_rank;
-    gp.wg = h->wg; gp.bcm = h->bcm; gp.u = h->u; gp.wup = h->wup;
+    gp.wg = h->wg; gp.bcm = h->bcm; gp.u = h->u; gp.wup = h->wup; gp.wdn = h->wdn;
     gp.force_all = dense ? 1 : 0;
     gp.tau = sel->tau;
     gp.zbuf = h->zbuf; gp.gbuf = h->gbuf; gp.sel = h->sel;
@@ -215,26 +232,31 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     gp.lst_idx = h->lst_idx; gp.lst_h = h->lst_h; gp.lst_mask = h->lst_mask; gp.seg_count = h->seg_count;
 
     const StreamGeom sg = stream_geom(h, n, gk);
+    if (sg.sb == 0) return fail(SFFN_ERR_UNSUPPORTED, "d=%d too large for the streaming gate's shared memory", c.d);
     gp.sb = sg.sb;
     gp.nb = sg.nb;
     gp.status = h->status;
     if (sel->kind == SFFN_SELECT_THRESHOLD) {
         gp.out = kOutSelectUp;
         SFFN_CUDA(launch_gate_stream(c.wdtype, gp, sg.nt, gk, P.g1, sg.smem, s, pdl), "gate/select/up launch");
+        h->last_names[launches] = "gate_select_up";
         record(h, ++launches, s);
     } else {
         gp.out = kOutWriteZ;
         SFFN_CUDA(launch_gate_stream(c.wdtype, gp, sg.nt, gk, P.g1, sg.smem, s, pdl), "gate launch");
+        h->last_names[launches] = "gate_z";
         record(h, ++launches, s);
         TopkParams tp{};
         tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
         SFFN_CUDA(launch_topk(tp, s, pdl), "top-K launch");
+        h->last_names[launches] = "topk";
         record(h, ++launches, s);
         gp.out = kOutSelectUp;
         const int nt = presel_nt(h, n);
         SFFN_CUDA(launch_gate(c.wdtype, gp, nt, 1, kGatePreselected, P.g1,
                               gate_smem_bytes(c.wdtype, nt, c.d, 0, kGatePreselected, P.cpb, P.mw), s, pdl),
                   "selected up launch");
+        h->last_names[launches] = "preselected_up";
         record(h, ++launches, s);
     }
 
@@ -249,6 +271,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     const int nseg = (P.g1 + P.down_chunks - 1) / P.down_chunks;
     SFFN_CUDA(launch_down(c.wdtype, dp, dnt, P.down_slices, down_smem_bytes(c.wdtype, dnt, nseg, P.cpb), s, pdl),
               "down launch");
+    h->last_names[launches] = "down";
     record(h, ++launches, s);
 
     h->last_n = n;
@@ -320,7 +343,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "device attribute"); }
 
     Plan& P = h->plan;
-    P.cpb = (c.d_ff + 2 * h->sms - 1) / (2 * h->sms);   // two gate CTAs per SM
+    P.cpb = (c.d_ff + h->sms - 1) / h->sms;           // one gate CTA per SM
     P.g1 = (c.d_ff + P.cpb - 1) / P.cpb;
     P.mw = (c.max_tokens + 31) / 32;
     P.down_slices = (c.d + down_slice_cols(c.wdtype) - 1) / down_slice_cols(c.wdtype);
@@ -336,7 +359,8 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_seg = take((size_t)P.g1 * 4);
     const size_t o_u = take(T * R * 4);
     const size_t o_dp = take((size_t)P.down_chunks * T * D * 4);
-    const size_t o_tk = take((size_t)P.down_slices * 4), o_st = take(4);
+    const size_t o_fp = take((size_t)P.g1 * (T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * D * 4);
+    const size_t o_tk = take((size_t)(P.down_slices > 2 ? P.down_slices : 2) * 4), o_st = take(4);
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
     e = cudaMalloc(&h->ws, off);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "workspace allocation"); }
@@ -350,6 +374,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->seg_count = reinterpret_cast<int*>(b + o_seg);
     h->u = reinterpret_cast<float*>(b + o_u);
     h->dpart = reinterpret_cast<float*>(b + o_dp);
+    h->fpart = reinterpret_cast<float*>(b + o_fp);
     h->tickets = reinterpret_cast<unsigned*>(b + o_tk);
     h->status = reinterpret_cast<int*>(b + o_st);
     h->xdev = b + o_x;
@@ -517,6 +542,11 @@ int sffn_last_launches(sffn_handle h, int32_t* launches) {
     if (!h || !launches) return fail(SFFN_ERR_INVALID_ARG, "handle or launches is NULL");
     *launches = h->last_launches;
     return SFFN_OK;
+}
+
+const char* sffn_last_kernel_name(sffn_handle h, int i) {
+    if (!h || i < 0 || i >= h->last_launches || i >= 8 || !h->last_names[i]) return "";
+    return h->last_names[i];
 }
 
 int sffn_destroy(sffn_handle h) {

@@ -92,12 +92,14 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
+// Waits (suspended, up to a hint of about 1 ms) for the phase with `parity`
+// to complete; false if it has not completed by then.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
@@ -193,6 +195,7 @@ struct GateParams {
     const void* bcm;        // [d_ff][r]      LoPA B rows
     const float* u;         // [n][r]         LoPA x A
     const void* wup;        // [d_ff][d]
+    const void* wdn;        // [d_ff][d]      W_down rows (L2 prefetch of active channels), may be NULL
     int out;                // GateOut
     int force_all;          // dense FFN: every channel is listed
     float tau;              // threshold
@@ -236,6 +239,28 @@ struct DownParams {
     void* y;                // [n][d] T
     int chunks;             // chunk CTAs per column slice (grid.y), each a run of gate segments
     int* status;            // sticky device status word (bit set on a failed check)
+};
+
+struct DecodeParams {
+    const void* x;          // [n][d] T, n <= the token tile
+    int n, d, d_ff, r;
+    const void* wg;         // [d_ff][d]   dense gate rows
+    const void* bcm;        // [d_ff][r]   LoPA B rows
+    const float* u;         // [n][r]      LoPA x A
+    const void* wup;        // [d_ff][d]
+    const void* wdn;        // [d_ff][d]
+    float tau;
+    int cpb, mw;
+    int* lst_idx;
+    float* lst_h;           // [d_ff][n]
+    uint32_t* lst_mask;     // [d_ff][mw]
+    int* seg_count;         // [CTAs]
+    int sb, nb;             // streamed piece bytes, pieces in flight per streaming warp
+    int* status;
+    float* part;            // [CTAs][n][d] per-CTA partials of y
+    unsigned* tickets;      // [2] zero between forwards
+    int reducers;           // CTAs that sum the partials (d / reducers a multiple of 4)
+    void* y;                // [n][d] T
 };
 
 // Bits of the device status word.
@@ -282,6 +307,12 @@ size_t gate_smem_bytes(int wdtype, int nt, int d, int r, int gate_kind, int cpb,
 cudaError_t launch_gate_stream(int wdtype, const GateParams& p, int nt, int gate_kind, int grid, size_t smem,
                                cudaStream_t s, bool pdl);
 size_t gate_stream_smem_bytes(int nt, int d, int r, int gate_kind, int cpb, int mw, int sb, int nb);
+// Largest dynamic shared memory a CTA may use on sm_100 (227 KB).
+constexpr size_t kMaxSmemPerCta = 232448;
+// Streaming geometry of the gate kernel for token tile nt: piece bytes *sb and
+// pieces per warp *nb maximising the bytes in flight (ties: more pieces) within
+// kMaxSmemPerCta; false if even two 2 KB pieces per warp do not fit.
+bool gate_stream_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* sb, int* nb, size_t* smem);
 cudaError_t launch_lopa_u(int wdtype, const LopaUParams& p, int nt, cudaStream_t s, bool pdl);
 constexpr int kLopaRowsPerCta = 2;
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s, bool pdl);
@@ -291,5 +322,9 @@ size_t down_smem_bytes(int wdtype, int nt, int nseg, int cpb);
 int down_slice_cols(int wdtype);
 cudaError_t launch_transpose(int wdtype, const void* src, void* dst, int rows, int cols,
                              cudaStream_t s);
+bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* sb, int* nb, size_t* smem);
+cudaError_t launch_decode(int wdtype, const DecodeParams& p, int nt, int gate_kind, int grid, size_t smem,
+                          cudaStream_t s, bool pdl);
+constexpr int kDecodeMaxTokens = 4;   // the fused decode path takes up to this many tokens
 
 }  // namespace sffn

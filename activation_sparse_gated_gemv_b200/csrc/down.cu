@@ -97,11 +97,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_down(const DownParams p) {
     const T* wcol = wdn + col0 + tc * V;
     for (int t0 = 0; t0 < p.n; t0 += NT) {
         const int nt = min(NT, p.n - t0);
-        float acc[NT][V];
+        float2 acc[NT][V / 2];
 #pragma unroll
         for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int e = 0; e < V; ++e) acc[t][e] = 0.f;
+            for (int e = 0; e < V / 2; ++e) acc[t][e] = make_float2(0.f, 0.f);
         for (int i0 = rg; i0 < rows; i0 += UB * RG) {
             uint4 w[UB];
             float h[UB][NT];
@@ -119,16 +119,20 @@ __global__ void __launch_bounds__(kThreads, 2) k_down(const DownParams p) {
                 float wf[V];
                 unpack<T>(w[u], wf);
 #pragma unroll
-                for (int t = 0; t < NT; ++t)
+                for (int t = 0; t < NT; ++t) {
+                    const float2 hh = make_float2(h[u][t], h[u][t]);
 #pragma unroll
-                    for (int e = 0; e < V; ++e) acc[t][e] = fmaf(h[u][t], wf[e], acc[t][e]);
+                    for (int e = 0; e < V / 2; ++e)
+                        acc[t][e] = __ffma2_rn(make_float2(wf[2 * e], wf[2 * e + 1]), hh, acc[t][e]);
+                }
             }
         }
         __syncthreads();
 #pragma unroll
         for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int e = 0; e < V; ++e) red[((size_t)rg * NT + t) * kSliceCols + tc * V + e] = acc[t][e];
+            for (int e = 0; e < V / 2; ++e)
+                *reinterpret_cast<float2*>(red + ((size_t)rg * NT + t) * kSliceCols + tc * V + 2 * e) = acc[t][e];
         __syncthreads();
         for (int i = threadIdx.x; i < NT * (kSliceCols / 4); i += kThreads) {
             const int t = i / (kSliceCols / 4), c = (i - t * (kSliceCols / 4)) * 4;
@@ -169,19 +173,21 @@ __global__ void __launch_bounds__(kThreads, 2) k_down(const DownParams p) {
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
         if (ok) {
             const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)t * p.d + col0 + c);
-            int ch = grp;
-            for (; ch + 15 * G < p.chunks; ch += 16 * G) {
+            // 16 loads in flight per batch; the last batch is predicated, so a
+            // short chunk list still costs a single round trip.
+            for (int ch = grp; ch < p.chunks; ch += 16 * G) {
                 float4 v[16];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) v[q] = __ldcg(src + (size_t)(ch + q * G) * stride);
+                for (int q = 0; q < 16; ++q) {
+                    const int c2 = ch + q * G;
+                    v[q] = c2 < p.chunks ? __ldcg(src + (size_t)c2 * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
-                    s.x += v[q].x; s.y += v[q].y; s.z += v[q].z; s.w += v[q].w;
+                    if (ch + q * G < p.chunks) {
+                        s.x += v[q].x; s.y += v[q].y; s.z += v[q].z; s.w += v[q].w;
+                    }
                 }
-            }
-            for (; ch < p.chunks; ch += G) {
-                const float4 v = __ldcg(src + (size_t)ch * stride);
-                s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
             }
         }
         if (G > 1) {

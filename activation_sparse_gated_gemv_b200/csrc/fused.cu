@@ -1,0 +1,518 @@
+// Fused decode path (threshold selection, a few tokens): one kernel streams
+// the gate, selects, takes the up dots, adds the CTA's share of the down
+// projection and sums the per-CTA partials.
+//
+// "Model Casting and Low-Parameter Gating" (abstract): the gating matrix is
+// evaluated first and the two other matrices are touched only for channels
+// whose activation is non-zero.  Here those touches overlap the gate stream:
+//
+// k_decode, one CTA per SM over its channel range [c0, c0 + cpb), 16 warps:
+//   * warps 0..13 stream the CTA's gate rows (dense W_gate, or LoPA's B) through
+//     per-warp rings of bulk copies (TMA engine, mbarriers) and leave per-piece
+//     dot products in shared memory.  When a row's last piece is in, the warp
+//     that finished it adds the pieces in order (z), selects (z > tau), and for
+//     an active channel pulls its W_down row into L2 and queues the channel;
+//   * warps 14 and 15 take queued channels at once and compute the up dot
+//     <x, W_up[:,k]> and h = (z - tau) u (the streaming warps join them when
+//     their pieces are done), so the W_up rows are read while the gate streams;
+//   * after a barrier the active channels are compacted in ascending order
+//     and every thread adds, for its 8 (or 4) output columns, h_k W_down[k,:]
+//     over that ordered list (rows mostly in L2 by now), and stores the CTA's
+//     fp32 partial of y.
+//   * each CTA writes its partial and takes a ticket; the last few CTAs sum
+//     the partials of a column slice each, in CTA order, and store y.
+// Every sum has a fixed order, so y is bitwise reproducible.
+#include "common.cuh"
+#include "dot.cuh"
+
+namespace sffn {
+
+constexpr int kDecWarps = 16;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecStreamWarps = 14;        // the other warps start as up workers
+constexpr int kQueueTail = 0, kQueueHead = 1, kGateDone = 2, kAbort = 3;
+
+struct DecodeSmem {
+    size_t xs, us, zpart, zfin, hs, done, queue, ctr, wl, mask, flag, scan, bars, bufs, total;
+};
+__host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, int gate_kind, int cpb, int mw,
+                                                         int sb, int nb) {
+    DecodeSmem L;
+    const int glen = gate_kind == kGateLopa ? r : d;
+    const int rb = glen * 4;                      // fp32 rows: an upper bound on the part count
+    const int ppr = rb <= sb ? 1 : (rb + sb - 1) / sb + 1;
+    size_t o = 0;
+    L.xs = o;    o += (size_t)nt * d * sizeof(float);
+    L.us = o;    o += gate_kind == kGateLopa ? (size_t)nt * r * sizeof(float) : 0;
+    L.zpart = o; o += (size_t)cpb * ppr * nt * sizeof(float);
+    L.zfin = o;  o += (size_t)cpb * nt * sizeof(float);
+    L.hs = o;    o += (size_t)cpb * nt * sizeof(float);
+    L.done = o;  o += (size_t)cpb * sizeof(int);
+    L.queue = o; o += (size_t)cpb * sizeof(int);
+    L.ctr = o;   o += 4 * sizeof(int);
+    L.wl = o;    o += (size_t)cpb * sizeof(int);
+    L.mask = o;  o += (size_t)cpb * mw * sizeof(uint32_t);
+    L.flag = o;  o += ((size_t)cpb + 15) & ~(size_t)15;
+    L.scan = o;  o += 48 * sizeof(int);
+    o = (o + 15) & ~(size_t)15;
+    L.bars = o;  o += (size_t)kDecStreamWarps * nb * sizeof(uint64_t);
+    o = (o + 127) & ~(size_t)127;
+    L.bufs = o;  o += (size_t)kDecStreamWarps * nb * sb;
+    L.total = o;
+    return L;
+}
+
+template <class T, int NT, int GATE>
+__global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p) {
+    constexpr int V = Elem<T>::kVec;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c0 = blockIdx.x * p.cpb;
+    const int nslots = max(0, min(p.cpb, p.d_ff - c0));
+    const int n = p.n;                                  // n <= NT
+    const DecodeSmem L = decode_smem_layout(NT, p.d, p.r, GATE, p.cpb, p.mw, p.sb, p.nb);
+    float* xs = reinterpret_cast<float*>(smem + L.xs);
+    float* us = reinterpret_cast<float*>(smem + L.us);
+    float* zpart = reinterpret_cast<float*>(smem + L.zpart);
+    float* zfin = reinterpret_cast<float*>(smem + L.zfin);
+    float* hs = reinterpret_cast<float*>(smem + L.hs);
+    int* done = reinterpret_cast<int*>(smem + L.done);
+    int* queue = reinterpret_cast<int*>(smem + L.queue);
+    int* ctr = reinterpret_cast<int*>(smem + L.ctr);
+    int* wl = reinterpret_cast<int*>(smem + L.wl);
+    uint32_t* smask = reinterpret_cast<uint32_t*>(smem + L.mask);
+    uint8_t* flag = reinterpret_cast<uint8_t*>(smem + L.flag);
+    int* scan_sh = reinterpret_cast<int*>(smem + L.scan);
+    const bool streamer = warp < kDecStreamWarps;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + (streamer ? warp : 0) * p.nb;
+    unsigned char* bufs = smem + L.bufs + (size_t)(streamer ? warp : 0) * p.nb * p.sb;
+
+    const int glen = GATE == kGateLopa ? p.r : p.d;
+    const float* gx = GATE == kGateLopa ? us : xs;
+    const int rb = glen * (int)sizeof(T);
+    const int cpr = glen / V;
+    const T* wup = static_cast<const T*>(p.wup);
+    const T* wdn = static_cast<const T*>(p.wdn);
+    const char* gbase = reinterpret_cast<const char*>(static_cast<const T*>(GATE == kGateLopa ? p.bcm : p.wg) +
+                                                      (size_t)c0 * glen);
+    int rpp, ppr, pb;
+    if (rb <= p.sb) {
+        const int per_warp = (nslots + kDecStreamWarps - 1) / kDecStreamWarps;
+        rpp = max(1, min(p.sb / rb, per_warp));
+        ppr = 1;
+        pb = rpp * rb;
+    } else {
+        rpp = 1;
+        ppr = (rb + p.sb - 1) / p.sb;
+        pb = ((rb + ppr - 1) / ppr + 15) & ~15;
+        ppr = (rb + pb - 1) / pb;
+    }
+    const int npieces = rb <= p.sb ? (nslots + rpp - 1) / rpp : nslots * ppr;
+    const int w0 = streamer ? (int)((long long)npieces * warp / kDecStreamWarps) : 0;
+    const int wcount = streamer ? (int)((long long)npieces * (warp + 1) / kDecStreamWarps) - w0 : 0;
+    const uint64_t pol = l2_evict_first();
+
+    // Cursor over this warp's pieces (w0 + j): row group g, part, ring slot, parity.
+    int ig = rb <= p.sb ? w0 : w0 / ppr, ipart = rb <= p.sb ? 0 : w0 - (w0 / ppr) * ppr, ibuf = 0;
+    int issued = 0;
+    auto issue_next = [&]() {
+        uint32_t bytes;
+        const char* src;
+        if (rb <= p.sb) {
+            const int r0 = ig * rpp;
+            bytes = (uint32_t)(min(rpp, nslots - r0) * rb);
+            src = gbase + (size_t)r0 * rb;
+        } else {
+            const int off = ipart * pb;
+            bytes = (uint32_t)min(pb, rb - off);
+            src = gbase + (size_t)ig * rb + off;
+        }
+        if (lane == 0) {
+            mbar_expect_tx(bars + ibuf, bytes);
+            bulk_load(bufs + (size_t)ibuf * p.sb, src, bytes, bars + ibuf, pol);
+        }
+        if (++ibuf == p.nb) ibuf = 0;
+        if (++ipart >= ppr) {
+            ipart = 0;
+            ++ig;
+        }
+        ++issued;
+    };
+
+    if (streamer) {
+        if (lane == 0) {
+            for (int b = 0; b < p.nb; ++b) mbar_init(bars + b, 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        // Weights never depend on an earlier kernel: fill the ring before the
+        // PDL wait, so the pieces land while the previous kernel finishes.
+        while (issued < min(p.nb, wcount)) issue_next();
+        __syncwarp();
+    }
+
+    griddep_wait();
+    griddep_launch_dependents();
+
+    for (int i = threadIdx.x; i < p.cpb; i += kDecThreads) {
+        flag[i] = 0;
+        done[i] = 0;
+        queue[i] = 0;
+    }
+    for (int i = threadIdx.x; i < p.cpb * p.mw; i += kDecThreads) smask[i] = 0u;
+    if (threadIdx.x < 4) ctr[threadIdx.x] = 0;
+    stage_rows<T, T, NT>(xs, static_cast<const T*>(p.x), p.d, 0, n);
+    if (GATE == kGateLopa) stage_rows<T, float, NT>(us, p.u, p.r, 0, n);
+    if (streamer) {
+        while (issued < min(p.nb, wcount)) issue_next();
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // Row s is complete: z from its parts in order, select, queue it.
+    auto finalize = [&](int s) {                         // lane 0 only
+        __threadfence_block();
+        uint32_t tokmask = 0u;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            float z = 0.f;
+            for (int q = 0; q < ppr; ++q) z += zpart[(s * ppr + q) * NT + t];
+            zfin[s * NT + t] = z;
+            if (t < n && z > p.tau) tokmask |= 1u << t;
+        }
+        if (tokmask) {
+            flag[s] = 1;
+            smask[s * p.mw] = tokmask;                   // n <= 4: tokens sit in mask word 0
+            bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+            const int slot = atomicAdd(ctr + kQueueTail, 1);
+            __threadfence_block();
+            reinterpret_cast<volatile int*>(queue)[slot] = s + 1;
+        }
+    };
+
+    // ---- streaming warps
+    if (streamer) {
+        int cbuf = 0, cpar = 0;
+        int g = rb <= p.sb ? w0 : w0 / ppr, part = rb <= p.sb ? 0 : w0 - (w0 / ppr) * ppr;
+        bool abort = false;
+        int abort_at = 0;
+        for (int j = 0; j < wcount; ++j) {
+            if (!abort && !mbar_wait_warp(bars + cbuf, (uint32_t)cpar)) {
+                abort = true;
+                abort_at = j;
+                if (lane == 0) {
+                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                    atomicExch(ctr + kAbort, 1);
+                }
+            }
+            if (!abort) {
+                const unsigned char* buf = bufs + (size_t)cbuf * p.sb;
+                if (rb <= p.sb) {
+                    const int r0 = g * rpp, cnt = min(rpp, nslots - r0);
+                    for (int q = 0; q < cnt; ++q) {
+                        float2 v2[NT];
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) v2[t] = make_float2(0.f, 0.f);
+                        piece_dot<T, NT>(buf + (size_t)q * rb, cpr, 0, gx, glen, v2);
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) {
+                            const float v = warp_sum(v2[t].x + v2[t].y);
+                            if (lane == t) zpart[(r0 + q) * NT + t] = v;
+                        }
+                        __syncwarp();
+                        if (lane == 0) finalize(r0 + q);
+                    }
+                } else {
+                    const int off = part * pb;
+                    float2 v2[NT];
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) v2[t] = make_float2(0.f, 0.f);
+                    piece_dot<T, NT>(buf, min(pb, rb - off) >> 4, off >> 4, gx, glen, v2);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        const float v = warp_sum(v2[t].x + v2[t].y);
+                        if (lane == t) zpart[(g * ppr + part) * NT + t] = v;
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence_block();
+                        if (atomicAdd(done + g, 1) == ppr - 1) finalize(g);
+                    }
+                }
+                __syncwarp();
+                if (issued < wcount) {
+                    if (lane == 0) fence_proxy_async();
+                    issue_next();
+                }
+            }
+            if (++cbuf == p.nb) {
+                cbuf = 0;
+                cpar ^= 1;
+            }
+            if (++part >= ppr) {
+                part = 0;
+                ++g;
+            }
+        }
+        if (abort) {
+            for (int q = abort_at; q < issued; ++q)
+                mbar_wait_warp(bars + (q % p.nb), (uint32_t)((q / p.nb) & 1));
+        }
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            atomicAdd(ctr + kGateDone, 1);
+        }
+    }
+
+    // ---- up workers (all warps once their streaming is done)
+    for (;;) {
+        int i = 0;
+        if (lane == 0) i = atomicAdd(ctr + kQueueHead, 1);
+        i = __shfl_sync(0xffffffffu, i, 0);
+        if (i >= nslots) break;
+        int s = 0;
+        if (lane == 0) {
+            const unsigned long long t0 = globaltimer_ns();
+            for (;;) {
+                s = reinterpret_cast<volatile int*>(queue)[i];
+                if (s) break;
+                const volatile int* vc = ctr;
+                if ((vc[kGateDone] == kDecStreamWarps && vc[kQueueTail] <= i) || vc[kAbort]) break;
+                __nanosleep(64);
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                    atomicExch(ctr + kAbort, 1);
+                    break;
+                }
+            }
+            __threadfence_block();
+        }
+        s = __shfl_sync(0xffffffffu, s, 0);
+        if (!s) break;
+        --s;
+        __syncwarp();
+        const int k = c0 + s;
+        float u[NT];
+        warp_dot_global<T, NT>(wup + (size_t)k * p.d, p.d / V, xs, p.d, u);
+        const uint32_t tokmask = smask[s * p.mw];
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+            if (lane == t && t < n) {
+                const float h = ((tokmask >> t) & 1u) ? (zfin[s * NT + t] - p.tau) * u[t] : 0.f;
+                hs[s * NT + t] = h;
+                p.lst_h[(size_t)k * n + t] = h;
+            }
+    }
+    __syncthreads();
+
+    // ---- the CTA's list (ascending, one warp, ballots), then its share of the down projection
+    if (warp == 0) {
+        int cnt = 0;
+        for (int base = 0; base < nslots; base += 32) {
+            const int sl = base + lane;
+            const bool f = sl < nslots && flag[sl];
+            const unsigned m = __ballot_sync(0xffffffffu, f);
+            if (f) wl[cnt + __popc(m & ((1u << lane) - 1u))] = sl;
+            cnt += __popc(m);
+        }
+        if (lane == 0) scan_sh[0] = cnt;
+    }
+    __syncthreads();
+    const int tot = scan_sh[0];
+    for (int i = threadIdx.x; i < tot; i += kDecThreads) {
+        const int sl = wl[i];
+        p.lst_idx[c0 + i] = c0 + sl;
+        for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + sl) * p.mw + w] = smask[sl * p.mw + w];
+    }
+    if (threadIdx.x == 0) p.seg_count[blockIdx.x] = tot;
+
+    constexpr int UB = 8;
+    const int cpd = p.d / V;                              // 16-byte chunks per output row
+    for (int cch = threadIdx.x; cch < cpd; cch += kDecThreads) {
+        float2 acc[NT][V / 2];
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int e = 0; e < V / 2; ++e) acc[t][e] = make_float2(0.f, 0.f);
+        for (int i0 = 0; i0 < tot; i0 += UB) {
+            uint4 w[UB];
+#pragma unroll
+            for (int u2 = 0; u2 < UB; ++u2) {
+                const int i = i0 + u2;
+                w[u2] = i < tot ? ld_stream(wdn + (size_t)(c0 + wl[i]) * p.d + (size_t)cch * V)
+                                : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u2 = 0; u2 < UB; ++u2) {
+                const int i = i0 + u2;
+                if (i < tot) {
+                    float wf[V];
+                    unpack<T>(w[u2], wf);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        const float h = hs[wl[i] * NT + t];
+                        const float2 hh = make_float2(h, h);
+#pragma unroll
+                        for (int e = 0; e < V / 2; ++e)
+                            acc[t][e] = __ffma2_rn(make_float2(wf[2 * e], wf[2 * e + 1]), hh, acc[t][e]);
+                    }
+                }
+            }
+        }
+        for (int t = 0; t < n; ++t) {
+            float* dst = p.part + ((size_t)blockIdx.x * n + t) * p.d + (size_t)cch * V;
+#pragma unroll
+            for (int e = 0; e < V / 2; e += 2)
+                *reinterpret_cast<float4*>(dst + 2 * e) =
+                    make_float4(acc[t][e].x, acc[t][e].y, acc[t][e + 1].x, acc[t][e + 1].y);
+        }
+    }
+
+    // ---- cross-CTA sum.  Each CTA takes a ticket once its partial is out; the
+    // last `reducers` CTAs wait (bounded) until every partial is written, then
+    // each adds a column slice over all CTAs in CTA order and stores y.  They
+    // wait only on CTAs that are already running, so this cannot deadlock.
+    __threadfence();
+    __syncthreads();
+    const int parts = gridDim.x;
+    const int reducers = p.reducers;
+    if (threadIdx.x == 0) scan_sh[1] = (int)atomicAdd(p.tickets, 1u);
+    __syncthreads();
+    const int rank = scan_sh[1] - (parts - reducers);
+    if (rank < 0) return;
+    if (threadIdx.x == 0) {
+        const unsigned long long t0 = globaltimer_ns();
+        int ok = 1;
+        while (*reinterpret_cast<volatile unsigned*>(p.tickets) < (unsigned)parts) {
+            __nanosleep(128);
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(p.status, (int)kStatusWaitTimeout);
+                ok = 0;
+                break;
+            }
+        }
+        scan_sh[2] = ok;
+        __threadfence();
+    }
+    __syncthreads();
+    if (scan_sh[2]) {
+        const int cols = p.d / reducers;                    // a multiple of 4
+        const int col0 = rank * cols;
+        const int c4n = cols / 4;
+        const int items = n * c4n;
+        const int G = items >= kDecThreads ? 1 : kDecThreads / items;
+        const int per_round = kDecThreads / G;
+        float4* gsum = reinterpret_cast<float4*>(smem + L.bufs);   // the streaming ring, idle now
+        const size_t stride = (size_t)n * p.d / 4;
+        T* y = static_cast<T*>(p.y);
+        for (int base = 0; base < items; base += per_round) {
+            const int item = base + (int)threadIdx.x % per_round;
+            const int grp = (int)threadIdx.x / per_round;
+            const int t = item / c4n, c = col0 + (item - t * c4n) * 4;
+            const bool ok = item < items && grp < G;
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (ok) {
+                const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)t * p.d + c);
+                for (int b = grp; b < parts; b += 16 * G) {
+                    float4 v[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int b2 = b + q * G;
+                        v[q] = b2 < parts ? __ldcg(src + (size_t)b2 * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (b + q * G < parts) {
+                            sum.x += v[q].x; sum.y += v[q].y; sum.z += v[q].z; sum.w += v[q].w;
+                        }
+                }
+            }
+            if (G > 1) {
+                __syncthreads();
+                gsum[threadIdx.x] = sum;
+                __syncthreads();
+                if (grp == 0 && ok)
+                    for (int q = 1; q < G; ++q) {
+                        const float4 v = gsum[q * per_round + (int)threadIdx.x % per_round];
+                        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+                    }
+            }
+            if (grp == 0 && ok) {
+                T* dst = y + (size_t)t * p.d + c;
+                dst[0] = from_f32<T>(sum.x);
+                dst[1] = from_f32<T>(sum.y);
+                dst[2] = from_f32<T>(sum.z);
+                dst[3] = from_f32<T>(sum.w);
+            }
+        }
+    }
+    // The last reducer to finish resets the tickets for the next forward.
+    __syncthreads();
+    if (threadIdx.x == 0 && atomicAdd(p.tickets + 1, 1u) == (unsigned)reducers - 1u) {
+        p.tickets[0] = 0u;
+        p.tickets[1] = 0u;
+        __threadfence();
+    }
+}
+
+// ---------------------------------------------------------------------------
+
+size_t decode_smem_bytes(int nt, int d, int r, int gate_kind, int cpb, int mw, int sb, int nb) {
+    return decode_smem_layout(nt, d, r, gate_kind, cpb, mw, sb, nb).total;
+}
+
+bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* sb, int* nb, size_t* smem) {
+    int best_sb = 0, best_nb = 0;
+    for (int cand_sb : {8192, 4096, 2048})
+        for (int cand_nb = 2; cand_nb <= 4; ++cand_nb) {
+            if (decode_smem_bytes(nt, d, r, gate_kind, cpb, mw, cand_sb, cand_nb) > kMaxSmemPerCta) continue;
+            const long cur = (long)cand_sb * cand_nb, best = (long)best_sb * best_nb;
+            if (cur > best || (cur == best && cand_nb > best_nb)) {
+                best_sb = cand_sb;
+                best_nb = cand_nb;
+            }
+        }
+    if (!best_sb) return false;
+    *sb = best_sb;
+    *nb = best_nb;
+    *smem = decode_smem_bytes(nt, d, r, gate_kind, cpb, mw, best_sb, best_nb);
+    return true;
+}
+
+template <class T, int NT, int GATE>
+static cudaError_t launch_decode_t(const DecodeParams& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
+    auto kern = k_decode<T, NT, GATE>;
+    static SmemAttrCache cache;
+    cudaError_t e = ensure_smem(kern, smem, cache);
+    if (e != cudaSuccess) return e;
+    return launch_ex(kern, dim3(grid), dim3(kDecThreads), smem, s, pdl, p);
+}
+
+template <class T, int NT>
+static cudaError_t launch_decode_nt(const DecodeParams& p, int gate_kind, int grid, size_t smem, cudaStream_t s,
+                                    bool pdl) {
+    return gate_kind == kGateLopa ? launch_decode_t<T, NT, kGateLopa>(p, grid, smem, s, pdl)
+                                  : launch_decode_t<T, NT, kGateDense>(p, grid, smem, s, pdl);
+}
+
+cudaError_t launch_decode(int wdtype, const DecodeParams& p, int nt, int gate_kind, int grid, size_t smem,
+                          cudaStream_t s, bool pdl) {
+    if (p.n > nt || p.mw < 1 || p.sb <= 0 || p.sb % 16 || p.nb <= 0) return cudaErrorInvalidValue;
+    if (wdtype == 0) {
+        switch (nt) {
+            case 1: return launch_decode_nt<bf16, 1>(p, gate_kind, grid, smem, s, pdl);
+            case 2: return launch_decode_nt<bf16, 2>(p, gate_kind, grid, smem, s, pdl);
+            case 4: return launch_decode_nt<bf16, 4>(p, gate_kind, grid, smem, s, pdl);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (nt) {
+        case 1: return launch_decode_nt<float, 1>(p, gate_kind, grid, smem, s, pdl);
+        case 2: return launch_decode_nt<float, 2>(p, gate_kind, grid, smem, s, pdl);
+        case 4: return launch_decode_nt<float, 4>(p, gate_kind, grid, smem, s, pdl);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace sffn

@@ -26,149 +26,55 @@
 // the rank-r product A B).  A split-d grid writes partial sums; the last CTA of
 // each column group (ticket counter) adds them in split order.
 #include "common.cuh"
+#include "dot.cuh"
 
 namespace sffn {
 
-constexpr int kStashRows = 16;   // rows per streamed piece, at most
-
-// Shared-memory x (and LoPA u) rows are fp32.  For 8-wide (bf16) chunks a row
-// of `len` floats holds the first halves of all chunks, then the second
-// halves, so consecutive lanes' 16-byte reads hit consecutive banks.
-template <int V>
-__device__ __forceinline__ int xpos(int len, int c, int e) {
-    if (V == 8) return e < 4 ? c * 4 + e : (len >> 1) + c * 4 + (e - 4);
-    return c * 4 + e;
-}
-
-// <16-byte weight chunk, x chunk c of one token row in shared memory>, added
-// into two accumulators (even and odd elements) to halve the FMA chain.
-template <class WT>
-__device__ __forceinline__ void chunk_dot(const uint4& w, const float* xrow, int len, int c, float& a0,
-                                          float& a1) {
-    constexpr int V = Elem<WT>::kVec;
-    float wf[V];
-    unpack<WT>(w, wf);
-    const float4 a = *reinterpret_cast<const float4*>(xrow + xpos<V>(len, c, 0));
-    a0 = fmaf(wf[0], a.x, a0);
-    a1 = fmaf(wf[1], a.y, a1);
-    a0 = fmaf(wf[2], a.z, a0);
-    a1 = fmaf(wf[3], a.w, a1);
-    if (V == 8) {
-        const float4 b = *reinterpret_cast<const float4*>(xrow + xpos<V>(len, c, 4));
-        a0 = fmaf(wf[4], b.x, a0);
-        a1 = fmaf(wf[5], b.y, a1);
-        a0 = fmaf(wf[6], b.z, a0);
-        a1 = fmaf(wf[7], b.w, a1);
-    }
-}
-
-// Stage tokens [t0, t0 + nt) of a global row-major n x len array (type XT) as
-// fp32 rows of `len` in shared memory (chunk layout of weight type WT); rows
-// nt..NT-1 are zero.  16-byte loads, all of a thread's loads issued before any
-// store (a handful of round trips at most).  All threads of the block take part.
-template <class WT, class XT, int NT>
-__device__ __forceinline__ void stage_rows(float* dst, const XT* src, int len, int t0, int nt) {
-    constexpr int V = Elem<WT>::kVec;
-    constexpr int XV = 16 / sizeof(XT);                 // elements per 16-byte load
-    constexpr int U = 4;
-    const int per_row = len / XV;                        // len is a multiple of 8
-    const int total = NT * per_row;
-    for (int base = threadIdx.x; base < total; base += U * blockDim.x) {
-        uint4 v[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int i = base + u * blockDim.x;
-            const int t = i / per_row;
-            v[u] = (i < total && t < nt)
-                       ? *reinterpret_cast<const uint4*>(src + (size_t)(t0 + t) * len + (size_t)(i - t * per_row) * XV)
-                       : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int i = base + u * blockDim.x;
-            if (i < total) {
-                const int t = i / per_row, j0 = (i - t * per_row) * XV;
-                float f[XV];
-                unpack<XT>(v[u], f);
-#pragma unroll
-                for (int e = 0; e < XV; ++e) {
-                    const int j = j0 + e;
-                    dst[t * len + xpos<V>(len, j / V, j % V)] = f[e];
-                }
-            }
-        }
-    }
-}
-
-// acc[t] = <row, x_t> over a global row of cpr 16-byte chunks, read with
-// L1-bypassing loads (16 in flight per lane); every lane ends with the sums.
-template <class WT, int NT>
-__device__ __forceinline__ void warp_dot_global(const WT* __restrict__ row, int cpr, const float* xs, int len,
-                                                float (&acc)[NT]) {
-    constexpr int UB = NT >= 4 ? 8 : 16;
-    const int lane = threadIdx.x & 31;
-    float acc1[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = acc1[t] = 0.f;
-    for (int cb = lane; cb < cpr; cb += 32 * UB) {
-        uint4 wv[UB];
-#pragma unroll
-        for (int u = 0; u < UB; ++u) {
-            const int c = cb + 32 * u;
-            wv[u] = c < cpr ? ld_stream(row + (size_t)c * Elem<WT>::kVec) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < UB; ++u) {
-            const int c = cb + 32 * u;
-            if (c < cpr) {
-#pragma unroll
-                for (int t = 0; t < NT; ++t) chunk_dot<WT>(wv[u], xs + t * len, len, c, acc[t], acc1[t]);
-            }
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = warp_sum(acc[t] + acc1[t]);
-}
-
-// Per-lane partial of <piece, x_t> over chunks [0, nch) of a shared-memory
-// piece whose chunk 0 is chunk `coff` of the row.
-template <class WT, int NT>
-__device__ __forceinline__ void piece_dot(const unsigned char* piece, int nch, int coff, const float* xs, int len,
-                                          float (&acc)[NT], float (&acc1)[NT]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll 2
-    for (int c = lane; c < nch; c += 32) {
-        const uint4 w = reinterpret_cast<const uint4*>(piece)[c];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) chunk_dot<WT>(w, xs + t * len, len, coff + c, acc[t], acc1[t]);
-    }
-}
+constexpr int kStreamWarps = 16;  // warps of a streaming gate CTA (one CTA per SM)
+constexpr int kStreamThreads = kStreamWarps * 32;
 
 // ---------------------------------------------------------------------------
 
 struct StreamSmem {
-    size_t xs, us, stash, mask, flag, scan, bars, bufs, total;
+    size_t xs, us, zpart, zfin, wl, mask, flag, scan, bars, bufs, total;
 };
+// zparts: partial gate dots per (slot, part), see k_gate_stream.
 __host__ __device__ inline StreamSmem stream_smem_layout(int nt, int d, int r, int gate_kind, int cpb, int mw,
                                                          int sb, int nb) {
     StreamSmem L;
+    const int glen = gate_kind == kGateLopa ? r : d;
+    const int rb = glen * 4;                      // worst case (fp32 rows) for the part count
+    const int ppr = rb <= sb ? 1 : (rb + sb - 1) / sb + 1;
     size_t o = 0;
     L.xs = o;    o += (size_t)nt * d * sizeof(float);
     L.us = o;    o += gate_kind == kGateLopa ? (size_t)nt * r * sizeof(float) : 0;
-    L.stash = o; o += (size_t)kWarps * kStashRows * nt * sizeof(float);
+    L.zpart = o; o += (size_t)cpb * ppr * nt * sizeof(float);
+    L.zfin = o;  o += (size_t)cpb * nt * sizeof(float);
+    L.wl = o;    o += (size_t)cpb * sizeof(int);
     L.mask = o;  o += (size_t)cpb * mw * sizeof(uint32_t);
     L.flag = o;  o += ((size_t)cpb + 15) & ~(size_t)15;
     L.scan = o;  o += 48 * sizeof(int);
     o = (o + 15) & ~(size_t)15;                      // mbarriers need 8-byte alignment
-    L.bars = o;  o += (size_t)kWarps * nb * sizeof(uint64_t);
+    L.bars = o;  o += (size_t)kStreamWarps * nb * sizeof(uint64_t);
     o = (o + 127) & ~(size_t)127;
-    L.bufs = o;  o += (size_t)kWarps * nb * sb;
+    L.bufs = o;  o += (size_t)kStreamWarps * nb * sb;
     L.total = o;
     return L;
 }
 
+// Two phases per token tile.
+//  Streaming: the CTA's gate rows are cut into pieces (whole rows, or equal
+//  parts of a row); warp w takes a contiguous, balanced range of pieces and
+//  streams it through its own ring of bulk copies; each piece leaves its
+//  per-token dot product (of whole rows, or a part of a row) in shared memory.
+//  No data-dependent work happens here, so every warp keeps streaming.
+//  Finish (after a barrier): z = the sum of a row's parts in part order;
+//  select; prefetch the active channels' W_down rows into L2; spread the rows
+//  that need an up dot evenly over the warps (all their loads in flight at
+//  once); h = (z - tau) u.  The dense FFN (force_all) takes the up dot of every
+//  row.  Finally the CTA's active channels are compacted into its list segment.
 template <class T, int NT, int GATE>
-__global__ void __launch_bounds__(kThreads, 2) k_gate_stream(const GateParams p) {
+__global__ void __launch_bounds__(kStreamThreads, 1) k_gate_stream(const GateParams p) {
     constexpr int V = Elem<T>::kVec;
     extern __shared__ __align__(128) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -177,7 +83,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_gate_stream(const GateParams p)
     const StreamSmem L = stream_smem_layout(NT, p.d, p.r, GATE, p.cpb, p.mw, p.sb, p.nb);
     float* xs = reinterpret_cast<float*>(smem + L.xs);
     float* us = reinterpret_cast<float*>(smem + L.us);
-    float* stash = reinterpret_cast<float*>(smem + L.stash) + warp * kStashRows * NT;
+    float* zpart = reinterpret_cast<float*>(smem + L.zpart);
+    float* zfin = reinterpret_cast<float*>(smem + L.zfin);
+    int* wl = reinterpret_cast<int*>(smem + L.wl);
     uint32_t* smask = reinterpret_cast<uint32_t*>(smem + L.mask);
     uint8_t* flag = reinterpret_cast<uint8_t*>(smem + L.flag);
     int* scan_sh = reinterpret_cast<int*>(smem + L.scan);
@@ -188,192 +96,242 @@ __global__ void __launch_bounds__(kThreads, 2) k_gate_stream(const GateParams p)
     const float* gx = GATE == kGateLopa ? us : xs;                  // what the gate row multiplies
     const int rb = glen * (int)sizeof(T);
     const int cpr = glen / V;
-    const bool alt = p.force_all && GATE == kGateDense && p.out == kOutSelectUp;
     const T* wup = static_cast<const T*>(p.wup);
     const char* gbase = reinterpret_cast<const char*>(static_cast<const T*>(GATE == kGateLopa ? p.bcm : p.wg) +
                                                       (size_t)c0 * glen);
-    const char* ubase = reinterpret_cast<const char*>(wup + (size_t)c0 * p.d);
-    const int wr0 = (int)((long long)nslots * warp / kWarps);
-    const int nrows = (int)((long long)nslots * (warp + 1) / kWarps) - wr0;
+    // pieces: rpp whole rows each, or ppr parts of one row (pb bytes, the last shorter)
     int rpp, ppr, pb;
     if (rb <= p.sb) {
-        rpp = min(p.sb / rb, kStashRows);
+        const int per_warp = (nslots + kStreamWarps - 1) / kStreamWarps;
+        rpp = max(1, min(p.sb / rb, per_warp));
         ppr = 1;
         pb = rpp * rb;
     } else {
         rpp = 1;
         ppr = (rb + p.sb - 1) / p.sb;
         pb = ((rb + ppr - 1) / ppr + 15) & ~15;
+        ppr = (rb + pb - 1) / pb;
     }
-    const int gpieces = rb <= p.sb ? (nrows + rpp - 1) / rpp : nrows * ppr;
-    const int ppt = alt ? 2 * gpieces : gpieces;
+    const int npieces = rb <= p.sb ? (nslots + rpp - 1) / rpp : nslots * ppr;   // per tile
+    const int w0 = (int)((long long)npieces * warp / kStreamWarps);
+    const int wcount = (int)((long long)npieces * (warp + 1) / kStreamWarps) - w0;
     const int ntiles = (p.n + NT - 1) / NT;
-    const int total = ppt * ntiles;
+    const int total = wcount * ntiles;
     const uint64_t pol = l2_evict_first();
 
-    auto issue = [&](int i) {
-        const int ip = i % ppt;
-        const int j = alt ? ip >> 1 : ip;
-        const char* base = ((alt && (ip & 1)) ? ubase : gbase) + (size_t)wr0 * rb;
+    // Cursor over this warp's pieces: (g, part) of piece w0 + j, ring slot and parity.
+    struct Cursor {
+        int j, g, part, buf, parity;
+    };
+    auto start_of = [&](Cursor& c) {
+        c.j = 0;
+        c.g = rb <= p.sb ? w0 : w0 / ppr;
+        c.part = rb <= p.sb ? 0 : w0 - c.g * ppr;
+    };
+    auto advance = [&](Cursor& c) {
+        if (++c.buf == p.nb) {
+            c.buf = 0;
+            c.parity ^= 1;
+        }
+        if (++c.j == wcount) {
+            start_of(c);
+        } else if (++c.part >= ppr) {
+            c.part = 0;
+            ++c.g;
+        }
+    };
+    auto issue = [&](const Cursor& c) {
         uint32_t bytes;
         const char* src;
         if (rb <= p.sb) {
-            const int r0 = j * rpp;
-            bytes = (uint32_t)(min(rpp, nrows - r0) * rb);
-            src = base + (size_t)r0 * rb;
+            const int r0 = c.g * rpp;
+            bytes = (uint32_t)(min(rpp, nslots - r0) * rb);
+            src = gbase + (size_t)r0 * rb;
         } else {
-            const int row = j / ppr, off = (j - row * ppr) * pb;
+            const int off = c.part * pb;
             bytes = (uint32_t)min(pb, rb - off);
-            src = base + (size_t)row * rb + off;
+            src = gbase + (size_t)c.g * rb + off;
         }
-        uint64_t* bar = bars + (i % p.nb);
+        uint64_t* bar = bars + c.buf;
         mbar_expect_tx(bar, bytes);
-        bulk_load(bufs + (size_t)(i % p.nb) * p.sb, src, bytes, bar, pol);
+        bulk_load(bufs + (size_t)c.buf * p.sb, src, bytes, bar, pol);
     };
 
+    Cursor ic{0, 0, 0, 0, 0};
+    start_of(ic);
+    int issued = 0;
     if (lane == 0) {
         for (int b = 0; b < p.nb; ++b) mbar_init(bars + b, 1);
         fence_mbar_init();
-        for (int i = 0; i < min(p.nb, total); ++i) issue(i);
+    }
+    __syncwarp();
+    // Weights never depend on an earlier kernel: start streaming before the
+    // PDL wait -- one piece per warp only, so that x, read right after the
+    // wait, does not queue behind a deep ring of weight traffic.
+    if (total > 0) {
+        if (lane == 0) issue(ic);
+        advance(ic);
+        ++issued;
     }
     __syncwarp();
 
     griddep_wait();
     griddep_launch_dependents();
 
-    for (int i = threadIdx.x; i < p.cpb; i += kThreads) flag[i] = 0;
-    for (int i = threadIdx.x; i < p.cpb * p.mw; i += kThreads) smask[i] = 0u;
-
-    // z -> selection -> (maybe) up -> h, for slot s of this CTA.  u_in: the up
-    // dot when it was streamed (alt), else it is fetched here.
-    auto finish = [&](int s, const float (&z)[NT], const float* u_in, int t0, int nt) {
-        const int k = c0 + s;
-        if (p.out == kOutWriteZ) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (lane == t && t < nt) p.zbuf[(size_t)(t0 + t) * p.d_ff + k] = z[t];
-            return;
-        }
-        uint32_t tokmask = 0u;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) tokmask |= (t < nt && z[t] > p.tau ? 1u : 0u) << t;
-        if (tokmask != 0u || p.force_all) {
-            float u[NT];
-            if (u_in) {
-#pragma unroll
-                for (int t = 0; t < NT; ++t) u[t] = u_in[t];
-            } else {
-                warp_dot_global<T, NT>(wup + (size_t)k * p.d, p.d / V, xs, p.d, u);
-            }
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (lane == t && t < nt)
-                    p.lst_h[(size_t)k * p.n + t0 + t] = ((tokmask >> t) & 1u) ? (z[t] - p.tau) * u[t] : 0.f;
-            if (lane == 0) {
-                flag[s] = 1;
-                smask[s * p.mw + (t0 >> 5)] |= tokmask << (t0 & 31);
-            }
-        } else if (ntiles > 1) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (lane == t && t < nt) p.lst_h[(size_t)k * p.n + t0 + t] = 0.f;
-        }
-    };
+    for (int i = threadIdx.x; i < p.cpb; i += kStreamThreads) flag[i] = 0;
+    for (int i = threadIdx.x; i < p.cpb * p.mw; i += kStreamThreads) smask[i] = 0u;
 
     bool abort = false;
-    int abort_at = 0;
-    int i = 0;
+    int abort_at = 0, consumed = 0;
+    Cursor cc{0, 0, 0, 0, 0};
+    start_of(cc);
     for (int tile = 0; tile < ntiles; ++tile) {
         const int t0 = tile * NT;
         const int nt = min(NT, p.n - t0);
         __syncthreads();
         stage_rows<T, T, NT>(xs, static_cast<const T*>(p.x), p.d, t0, nt);
         if (GATE == kGateLopa) stage_rows<T, float, NT>(us, p.u, p.r, t0, nt);
+        // x is on its way: fill the rest of the ring.
+        for (; tile == 0 && issued < min(p.nb, total); ++issued) {
+            if (lane == 0) issue(ic);
+            advance(ic);
+        }
         __syncthreads();
-        float accz[NT], accu[NT], accz1[NT], accu1[NT];
+
+        // ---- streaming phase
+        // Rows selected while streaming get their W_up and W_down rows pulled
+        // into L2 at once, so the up dots and the down pass read them from L2.
+        const bool prefetch_rows = p.out == kOutSelectUp && !p.force_all;
+        auto prefetch_active = [&](int k) {
+            bulk_prefetch_l2(wup + (size_t)k * p.d, (uint32_t)(p.d * sizeof(T)));
+            if (p.wdn)
+                bulk_prefetch_l2(static_cast<const T*>(p.wdn) + (size_t)k * p.d, (uint32_t)(p.d * sizeof(T)));
+        };
+        float zrow[NT];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) accz[t] = accu[t] = accz1[t] = accu1[t] = 0.f;
-        for (int ip = 0; ip < ppt; ++ip, ++i) {
+        for (int t = 0; t < NT; ++t) zrow[t] = 0.f;
+        for (int j = 0; j < wcount; ++j) {
             if (abort) continue;
-            if (!mbar_wait_warp(bars + (i % p.nb), (uint32_t)((i / p.nb) & 1))) {
+            if (!mbar_wait_warp(bars + cc.buf, (uint32_t)cc.parity)) {
                 abort = true;
-                abort_at = i;
+                abort_at = consumed;
                 if (lane == 0) atomicOr(p.status, (int)kStatusWaitTimeout);
                 continue;
             }
-            const unsigned char* buf = bufs + (size_t)(i % p.nb) * p.sb;
-            const int j = alt ? ip >> 1 : ip;
-            const bool up_piece = alt && (ip & 1);
+            const unsigned char* buf = bufs + (size_t)cc.buf * p.sb;
             if (rb <= p.sb) {
-                const int r0 = j * rpp, cnt = min(rpp, nrows - r0);
+                const int r0 = cc.g * rpp, cnt = min(rpp, nslots - r0);
                 for (int q = 0; q < cnt; ++q) {
-                    float v[NT], v1[NT];
+                    float2 v2[NT];
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) v[t] = v1[t] = 0.f;
-                    piece_dot<T, NT>(buf + (size_t)q * rb, cpr, 0, up_piece ? xs : gx, up_piece ? p.d : glen, v,
-                                     v1);
-#pragma unroll
-                    for (int t = 0; t < NT; ++t) v[t] = warp_sum(v[t] + v1[t]);
-                    const int s = wr0 + r0 + q;
-                    if (!alt) {
-                        finish(s, v, nullptr, t0, nt);
-                    } else if (!up_piece) {
-#pragma unroll
-                        for (int t = 0; t < NT; ++t)
-                            if (lane == t) stash[q * NT + t] = v[t];
-                    } else {
-                        float z[NT];
-#pragma unroll
-                        for (int t = 0; t < NT; ++t) z[t] = stash[q * NT + t];
-                        finish(s, z, v, t0, nt);
-                    }
-                }
-            } else {
-                const int row = j / ppr, part = j - row * ppr, off = part * pb;
-                const int nch = min(pb, rb - off) / 16;
-                if (up_piece) piece_dot<T, NT>(buf, nch, off / 16, xs, p.d, accu, accu1);
-                else piece_dot<T, NT>(buf, nch, off / 16, gx, glen, accz, accz1);
-                if (part == ppr - 1 && (up_piece || !alt)) {
-                    float z[NT], u[NT];
+                    for (int t = 0; t < NT; ++t) v2[t] = make_float2(0.f, 0.f);
+                    piece_dot<T, NT>(buf + (size_t)q * rb, cpr, 0, gx, glen, v2);
+                    bool act = false;
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
-                        z[t] = warp_sum(accz[t] + accz1[t]);
-                        u[t] = warp_sum(accu[t] + accu1[t]);
-                        accz[t] = accu[t] = accz1[t] = accu1[t] = 0.f;
+                        const float v = warp_sum(v2[t].x + v2[t].y);
+                        if (lane == t) zpart[(r0 + q) * NT + t] = v;
+                        act |= t < nt && v > p.tau;
                     }
-                    finish(wr0 + row, z, alt ? u : nullptr, t0, nt);
+                    if (act && lane == 0 && prefetch_rows) prefetch_active(c0 + r0 + q);
+                }
+            } else {
+                const int off = cc.part * pb;
+                float2 v2[NT];
+#pragma unroll
+                for (int t = 0; t < NT; ++t) v2[t] = make_float2(0.f, 0.f);
+                piece_dot<T, NT>(buf, min(pb, rb - off) >> 4, off >> 4, gx, glen, v2);
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const float v = warp_sum(v2[t].x + v2[t].y);
+                    if (lane == t) zpart[(cc.g * ppr + cc.part) * NT + t] = v;
+                    zrow[t] = cc.part == 0 ? v : zrow[t] + v;
+                }
+                // The whole row went through this warp: its z is known now.
+                if (cc.part == ppr - 1 && cc.j >= cc.part && prefetch_rows && lane == 0) {
+                    bool act = false;
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) act |= t < nt && zrow[t] > p.tau;
+                    if (act) prefetch_active(c0 + cc.g);
                 }
             }
             __syncwarp();
-            if (lane == 0 && i + p.nb < total) {
-                fence_proxy_async();
-                issue(i + p.nb);
+            if (issued < total) {
+                if (lane == 0) {
+                    fence_proxy_async();
+                    issue(ic);
+                }
+                advance(ic);
+                ++issued;
+            }
+            advance(cc);
+            ++consumed;
+        }
+        __syncthreads();
+
+        // ---- finish: z, selection, up dots
+        for (int sl = threadIdx.x; sl < nslots; sl += kStreamThreads) {
+            const int k = c0 + sl;
+            uint32_t tokmask = 0u;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                float z = 0.f;
+                for (int q = 0; q < ppr; ++q) z += zpart[(sl * ppr + q) * NT + t];
+                zfin[sl * NT + t] = z;
+                if (t < nt) {
+                    if (p.out == kOutWriteZ) p.zbuf[(size_t)(t0 + t) * p.d_ff + k] = z;
+                    else if (z > p.tau) tokmask |= 1u << t;
+                }
+            }
+            if (p.out == kOutSelectUp && (tokmask || p.force_all)) {
+                // The down pass will read this channel's W_down row: start
+                // bringing it into L2 now.
+                if (tokmask && !flag[sl] && !p.force_all && p.wdn)
+                    bulk_prefetch_l2(static_cast<const T*>(p.wdn) + (size_t)k * p.d, (uint32_t)(p.d * sizeof(T)));
+                flag[sl] = 1;
+                smask[sl * p.mw + (t0 >> 5)] |= tokmask << (t0 & 31);
+            }
+            wl[sl] = (int)tokmask;                      // this tile's selection, read back below
+        }
+        __syncthreads();
+        if (p.out == kOutWriteZ) continue;
+        // rows needing an up dot in this tile, in order
+        int* work = reinterpret_cast<int*>(zpart);     // zpart is free until the next tile
+        const int nwork = block_compact(nslots, [&](int sl) { return wl[sl] != 0 || p.force_all; }, work, scan_sh);
+        for (int i = warp; i < nwork; i += kStreamWarps) {
+            const int sl = work[i], k = c0 + sl;
+            const uint32_t tokmask = (uint32_t)wl[sl];
+            float u[NT];
+            warp_dot_global<T, NT>(wup + (size_t)k * p.d, p.d / V, xs, p.d, u);
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+                if (lane == t && t < nt)
+                    p.lst_h[(size_t)k * p.n + t0 + t] =
+                        ((tokmask >> t) & 1u) ? (zfin[sl * NT + t] - p.tau) * u[t] : 0.f;
+        }
+        if (ntiles > 1 && !p.force_all) {
+            // channels active in another tile only: h = 0 for this tile's tokens
+            for (int i = threadIdx.x; i < nslots * NT; i += kStreamThreads) {
+                const int sl = i / NT, t = i - sl * NT;
+                if (t < nt && wl[sl] == 0) p.lst_h[(size_t)(c0 + sl) * p.n + t0 + t] = 0.f;
             }
         }
+        __syncthreads();
     }
     if (abort) {
-        // Pieces [abort_at, abort_at + nb) were issued and not consumed: give each
-        // a bounded wait so no copy lands after the CTA has gone.
-        for (int q = abort_at; q < min(abort_at + p.nb, total); ++q)
+        // Pieces [abort_at, issued) were issued and not consumed: give each a
+        // bounded wait so no copy lands after the CTA has gone.
+        for (int q = abort_at; q < issued; ++q)
             mbar_wait_warp(bars + (q % p.nb), (uint32_t)((q / p.nb) & 1));
     }
     if (p.out == kOutWriteZ) return;
 
     __syncthreads();
-    const int per = (nslots + kThreads - 1) / kThreads;
-    const int sb0 = threadIdx.x * per;
-    int cnt = 0;
-    for (int q = 0; q < per; ++q)
-        if (sb0 + q < nslots && flag[sb0 + q]) ++cnt;
-    int tot = 0;
-    int pos = block_exclusive_scan(cnt, &tot, scan_sh);
-    for (int q = 0; q < per; ++q) {
-        const int s = sb0 + q;
-        if (s < nslots && flag[s]) {
-            p.lst_idx[c0 + pos] = c0 + s;
-            for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + s) * p.mw + w] = smask[s * p.mw + w];
-            ++pos;
-        }
+    const int tot = block_compact(nslots, [&](int sl) { return flag[sl] != 0; }, wl, scan_sh);
+    for (int i = threadIdx.x; i < tot; i += kStreamThreads) {
+        const int sl = wl[i];
+        p.lst_idx[c0 + i] = c0 + sl;
+        for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + sl) * p.mw + w] = smask[sl * p.mw + w];
     }
     if (threadIdx.x == 0) p.seg_count[blockIdx.x] = tot;
 }
@@ -505,9 +463,9 @@ __global__ void __launch_bounds__(kThreads) k_lopa_u(const LopaUParams p) {
 
     for (int t0 = 0; t0 < p.n; t0 += NT) {
         const int nt = min(NT, p.n - t0);
-        float a0[NT], a1[NT];
+        float2 a2[NT];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) a0[t] = a1[t] = 0.f;
+        for (int t = 0; t < NT; ++t) a2[t] = make_float2(0.f, 0.f);
         for (int cb = tr; cb < cpr; cb += UB * TPR) {
             uint4 w[UB], xv[UB][NT];
 #pragma unroll
@@ -522,23 +480,20 @@ __global__ void __launch_bounds__(kThreads) k_lopa_u(const LopaUParams p) {
             }
 #pragma unroll
             for (int u = 0; u < UB; ++u) {
-                float wf[V];
-                unpack<T>(w[u], wf);
+                float2 wf[V / 2];
+                unpack2<T>(w[u], wf);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
-                    float xf[V];
-                    unpack<T>(xv[u][t], xf);
+                    float2 xf[V / 2];
+                    unpack2<T>(xv[u][t], xf);
 #pragma unroll
-                    for (int e = 0; e < V; e += 2) {
-                        a0[t] = fmaf(wf[e], xf[e], a0[t]);
-                        a1[t] = fmaf(wf[e + 1], xf[e + 1], a1[t]);
-                    }
+                    for (int e = 0; e < V / 2; ++e) a2[t] = __ffma2_rn(wf[e], xf[e], a2[t]);
                 }
             }
         }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-            const float v = warp_sum(a0[t] + a1[t]);
+            const float v = warp_sum(a2[t].x + a2[t].y);
             if (lane == 0) red[rr][wq][t] = v;
         }
         __syncthreads();
@@ -565,6 +520,24 @@ size_t gate_smem_bytes(int /*wdtype*/, int nt, int d, int /*r*/, int /*gate_kind
 
 size_t gate_stream_smem_bytes(int nt, int d, int r, int gate_kind, int cpb, int mw, int sb, int nb) {
     return stream_smem_layout(nt, d, r, gate_kind, cpb, mw, sb, nb).total;
+}
+
+bool gate_stream_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* sb, int* nb, size_t* smem) {
+    int best_sb = 0, best_nb = 0;
+    for (int cand_sb : {8192, 4096, 2048})
+        for (int cand_nb = 2; cand_nb <= 4; ++cand_nb) {
+            if (gate_stream_smem_bytes(nt, d, r, gate_kind, cpb, mw, cand_sb, cand_nb) > kMaxSmemPerCta) continue;
+            const long cur = (long)cand_sb * cand_nb, best = (long)best_sb * best_nb;
+            if (cur > best || (cur == best && cand_nb > best_nb)) {
+                best_sb = cand_sb;
+                best_nb = cand_nb;
+            }
+        }
+    if (!best_sb) return false;
+    *sb = best_sb;
+    *nb = best_nb;
+    *smem = gate_stream_smem_bytes(nt, d, r, gate_kind, cpb, mw, best_sb, best_nb);
+    return true;
 }
 
 template <class T, int NT>
@@ -600,7 +573,7 @@ static cudaError_t launch_stream_t(const GateParams& p, int grid, size_t smem, c
     static SmemAttrCache cache;
     cudaError_t e = ensure_smem(kern, smem, cache);
     if (e != cudaSuccess) return e;
-    return launch_ex(kern, dim3(grid), dim3(kThreads), smem, s, pdl, p);
+    return launch_ex(kern, dim3(grid), dim3(kStreamThreads), smem, s, pdl, p);
 }
 
 template <class T, int NT>

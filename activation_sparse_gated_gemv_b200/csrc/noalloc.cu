@@ -113,19 +113,18 @@ extern "C" int sffn_forward_noalloc(const void* w_gate_cm, const void* w_up_cm, 
     char* b = static_cast<char*>(base);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    // Plan: two gate CTAs per SM; down chunks so that slices x chunks ~ SMs.
-    const int cpb = (d_ff + 2 * sms - 1) / (2 * sms);
+    // Plan: one gate CTA per SM; down chunks so that slices x chunks ~ SMs.
+    const int cpb = (d_ff + sms - 1) / sms;
     const int g1 = (d_ff + cpb - 1) / cpb;
     const int slices = (d + down_slice_cols(wdtype) - 1) / down_slice_cols(wdtype);
     int chunks = sms / slices;
     if (chunks < 1) chunks = 1;
     if (chunks > g1) chunks = g1;
     const int nt = n_tokens <= 1 ? 1 : n_tokens <= 2 ? 2 : n_tokens <= 4 ? 4 : 8;
-    const int sb = 4096, nb = 2;
-    int gnt = nt;
-    while (gnt > 1 && gate_stream_smem_bytes(gnt, d, 0, kGateDense, cpb, 1, sb, nb) > 110 * 1024) gnt /= 2;
-    const size_t gsmem = gate_stream_smem_bytes(gnt, d, 0, kGateDense, cpb, 1, sb, nb);
-    if (gsmem > 110 * 1024) return na_fail(SFFN_ERR_UNSUPPORTED, "shape does not fit shared memory");
+    int gnt = nt, sb = 0, nb = 0;
+    size_t gsmem = 0;
+    while (!gate_stream_geometry(gnt, d, 0, kGateDense, cpb, 1, &sb, &nb, &gsmem) && gnt > 1) gnt /= 2;
+    if (!sb) return na_fail(SFFN_ERR_UNSUPPORTED, "shape does not fit shared memory");
 
     // The ticket counters and the status word must start at zero: clear them.
     e = cudaMemsetAsync(b + kOffTickets, 0, kOffStatus + 256 - kOffTickets, s);
@@ -133,7 +132,7 @@ extern "C" int sffn_forward_noalloc(const void* w_gate_cm, const void* w_up_cm, 
 
     GateParams gp{};
     gp.x = x; gp.n = n_tokens; gp.d = d; gp.d_ff = d_ff; gp.r = 0;
-    gp.wg = w_gate_cm; gp.wup = w_up_cm;
+    gp.wg = w_gate_cm; gp.wup = w_up_cm; gp.wdn = w_down;
     gp.out = kOutSelectUp; gp.force_all = 0; gp.tau = tau;
     gp.cpb = cpb; gp.mw = 1;
     gp.lst_idx = reinterpret_cast<int*>(b + kOffIdx);

@@ -414,13 +414,15 @@ def main():
         for i in range(launches):
             per_kernel[i] += evs[i].elapsed_time(evs[i + 1])
     per_kernel /= K2
-    kernel_names = (["lopa_u"] if wl.gate == "lopa" else []) + (
-        ["gate_select_up"] if wl.select == "threshold" else ["gate_z", "topk", "preselected_up"]) + ["down"]
+    kernel_names = ffns[0].last_kernel_names()
     dominant = int(np.argmax(per_kernel))
     peaks, peak_kind = measured_peaks()
     dom_name = kernel_names[dominant] if dominant < len(kernel_names) else f"k{dominant}"
     w = bytes_per_elem(wl.dtype)
-    if dom_name == "gate_select_up":
+    if dom_name == "decode_fused":
+        dom_bytes = algorithmic_bytes(wl, union) - wl.n * wl.d * bytes_per_elem(wl.dtype) - (
+            wl.d * wl.r * bytes_per_elem(wl.dtype) if wl.gate == "lopa" else 0)
+    elif dom_name == "gate_select_up":
         dom_bytes = algorithmic_bytes(wl, union, gate_kernel_only=True)
     elif dom_name == "down":
         dom_bytes = union * wl.d * w + 4 * union * wl.n + wl.n * wl.d * w

@@ -130,6 +130,10 @@ int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union
 int sffn_set_stage_events(sffn_handle h, void* const* events, int n_events);
 int sffn_last_launches(sffn_handle h, int32_t* launches);
 
+/* Name of kernel i (0-based, launch order) of the last forward, for
+ * profiles and timing reports; "" when there is no such kernel. */
+const char* sffn_last_kernel_name(sffn_handle h, int i);
+
 /* Synchronise the device and read the handle's sticky device status word,
  * which kernels set when one of their own bounds checks fails (they then skip
  * the access instead of faulting).  Returns SFFN_OK or SFFN_ERR_DEVICE_CHECK
