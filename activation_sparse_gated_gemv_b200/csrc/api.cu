@@ -2,8 +2,12 @@
 //
 // Host-side orchestration only: argument checks, the device workspace plan,
 // weight repacking, and the kernel sequence of one forward:
-//   threshold:  [LoPA x A] -> gate+select+up -> down
-//   top-K:      [LoPA x A] -> gate (z) -> top-K -> preselected up -> down
+//   threshold, n <= 4:  [LoPA x A] -> one fused decode kernel
+//   n > 4, bf16 (tensor cores):
+//               gate GEMM (z) [-> top-K] -> union list -> up GEMM -> down GEMM
+//               (LoPA: x A GEMM, then the z GEMM)
+//   otherwise:  [LoPA x A] -> gate+select+up -> down, or for top-K
+//               [LoPA x A] -> gate (z) -> top-K -> preselected up -> down
 // Every kernel is launched with programmatic dependent launch so its launch
 // latency overlaps the previous kernel's tail; each kernel waits on its
 // predecessor before touching shared buffers.
@@ -90,6 +94,17 @@ struct sffn_ctx {
     int* status = nullptr;
     void* xdev = nullptr;
     void* ydev = nullptr;
+    // tensor-core batched path (bf16 handles with max_tokens > kDecodeMaxTokens)
+    bool tc = false;
+    int tc_npad_max = 0;
+    long long tc_ldh = 0;
+    uint32_t* ubits = nullptr;
+    int* u_count = nullptr;
+    void* h2 = nullptr;          // [2 npad][tc_ldh] bf16: h as hi/lo rows
+    void* u2 = nullptr;          // [2 npad][r] bf16: LoPA x A as hi/lo rows
+    float* tc_part = nullptr;    // [sms][2][2 npad][128]
+    unsigned* tc_tickets = nullptr;
+    bool last_tc = false;
     Plan plan;
     int last_n = -1;
     cudaStream_t last_stream = nullptr;
@@ -176,6 +191,95 @@ int check_forward(const sffn_ctx* h, const void* x, int n, int gate_mode, const 
     return SFFN_OK;
 }
 
+// Batched forward on the tensor cores: gate GEMM -> [top-K] -> union list ->
+// up GEMM -> down GEMM, every GEMM one stream-K tcgen05 kernel over all SMs.
+int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel, void* out, cudaStream_t s,
+           bool dense, int& launches) {
+    const sffn_config& c = h->cfg;
+    const bool topk = sel->kind == SFFN_SELECT_TOPK;
+    const int npad = (int)round_up(n, 16);
+    const float tau = topk ? 0.f : sel->tau;
+    TcParams base{};
+    base.n = n;
+    base.npad = npad;
+    base.tau = tau;
+    base.topk = topk ? 1 : 0;
+    base.part = h->tc_part;
+    base.tickets = h->tc_tickets;
+    base.status = h->status;
+
+    TcParams g = base;
+    g.mode = kTcGateZ;
+    g.z = h->zbuf;
+    g.ldz = c.d_ff;
+    g.ubits = h->ubits;
+    g.m_total = c.d_ff;
+    if (lopa) {
+        TcParams u = base;                      // u = x A, as hi/lo bf16 rows
+        u.mode = kTcGateSplit;
+        u.a = h->a; u.lda = c.d; u.m_total = c.lopa_rank; u.k_total = c.d;
+        u.b = x; u.ldb = c.d; u.b_rows = n; u.b_cols = c.d; u.nb = npad;
+        u.out = h->u2; u.ldo = c.lopa_rank;
+        SFFN_CUDA(launch_tc(u, h->sms, s, true), "tensor-core x A launch");
+        h->last_names[launches] = "tc_lopa_u";
+        record(h, ++launches, s);
+        g.a = h->bcm; g.lda = c.lopa_rank; g.k_total = c.lopa_rank;
+        g.b = h->u2; g.ldb = c.lopa_rank; g.b_rows = 2 * npad; g.b_cols = c.lopa_rank;
+        g.nb = 2 * npad; g.paired = 1;
+    } else {
+        g.a = h->wg; g.lda = c.d; g.k_total = c.d;
+        g.b = x; g.ldb = c.d; g.b_rows = n; g.b_cols = c.d; g.nb = npad;
+    }
+    SFFN_CUDA(launch_tc(g, h->sms, s, true), "tensor-core gate launch");
+    h->last_names[launches] = "tc_gate";
+    record(h, ++launches, s);
+
+    if (topk) {
+        TopkParams tp{};
+        tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
+        tp.ubits = h->ubits;
+        SFFN_CUDA(launch_topk(tp, s, true), "top-K launch");
+        h->last_names[launches] = "topk";
+        record(h, ++launches, s);
+    }
+
+    UnionParams up{};
+    up.ubits = h->ubits; up.d_ff = c.d_ff; up.n = n; up.mw = h->plan.mw;
+    up.z = h->zbuf; up.sel = h->sel; up.tau = tau; up.topk = topk ? 1 : 0; up.force_all = dense ? 1 : 0;
+    up.lst = h->lst_idx; up.u_count = h->u_count; up.lst_mask = h->lst_mask;
+    SFFN_CUDA(launch_union(up, s, true), "union list launch");
+    h->last_names[launches] = "union";
+    record(h, ++launches, s);
+
+    TcParams w = base;                          // h = g * <x, W_up[i]> over the union
+    w.mode = kTcUp;
+    w.a = h->wup; w.lda = c.d; w.a_rows = h->lst_idx; w.u_count = h->u_count; w.u_cap = c.d_ff;
+    w.k_total = c.d;
+    w.b = x; w.ldb = c.d; w.b_rows = n; w.b_cols = c.d; w.nb = npad;
+    w.out = h->h2; w.ldo = h->tc_ldh; w.h_pairs = 1;
+    w.zsel = h->zbuf; w.gsel = h->gbuf; w.ldsel = c.d_ff;
+    SFFN_CUDA(launch_tc(w, h->sms, s, true), "tensor-core up launch");
+    h->last_names[launches] = "tc_up";
+    record(h, ++launches, s);
+
+    TcParams dn = base;                         // y = sum over the union of h W_down[i]
+    dn.mode = kTcDown;
+    dn.a = h->wdn; dn.lda = c.d; dn.a_rows = h->lst_idx; dn.u_count = h->u_count; dn.u_cap = c.d_ff;
+    dn.m_total = c.d;
+    dn.b = h->h2; dn.ldb = h->tc_ldh; dn.b_rows = 2 * npad; dn.b_cols = (int)h->tc_ldh;
+    dn.nb = 2 * npad; dn.paired = 1;
+    dn.out = out; dn.ldo = c.d;
+    SFFN_CUDA(launch_tc(dn, h->sms, s, true), "tensor-core down launch");
+    h->last_names[launches] = "tc_down";
+    record(h, ++launches, s);
+
+    h->last_n = n;
+    h->last_stream = s;
+    h->last_launches = launches;
+    h->last_tc = true;
+    return SFFN_OK;
+}
+
 int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_select* sel, void* out,
                 cudaStream_t s, bool dense) {
     const sffn_config& c = h->cfg;
@@ -194,6 +298,9 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     const bool fused = sel->kind == SFFN_SELECT_THRESHOLD && !dense && n <= kDecodeMaxTokens &&
                        decode_geometry(dec_nt, c.d, lopa ? c.lopa_rank : 0, gk, P.cpb, P.mw, &dec_sb, &dec_nb,
                                        &dec_smem);
+
+    h->last_tc = false;
+    if (h->tc && n > kDecodeMaxTokens && n <= kTcMaxTokens) return run_tc(h, x, n, lopa, sel, out, s, dense, launches);
 
     if (lopa) {
         LopaUParams lp{};
@@ -362,6 +469,17 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_fp = take((size_t)P.g1 * (T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * D * 4);
     const size_t o_tk = take((size_t)(P.down_slices > 2 ? P.down_slices : 2) * 4), o_st = take(4);
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
+    // tensor-core path buffers
+    h->tc = c.wdtype == SFFN_BF16 && c.max_tokens > kDecodeMaxTokens;
+    h->tc_npad_max = (int)round_up(c.max_tokens < kTcMaxTokens ? c.max_tokens : kTcMaxTokens, 16);
+    h->tc_ldh = (long long)round_up(F, 128);
+    const size_t NP = h->tc ? (size_t)h->tc_npad_max : 0;
+    const size_t FDR = F > D ? (F > R ? F : R) : (D > R ? D : R);
+    const size_t tiles = round_up(FDR, 128) / 128 + 1;
+    const size_t o_ub = take(h->tc ? tiles * 4 * 4 : 0), o_uc = take(h->tc ? 4 : 0);
+    const size_t o_h2 = take(2 * NP * (size_t)h->tc_ldh * 2), o_u2 = take(2 * NP * R * 2);
+    // stream-K partial tiles: two slots per CTA of up to 256 accumulator columns x 128 rows
+    const size_t o_tp = take(h->tc ? (size_t)h->sms * 2 * 256 * 128 * 4 : 0), o_tt = take(h->tc ? tiles * 4 : 0);
     e = cudaMalloc(&h->ws, off);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "workspace allocation"); }
     char* b = static_cast<char*>(h->ws);
@@ -379,6 +497,14 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->status = reinterpret_cast<int*>(b + o_st);
     h->xdev = b + o_x;
     h->ydev = b + o_y;
+    if (h->tc) {
+        h->ubits = reinterpret_cast<uint32_t*>(b + o_ub);
+        h->u_count = reinterpret_cast<int*>(b + o_uc);
+        h->h2 = b + o_h2;
+        h->u2 = b + o_u2;
+        h->tc_part = reinterpret_cast<float*>(b + o_tp);
+        h->tc_tickets = reinterpret_cast<unsigned*>(b + o_tt);
+    }
     e = cudaMemset(h->ws, 0, off);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(e, "workspace init"); }
@@ -507,6 +633,30 @@ int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union
     const int n = h->last_n, F = h->cfg.d_ff;
     std::vector<int> seg(P.g1), lidx(F);
     std::vector<uint32_t> mask((size_t)F * P.mw);
+    if (h->last_tc) {
+        // one ordered union list of u_count entries
+        int U = 0;
+        SFFN_CUDA(cudaMemcpy(&U, h->u_count, 4, cudaMemcpyDeviceToHost), "list copy");
+        if (U < 0 || U > F) return fail(SFFN_ERR_DEVICE_CHECK, "union size %d", U);
+        SFFN_CUDA(cudaMemcpy(lidx.data(), h->lst_idx, (size_t)U * 4, cudaMemcpyDeviceToHost), "list copy");
+        SFFN_CUDA(cudaMemcpy(mask.data(), h->lst_mask, mask.size() * 4, cudaMemcpyDeviceToHost), "list copy");
+        for (int t = 0; t < n; ++t) counts[t] = 0;
+        int uni = 0, prev = -1;
+        for (int i = 0; i < U; ++i) {
+            const int k = lidx[i];
+            if (k <= prev || k >= F) return fail(SFFN_ERR_DEVICE_CHECK, "union list entry %d = %d", i, k);
+            prev = k;
+            bool any = false;
+            for (int t = 0; t < n; ++t)
+                if ((mask[(size_t)k * P.mw + (t >> 5)] >> (t & 31)) & 1u) {
+                    idx[(size_t)t * F + counts[t]++] = k;
+                    any = true;
+                }
+            uni += any;
+        }
+        if (union_size) *union_size = uni;
+        return SFFN_OK;
+    }
     SFFN_CUDA(cudaMemcpy(seg.data(), h->seg_count, seg.size() * 4, cudaMemcpyDeviceToHost), "list copy");
     SFFN_CUDA(cudaMemcpy(lidx.data(), h->lst_idx, lidx.size() * 4, cudaMemcpyDeviceToHost), "list copy");
     SFFN_CUDA(cudaMemcpy(mask.data(), h->lst_mask, mask.size() * 4, cudaMemcpyDeviceToHost), "list copy");

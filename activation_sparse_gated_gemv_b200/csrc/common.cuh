@@ -225,6 +225,7 @@ struct TopkParams {
     int n, d_ff, k;
     float* gbuf;            // [n][d_ff]
     uint8_t* sel;           // [n][d_ff]
+    uint32_t* ubits;        // [d_ff/32] union bitmap, OR-ed into (NULL: none)
 };
 
 struct DownParams {
@@ -261,6 +262,60 @@ struct DecodeParams {
     unsigned* tickets;      // [2] zero between forwards
     int reducers;           // CTAs that sum the partials (d / reducers a multiple of 4)
     void* y;                // [n][d] T
+};
+
+// Batched tensor-core GEMM (tcgen05): modes and parameters.
+enum TcMode {
+    kTcGateZ = 0,       // z[t][m] fp32 (+ union bitmap) from weight rows x token rows
+    kTcGateSplit = 1,   // u[t][m] as bf16 hi rows [0,npad) and lo rows [npad,2 npad)
+    kTcUp = 2,          // h = g * <x, W_up[list[m]]>, bf16 hi/lo rows at union position m
+    kTcDown = 3         // y[t][m] = sum over union positions of h * W_down[list[pos]][m]
+};
+
+struct TcParams {
+    int mode;
+    const void* a;          // bf16 weight rows; row stride lda elements
+    long long lda;
+    const int* a_rows;      // union list (up, down), else NULL
+    int m_total;            // accumulator rows: gate rows, or d for down
+    int k_total;            // contraction length for gate and up
+    const int* u_count;     // union size (up, down)
+    int u_cap;              // upper bound of the union size
+    const void* b;          // bf16 token rows, K-major; row stride ldb
+    long long ldb;
+    int b_rows, b_cols;     // rows and columns of b that exist (the rest reads as zero)
+    int n, npad, nb;        // tokens, tokens padded to 16, MMA N (npad or 2 npad)
+    int paired;             // accumulator columns t and npad+t are hi and lo parts
+    float* z;               // GateZ output [n][ldz]
+    long long ldz;
+    void* out;              // GateSplit / Up: bf16 [2 npad][ldo]; Down: bf16 y [n][ldo]
+    long long ldo;
+    const float* zsel;      // Up, threshold: z [n][ldsel]
+    const float* gsel;      // Up, top-K: gbuf [n][ldsel]
+    long long ldsel;
+    float tau;
+    int topk;
+    uint32_t* ubits;        // GateZ: union bitmap out (threshold), zeroed (top-K)
+    float* part;            // [CTAs][2][nb][128] stream-K partial tiles
+    unsigned* tickets;      // per tile, zero between launches
+    int* status;
+    int h_pairs;            // Up: also write the lo rows of h (B of a paired down)
+    int stages;             // set by the launcher
+    int ks;                 // set by the launcher: 64-wide k-blocks per iteration (gate, up)
+    int mt;                 // set by the launcher: 128-row accumulator tiles per work tile (down)
+    uint32_t tmem_cols;     // set by the launcher
+};
+
+struct UnionParams {
+    const uint32_t* ubits;  // [ceil(d_ff/32)]
+    int d_ff, n, mw;
+    const float* z;         // threshold: [n][d_ff]
+    const uint8_t* sel;     // top-K: [n][d_ff]
+    float tau;
+    int topk, force_all;
+    int* lst;               // [d_ff] ordered union
+    int* u_count;
+    uint32_t* lst_mask;     // [d_ff][mw] tokens that selected each listed channel
 };
 
 // Bits of the device status word.
@@ -326,5 +381,9 @@ bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* 
 cudaError_t launch_decode(int wdtype, const DecodeParams& p, int nt, int gate_kind, int grid, size_t smem,
                           cudaStream_t s, bool pdl);
 constexpr int kDecodeMaxTokens = 4;   // the fused decode path takes up to this many tokens
+size_t tc_smem_bytes(int a_sub, int ks, int nb, int* stages);
+cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_union(const UnionParams& p, cudaStream_t s, bool pdl);
+constexpr int kTcMaxTokens = 128;     // token columns of one tensor-core pass (hi/lo pairs fill N = 256)
 
 }  // namespace sffn

@@ -7,7 +7,8 @@
 // warp-aggregated shared-memory histograms) finds the K-th largest key, then a
 // block-wide prefix sum over channel order takes the ties at that key from the
 // lowest channel index up.  Outputs: sel[t][k] (1 = selected) and
-// gbuf[t][k] = SiLU(z) on selected channels, 0 elsewhere.
+// gbuf[t][k] = SiLU(z) on selected channels, 0 elsewhere; optionally the
+// selected channels are OR-ed into a union bitmap (bit k of word k/32).
 #include "common.cuh"
 
 namespace sffn {
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
         }
         p.sel[row + k] = s ? 1 : 0;
         p.gbuf[row + k] = s ? gv : 0.f;
+        if (s && p.ubits) atomicOr(&p.ubits[k >> 5], 1u << (k & 31));
     }
 }
 

@@ -431,6 +431,14 @@ def main():
         dom_bytes = (wl.d * wl.d_ff * w if wl.gate == "dense" else wl.r * wl.d_ff * w) + wl.n * wl.d * w
     elif dom_name == "preselected_up":
         dom_bytes = union * wl.d * w + wl.n * wl.d * w
+    elif dom_name == "tc_gate":
+        dom_bytes = (wl.d * wl.d_ff if wl.gate == "dense" else wl.r * wl.d_ff) * w + wl.n * wl.d * w
+    elif dom_name == "tc_up":
+        dom_bytes = union * wl.d * w + wl.n * wl.d * w
+    elif dom_name == "tc_down":
+        dom_bytes = union * wl.d * w + wl.n * wl.d * w
+    elif dom_name == "tc_lopa_u":
+        dom_bytes = wl.d * wl.r * w + wl.n * wl.d * w
     else:
         dom_bytes = wl.d * wl.r * w + wl.n * wl.d * w
     # Stage events put an event node between kernels, which stops the next

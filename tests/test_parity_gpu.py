@@ -131,6 +131,13 @@ SMALL = [
     (1032, 1536, 0, 4, "bf16", "dense", "topk"),
     (8, 300, 8, 1, "f32", "lopa", "threshold"),
     (64, 256, 0, 1024, "bf16", "dense", "threshold"),    # the largest token count
+    # batched tensor-core path (bf16, 5 <= n <= 128): ragged row tiles and k-blocks
+    (136, 4100, 0, 64, "bf16", "dense", "threshold"),
+    (520, 3000, 64, 33, "bf16", "lopa", "threshold"),
+    (264, 1000, 0, 16, "bf16", "dense", "topk"),
+    (264, 1000, 32, 128, "bf16", "lopa", "topk"),
+    (64, 300, 8, 6, "bf16", "lopa", "topk"),
+    (1024, 640, 0, 100, "bf16", "dense", "threshold"),
 ]
 
 
@@ -142,15 +149,16 @@ def test_small_ragged(sffn, d, d_ff, r, n, dtype, gate, select):
     ffn.set_weights(**w)
     tau = workloads.tau_for_sparsity(0.85)
     k = max(1, d_ff // 8)
-    tokens = None if n <= 32 else [0, 1, 511, 1023]
+    tokens = None if n <= 32 else [0, 1, n // 2, n - 1]
     check_forward(ffn, w, x, gate, select, tau=tau, k=k, tokens=tokens)
     ffn.close()
 
 
+@pytest.mark.parametrize("n", [3, 20])
 @pytest.mark.parametrize("select", ["threshold", "topk"])
 @pytest.mark.parametrize("gate", ["dense", "lopa"])
-def test_dense_path_matches_oracle_and_sparse(sffn, gate, select):
-    d, d_ff, r, n = 128, 1500, 16, 3
+def test_dense_path_matches_oracle_and_sparse(sffn, gate, select, n):
+    d, d_ff, r = 128, 1500, 16
     w = workloads.ffn_weights(d, d_ff, "bf16", seed=5, gate="both", r=r)
     x = workloads.tokens(n, d, "bf16", seed=5)
     ffn = sffn.SparseFFN(d, d_ff, r, n, "bf16")
