@@ -102,8 +102,12 @@ struct sffn_ctx {
     int* u_count = nullptr;
     void* h2 = nullptr;          // [2 npad][tc_ldh] bf16: h as hi/lo rows
     void* u2 = nullptr;          // [2 npad][r] bf16: LoPA x A as hi/lo rows
-    float* tc_part = nullptr;    // [sms][2][2 npad][128]
+    float* tc_part = nullptr;    // [sms][2][128][256]
     unsigned* tc_tickets = nullptr;
+    int* blk_list = nullptr;     // 128-channel blocks holding a selected channel
+    int* blk_count = nullptr;
+    bool maps_ok = false;        // weight tensor maps encoded
+    CUtensorMap map_wg{}, map_at{}, map_bcm{}, map_wup{}, map_wdn{};
     bool last_tc = false;
     Plan plan;
     int last_n = -1;
@@ -193,12 +197,22 @@ int check_forward(const sffn_ctx* h, const void* x, int n, int gate_mode, const 
 
 // Batched forward on the tensor cores: gate GEMM -> [top-K] -> union list ->
 // up GEMM -> down GEMM, every GEMM one stream-K tcgen05 kernel over all SMs.
+// Returns SFFN_ERR_UNSUPPORTED (nothing launched) when a tensor map cannot be
+// made for this call; the caller then takes the CUDA-core path.
 int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel, void* out, cudaStream_t s,
            bool dense, int& launches) {
     const sffn_config& c = h->cfg;
     const bool topk = sel->kind == SFFN_SELECT_TOPK;
     const int npad = (int)round_up(n, 16);
     const float tau = topk ? 0.f : sel->tau;
+    if (!h->maps_ok || (lopa && c.lopa_rank < 64)) return SFFN_ERR_UNSUPPORTED;
+    CUtensorMap map_x{}, map_u2{}, map_h2{};
+    if (encode_tile_map(&map_x, x, c.d, n, (uint64_t)c.d * 2, 64, npad) != cudaSuccess ||
+        encode_tile_map(&map_h2, h->h2, h->tc_ldh, 2 * npad, (uint64_t)h->tc_ldh * 2, 64, 2 * npad) != cudaSuccess ||
+        (lopa && encode_tile_map(&map_u2, h->u2, c.lopa_rank, 2 * npad, (uint64_t)c.lopa_rank * 2, 64, 2 * npad) !=
+                     cudaSuccess))
+        return SFFN_ERR_UNSUPPORTED;
+
     TcParams base{};
     base.n = n;
     base.npad = npad;
@@ -217,18 +231,17 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     if (lopa) {
         TcParams u = base;                      // u = x A, as hi/lo bf16 rows
         u.mode = kTcGateSplit;
-        u.a = h->a; u.lda = c.d; u.m_total = c.lopa_rank; u.k_total = c.d;
-        u.b = x; u.ldb = c.d; u.b_rows = n; u.b_cols = c.d; u.nb = npad;
+        u.ta = h->map_at; u.tb = map_x;
+        u.m_total = c.lopa_rank; u.k_total = c.d; u.nb = npad;
         u.out = h->u2; u.ldo = c.lopa_rank;
         SFFN_CUDA(launch_tc(u, h->sms, s, true), "tensor-core x A launch");
         h->last_names[launches] = "tc_lopa_u";
         record(h, ++launches, s);
-        g.a = h->bcm; g.lda = c.lopa_rank; g.k_total = c.lopa_rank;
-        g.b = h->u2; g.ldb = c.lopa_rank; g.b_rows = 2 * npad; g.b_cols = c.lopa_rank;
-        g.nb = 2 * npad; g.paired = 1;
+        g.ta = h->map_bcm; g.tb = map_u2;
+        g.k_total = c.lopa_rank; g.nb = 2 * npad; g.paired = 1;
     } else {
-        g.a = h->wg; g.lda = c.d; g.k_total = c.d;
-        g.b = x; g.ldb = c.d; g.b_rows = n; g.b_cols = c.d; g.nb = npad;
+        g.ta = h->map_wg; g.tb = map_x;
+        g.k_total = c.d; g.nb = npad;
     }
     SFFN_CUDA(launch_tc(g, h->sms, s, true), "tensor-core gate launch");
     h->last_names[launches] = "tc_gate";
@@ -247,27 +260,28 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     up.ubits = h->ubits; up.d_ff = c.d_ff; up.n = n; up.mw = h->plan.mw;
     up.z = h->zbuf; up.sel = h->sel; up.tau = tau; up.topk = topk ? 1 : 0; up.force_all = dense ? 1 : 0;
     up.lst = h->lst_idx; up.u_count = h->u_count; up.lst_mask = h->lst_mask;
+    up.blk_list = h->blk_list; up.blk_count = h->blk_count;
     SFFN_CUDA(launch_union(up, s, true), "union list launch");
     h->last_names[launches] = "union";
     record(h, ++launches, s);
 
-    TcParams w = base;                          // h = g * <x, W_up[i]> over the union
+    const int nblk = (c.d_ff + 127) / 128;
+    TcParams w = base;                          // h = g * <x, W_up[ch]> over the active channel blocks
     w.mode = kTcUp;
-    w.a = h->wup; w.lda = c.d; w.a_rows = h->lst_idx; w.u_count = h->u_count; w.u_cap = c.d_ff;
-    w.k_total = c.d;
-    w.b = x; w.ldb = c.d; w.b_rows = n; w.b_cols = c.d; w.nb = npad;
+    w.ta = h->map_wup; w.tb = map_x;
+    w.blk_list = h->blk_list; w.blk_count = h->blk_count; w.blk_cap = nblk;
+    w.m_total = c.d_ff; w.k_total = c.d; w.nb = npad;
     w.out = h->h2; w.ldo = h->tc_ldh; w.h_pairs = 1;
     w.zsel = h->zbuf; w.gsel = h->gbuf; w.ldsel = c.d_ff;
     SFFN_CUDA(launch_tc(w, h->sms, s, true), "tensor-core up launch");
     h->last_names[launches] = "tc_up";
     record(h, ++launches, s);
 
-    TcParams dn = base;                         // y = sum over the union of h W_down[i]
+    TcParams dn = base;                         // y = sum over the active blocks of h W_down[ch]
     dn.mode = kTcDown;
-    dn.a = h->wdn; dn.lda = c.d; dn.a_rows = h->lst_idx; dn.u_count = h->u_count; dn.u_cap = c.d_ff;
-    dn.m_total = c.d;
-    dn.b = h->h2; dn.ldb = h->tc_ldh; dn.b_rows = 2 * npad; dn.b_cols = (int)h->tc_ldh;
-    dn.nb = 2 * npad; dn.paired = 1;
+    dn.ta = h->map_wdn; dn.tb = map_h2;
+    dn.blk_list = h->blk_list; dn.blk_count = h->blk_count; dn.blk_cap = nblk;
+    dn.m_total = c.d; dn.nb = 2 * npad; dn.paired = 1;
     dn.out = out; dn.ldo = c.d;
     SFFN_CUDA(launch_tc(dn, h->sms, s, true), "tensor-core down launch");
     h->last_names[launches] = "tc_down";
@@ -300,7 +314,10 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
                                        &dec_smem);
 
     h->last_tc = false;
-    if (h->tc && n > kDecodeMaxTokens && n <= kTcMaxTokens) return run_tc(h, x, n, lopa, sel, out, s, dense, launches);
+    if (h->tc && n > kDecodeMaxTokens && n <= kTcMaxTokens) {
+        const int rc = run_tc(h, x, n, lopa, sel, out, s, dense, launches);
+        if (rc != SFFN_ERR_UNSUPPORTED) return rc;
+    }
 
     if (lopa) {
         LopaUParams lp{};
@@ -479,7 +496,8 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_ub = take(h->tc ? tiles * 4 * 4 : 0), o_uc = take(h->tc ? 4 : 0);
     const size_t o_h2 = take(2 * NP * (size_t)h->tc_ldh * 2), o_u2 = take(2 * NP * R * 2);
     // stream-K partial tiles: two slots per CTA of up to 256 accumulator columns x 128 rows
-    const size_t o_tp = take(h->tc ? (size_t)h->sms * 2 * 256 * 128 * 4 : 0), o_tt = take(h->tc ? tiles * 4 : 0);
+    const size_t o_tp = take(h->tc ? (size_t)h->sms * 2 * 256 * 128 * 4 : 0), o_tt = take(h->tc ? tiles * 8 : 0);
+    const size_t o_bl = take(h->tc ? (round_up(F, 128) / 128 + 1) * 4 : 0), o_bc = take(h->tc ? 4 : 0);
     e = cudaMalloc(&h->ws, off);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "workspace allocation"); }
     char* b = static_cast<char*>(h->ws);
@@ -504,6 +522,8 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
         h->u2 = b + o_u2;
         h->tc_part = reinterpret_cast<float*>(b + o_tp);
         h->tc_tickets = reinterpret_cast<unsigned*>(b + o_tt);
+        h->blk_list = reinterpret_cast<int*>(b + o_bl);
+        h->blk_count = reinterpret_cast<int*>(b + o_bc);
     }
     e = cudaMemset(h->ws, 0, off);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -580,6 +600,18 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
     h->has_dense = w_gate != nullptr;
     h->has_lopa = A != nullptr;
     h->ready = true;
+    // tensor maps of the weights for the batched tensor-core path (host-side encoding only)
+    h->maps_ok = false;
+    if (h->tc && c.d >= 64) {
+        const uint64_t F = c.d_ff, D = c.d, R = c.lopa_rank;
+        bool ok = encode_tile_map(&h->map_wup, h->wup, D, F, D * 2, 64, 128) == cudaSuccess &&
+                  encode_tile_map(&h->map_wdn, h->wdn, D, F, D * 2, 64, 64) == cudaSuccess;
+        if (ok && h->wg) ok = encode_tile_map(&h->map_wg, h->wg, D, F, D * 2, 64, 128) == cudaSuccess;
+        if (ok && h->a && R >= 64)
+            ok = encode_tile_map(&h->map_at, h->a, D, R, D * 2, 64, 128) == cudaSuccess &&
+                 encode_tile_map(&h->map_bcm, h->bcm, R, F, R * 2, 64, 128) == cudaSuccess;
+        h->maps_ok = ok;
+    }
     return SFFN_OK;
 }
 

@@ -17,6 +17,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -268,41 +269,36 @@ struct DecodeParams {
 enum TcMode {
     kTcGateZ = 0,       // z[t][m] fp32 (+ union bitmap) from weight rows x token rows
     kTcGateSplit = 1,   // u[t][m] as bf16 hi rows [0,npad) and lo rows [npad,2 npad)
-    kTcUp = 2,          // h = g * <x, W_up[list[m]]>, bf16 hi/lo rows at union position m
-    kTcDown = 3         // y[t][m] = sum over union positions of h * W_down[list[pos]][m]
+    kTcUp = 2,          // h[t][ch] = g[t][ch] * <x[t], W_up[ch]> over the active channel blocks
+    kTcDown = 3         // y[t][m] = sum over the active channel blocks of h[t][ch] * W_down[ch][m]
 };
 
-struct TcParams {
+struct alignas(64) TcParams {
+    CUtensorMap ta;         // A operand: weight rows, tile box 64 x 128 (down: W_down, box 64 x 64)
+    CUtensorMap tb;         // B operand: token rows, tile box 64 x nb
     int mode;
-    const void* a;          // bf16 weight rows; row stride lda elements
-    long long lda;
-    const int* a_rows;      // union list (up, down), else NULL
-    int m_total;            // accumulator rows: gate rows, or d for down
-    int k_total;            // contraction length for gate and up
-    const int* u_count;     // union size (up, down)
-    int u_cap;              // upper bound of the union size
-    const void* b;          // bf16 token rows, K-major; row stride ldb
-    long long ldb;
-    int b_rows, b_cols;     // rows and columns of b that exist (the rest reads as zero)
+    int m_total;            // output rows: gate rows, d_ff (up), d (down)
+    int k_total;            // contraction length of gate and up
+    const int* blk_list;    // up, down: 128-channel blocks holding a selected channel, ascending
+    const int* blk_count;
+    int blk_cap;
     int n, npad, nb;        // tokens, tokens padded to 16, MMA N (npad or 2 npad)
     int paired;             // accumulator columns t and npad+t are hi and lo parts
-    float* z;               // GateZ output [n][ldz]
+    int h_pairs;            // up: also write the lo rows of h (B of a paired down)
+    float* z;               // gate: z [n][ldz]
     long long ldz;
-    void* out;              // GateSplit / Up: bf16 [2 npad][ldo]; Down: bf16 y [n][ldo]
+    void* out;              // gate-split, up: bf16 [2 npad][ldo]; down: bf16 y [n][ldo]
     long long ldo;
-    const float* zsel;      // Up, threshold: z [n][ldsel]
-    const float* gsel;      // Up, top-K: gbuf [n][ldsel]
+    const float* zsel;      // up, threshold: z [n][ldsel]
+    const float* gsel;      // up, top-K: gbuf [n][ldsel]
     long long ldsel;
     float tau;
     int topk;
-    uint32_t* ubits;        // GateZ: union bitmap out (threshold), zeroed (top-K)
-    float* part;            // [CTAs][2][nb][128] stream-K partial tiles
-    unsigned* tickets;      // per tile, zero between launches
+    uint32_t* ubits;        // gate: union bitmap out (threshold), zeroed (top-K)
+    float* part;            // [CTAs][2][128][nb] stream-K partial tiles
+    unsigned* tickets;      // two counters per tile (parts arrived, quarters summed), zero between launches
     int* status;
-    int h_pairs;            // Up: also write the lo rows of h (B of a paired down)
     int stages;             // set by the launcher
-    int ks;                 // set by the launcher: 64-wide k-blocks per iteration (gate, up)
-    int mt;                 // set by the launcher: 128-row accumulator tiles per work tile (down)
     uint32_t tmem_cols;     // set by the launcher
 };
 
@@ -316,6 +312,8 @@ struct UnionParams {
     int* lst;               // [d_ff] ordered union
     int* u_count;
     uint32_t* lst_mask;     // [d_ff][mw] tokens that selected each listed channel
+    int* blk_list;          // [ceil(d_ff/128)] 128-channel blocks holding a listed channel
+    int* blk_count;
 };
 
 // Bits of the device status word.
@@ -381,7 +379,9 @@ bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* 
 cudaError_t launch_decode(int wdtype, const DecodeParams& p, int nt, int gate_kind, int grid, size_t smem,
                           cudaStream_t s, bool pdl);
 constexpr int kDecodeMaxTokens = 4;   // the fused decode path takes up to this many tokens
-size_t tc_smem_bytes(int a_sub, int ks, int nb, int* stages);
+size_t tc_smem_bytes(int nb, int* stages);
+cudaError_t encode_tile_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                            uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
 cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_union(const UnionParams& p, cudaStream_t s, bool pdl);
 constexpr int kTcMaxTokens = 128;     // token columns of one tensor-core pass (hi/lo pairs fill N = 256)

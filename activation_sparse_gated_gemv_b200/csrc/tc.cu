@@ -1,40 +1,52 @@
 // Batched path on the 5th-generation tensor cores (tcgen05).
 //
-// With several tokens per step the gate and the gathered up and down passes
-// are dense contractions (a token batch against weight rows), so they run as
-// one tcgen05 GEMM kernel with three epilogues:
+// With several tokens per step the gate and the up and down passes are dense
+// contractions of a token batch against weight rows, so they run as one
+// tcgen05 GEMM kernel with four epilogues:
 //
-//   gate   Z^T[rows x n] = W[rows x K] . X^T      A = weight rows (K-major),
-//                                                 B = x rows (K-major)
-//   up     H^T[U x n]    = W_up[union rows] . X^T, times the gate activation
-//   down   Y^T[d x n]    = W_down[union rows]^T . H^T
-//                                                 A = W_down rows read as an
-//                                                 MN-major operand, B = H rows
+//   gate        Z^T[rows x n] = W[rows x K] . X^T        (z, fp32)
+//   gate-split  the same, written as bf16 hi/lo rows      (LoPA: u = x A)
+//   up          H^T[ch x n]   = W_up[ch] . X^T times the gate activation of ch
+//   down        Y^T[d x n]    = W_down[ch]^T . H^T
 //
-// "Model Casting and Low-Parameter Gating" (abstract): gate first, then only
-// the active channels' rows of the other two matrices.  "Mixture-of-Channels"
-// (section "Dentro MoC"): rows of the union of the batch's selected channels
-// are loaded once and shared by the tokens that selected them; a token that
-// did not select a channel gets a zero activation for it.
+// "Model Casting and Low-Parameter Gating" (abstract): gate first, then the
+// other two matrices only where the activation is non-zero.
+// "Mixture-of-Channels" (section "Dentro MoC"): rows of the channels the batch
+// selected are loaded once and shared by the tokens that selected them; a
+// token that did not select a channel gets a zero activation for it.
 //
-// Kernel structure (one CTA per SM, 288 threads):
-//   warps 0-3  producers: cp.async 16-byte copies of the A and B tiles of each
-//              64-wide k-block straight into the 128-byte-swizzled shared
-//              memory layout the MMA reads (rows gathered through the union
-//              list where needed), a ring of up to 8 stages on mbarriers;
-//   warp 8     one thread issues tcgen05.mma (M = 128, N = token columns,
-//              K = 16 per instruction, bf16 in, fp32 accumulate in tensor
-//              memory) and tcgen05.commit to release stages and accumulators;
-//   warps 4-7  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
+// Rows are skipped at the granularity of 128-channel blocks: the up and down
+// passes read every block holding at least one channel that some token of the
+// batch selected (a channel of such a block that a token did not select gets
+// g = 0 for it).  With several independent tokens nearly every block holds one
+// (a block is skipped only if all its 128 channels stay inactive for every
+// token), so the batched passes read what a per-channel gather would, in whole
+// tiles the TMA engine moves with one instruction.
+//
+// Kernel structure (one CTA per SM, 192 threads):
+//   warp 0     one thread: TMA 2-D tile copies (cp.async.bulk.tensor, 128-byte
+//              swizzle, no multicast) of the A and B tiles of each 64-wide
+//              k-block into a ring of stages on mbarriers;
+//   warp 1     allocates tensor memory; one thread issues tcgen05.mma (M = 128,
+//              N = token columns, K = 16 per instruction, bf16 in, fp32
+//              accumulate in tensor memory) and tcgen05.commit;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
 //              lanes), the mode's epilogue, stores.
 // Work is split stream-K: the (tile, k-block) iterations are cut into one
 // contiguous range per CTA, so every SM streams the same number of weight
 // bytes.  A tile cut between CTAs is summed in a fixed order (by CTA index)
-// by the CTA that completes it last (ticket), so results are deterministic.
+// once all its parts have arrived, each 32-row quarter by one of the tile's
+// CTAs after it has written all of its own parts (so no wait can hold back a
+// part another CTA needs); results are deterministic and no single CTA
+// serialises the tail.
 //
 // fp32 intermediates that feed a later MMA (LoPA's u = x A, and h) are passed
 // as two bf16 rows, hi = bf16(v) and lo = bf16(v - hi); the MMA multiplies both
 // and the epilogue adds the two columns, which keeps about 16 significant bits.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 
 namespace sffn {
@@ -42,12 +54,15 @@ namespace {
 
 constexpr int kBM = 128;            // accumulator rows (MMA M)
 constexpr int kBK = 64;             // k-block: 64 bf16 = one 128-byte swizzle row
-constexpr int kProd = 4;            // producer warps
-constexpr int kEpi = 4;             // epilogue warps
-constexpr int kMmaWarp = kProd + kEpi;
-constexpr int kTcThreads = (kProd + kEpi + 1) * 32;
+constexpr int kProdWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kEpiWarp0 = 2;        // epilogue warps 2..5
+constexpr int kEpi = 4;
+constexpr int kTcThreads = (kEpiWarp0 + kEpi) * 32;
 constexpr uint32_t kTileA = kBM * kBK * 2;   // 16 KB
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
+constexpr int kMaxBlocks = 1024;    // 128-channel blocks (d_ff <= 131072)
+constexpr int kMinIters = 16;       // iterations per CTA at least, so few tiles are cut many ways
 
 struct TcShared {
     uint64_t full[kMaxStages];
@@ -58,10 +73,10 @@ struct TcShared {
     uint32_t tmem_base;
     int abort;
     int reducer;
-    int rows[kBM];          // up: union rows of the current tile
+    int blk[kMaxBlocks];    // up/down: the active 128-channel blocks
 };
 
-// ---- tcgen05 / cp.async primitives -------------------------------------------
+// ---- tcgen05 / TMA primitives ------------------------------------------------
 
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -117,21 +132,26 @@ __device__ __forceinline__ bool mbar_wait_one(uint64_t* bar, uint32_t parity) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
     }
 }
-// 16-byte global -> shared copy; src_bytes 0 fills the 16 bytes with zeros.
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t src_bytes, uint64_t pol) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes), "l"(pol)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// 2-D tile of the tensor map at element coordinates (x = column, y = row) into
+// this CTA's shared memory (1024-byte aligned), completing on `bar`.
+// x is a multiple of 64 elements (128 bytes).
+__device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
 }
 __device__ __forceinline__ uint64_t l2_evict_last() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
     return pol;
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -154,11 +174,6 @@ __device__ __forceinline__ uint32_t mma_idesc(int n, int a_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(kBM >> 4) << 24);
 }
-// Byte offset of 16-byte chunk c (0..7) of row r in a K-major 128B-swizzled
-// tile whose 8-row groups are 1024 B apart.
-__device__ __forceinline__ uint32_t kmaj_off(int r, int c) {
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
 
 __device__ __forceinline__ void set_status(int* st, int bits) {
     if (st) atomicOr(st, bits);
@@ -175,29 +190,26 @@ struct Seg {
 };
 
 struct Problem {
-    int T, KB, U;
-    int MT;                 // 128-row accumulator tiles per work tile (down: MN-major, several)
-    int C;                  // CTAs that take work: min(grid, I), so none has an empty range
+    int T, KB, nblk;
+    int C;                  // CTAs that take work
     long long I, it0, it1;
 };
 
 __device__ __forceinline__ Problem make_problem(const TcParams& p) {
     Problem q;
-    q.U = p.u_count ? min(max(*p.u_count, 0), p.u_cap) : 0;
-    q.MT = p.mode == kTcDown ? p.mt : 1;
-    const int kstep = kBK * p.ks;                     // contraction per iteration
+    q.nblk = p.blk_count ? min(max(*p.blk_count, 0), min(p.blk_cap, kMaxBlocks)) : 0;
     if (p.mode == kTcUp) {
-        q.T = (q.U + kBM - 1) / kBM;
-        q.KB = (p.k_total + kstep - 1) / kstep;
+        q.T = q.nblk;
+        q.KB = (p.k_total + kBK - 1) / kBK;
     } else if (p.mode == kTcDown) {
-        q.T = (p.m_total + kBM * q.MT - 1) / (kBM * q.MT);
-        q.KB = (q.U + kstep - 1) / kstep;
+        q.T = (p.m_total + kBM - 1) / kBM;
+        q.KB = 2 * q.nblk;
     } else {
         q.T = (p.m_total + kBM - 1) / kBM;
-        q.KB = (p.k_total + kstep - 1) / kstep;
+        q.KB = (p.k_total + kBK - 1) / kBK;
     }
     q.I = (long long)q.T * q.KB;
-    q.C = (int)min((long long)gridDim.x, q.I);
+    q.C = (int)min((long long)gridDim.x, (q.I + kMinIters - 1) / kMinIters);
     if ((int)blockIdx.x < q.C) {
         q.it0 = q.I * blockIdx.x / q.C;
         q.it1 = q.I * (blockIdx.x + 1) / q.C;
@@ -216,129 +228,39 @@ __device__ __forceinline__ bool next_seg(const Problem& q, long long& it, Seg& s
     return true;
 }
 
-// Stage layout: A sub-tiles of 16 KB (gate/up: one per 64-wide k-block of the
-// iteration; down: one per 128-row accumulator tile), then B sub-tiles of
-// nb x 128 B (one per 64-wide k-block).
-__device__ __forceinline__ int a_subtiles(const TcParams& p) { return p.mode == kTcDown ? p.mt : p.ks; }
+// ---- producer: one thread issues the TMA copies --------------------------------
 
-// ---- producer: A and B tiles of one iteration into stage memory ---------------
-
-template <int LAG>
 __device__ void run_producer(const TcParams& p, const Problem& q, unsigned char* stages, uint32_t stage_bytes,
                              TcShared* sh) {
-    const int tid = threadIdx.x;                      // 0..127
-    const int w = tid >> 5, l = tid & 31;
     const uint64_t pol_w = l2_evict_first(), pol_b = l2_evict_last();
-    const bf16* A = static_cast<const bf16*>(p.a);
-    const bf16* B = static_cast<const bf16*>(p.b);
     const int S = p.stages;
-    const int KS = p.ks;
-    const int CPR = KS * 8;                           // 16-byte chunks of a K-major row per iteration
-    const int RPI = 32 / CPR;                         // rows per warp instruction (4, 2 or 1)
-    const int rsub = l / CPR, chunk = l % CPR;
-    const int kstep = kBK * KS;
-    const uint32_t b_off = (uint32_t)a_subtiles(p) * kTileA;
-    long long it = q.it0;
-    long long g = 0;                                  // iterations issued by this CTA
+    const uint32_t tx = kTileA + (uint32_t)p.nb * 128u;
+    long long it = q.it0, g = 0;
     Seg s;
-    bool ok = true;
-    while (ok && next_seg(q, it, s)) {
-        const int m0 = s.t * kBM * q.MT;
-        if (p.mode == kTcUp) {
-            // the tile's 128 union rows, shared by the producer warps
-            named_sync(2, kProd * 32);
-            const int m = m0 + tid;
-            sh->rows[tid] = m < q.U ? __ldg(p.a_rows + m) : -1;
-            named_sync(2, kProd * 32);
-        }
-        // down: the union rows of iteration kb (k-rows w + 4 j), fetched one iteration ahead
-        int rcur[16], rnxt[16];
-        if (p.mode == kTcDown) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int pos = s.kb0 * kBK + w + 4 * j;
-                rcur[j] = pos < q.U ? __ldg(p.a_rows + pos) : -1;
-            }
-        }
+    while (next_seg(q, it, s)) {
+        const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++g) {
-            if (p.mode == kTcDown) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int pos = (kb + 1) * kBK + w + 4 * j;
-                    rnxt[j] = (kb + 1 < s.kb1 && pos < q.U) ? __ldg(p.a_rows + pos) : -1;
-                }
-            }
             const int st = (int)(g % S);
-            const uint32_t use = (uint32_t)(g / S);
-            if (!mbar_wait_warp(&sh->empty[st], (use & 1u) ^ 1u)) {
+            if (!mbar_wait_one(&sh->empty[st], (uint32_t)(((g / S) & 1) ^ 1))) {
                 sh->abort = 1;
                 set_status(p.status, kStatusWaitTimeout);
-                ok = false;
-                break;
+                return;
             }
             const uint32_t sA = smem_addr(stages + (size_t)st * stage_bytes);
-            const uint32_t sB = sA + b_off;
-            const int k0 = kb * kstep;
-            if (p.mode != kTcDown) {
-                // K-major A: row r, chunk `chunk` of its KS*128 contiguous bytes
-                const int sub = chunk >> 3, c = chunk & 7;
-                const int k = k0 + chunk * 8;
-                for (int r = w * RPI + rsub; r < kBM; r += 4 * RPI) {
-                    long long row;
-                    bool v;
-                    if (p.mode == kTcUp) {
-                        row = sh->rows[r];
-                        v = row >= 0;
-                    } else {
-                        row = m0 + r;
-                        v = row < p.m_total;
-                    }
-                    v = v && k < p.k_total;
-                    const bf16* src = v ? A + row * p.lda + k : A;
-                    cp16(sA + sub * kTileA + kmaj_off(r, c), src, v ? 16u : 0u, pol_w);
-                }
+            const uint32_t sB = sA + kTileA;
+            mbar_expect_tx(&sh->full[st], tx);
+            if (p.mode == kTcDown) {
+                // MN-major A: 64 channels (k) x 128 output columns (m) of W_down, two 64-column boxes
+                const int c0 = sh->blk[kb >> 1] * kBM + (kb & 1) * kBK;
+                tma_tile(sA, &p.ta, m0, c0, &sh->full[st], pol_w);
+                tma_tile(sA + 8192, &p.ta, m0 + 64, c0, &sh->full[st], pol_w);
+                tma_tile(sB, &p.tb, c0, 0, &sh->full[st], pol_b);
             } else {
-                // MN-major A: k-row kr holds W_down[list[kb*64+kr]][m0 .. m0 + 128 MT); 16 MT chunks
-                const int cpr = q.MT * 16;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int kr = w + 4 * j;
-                    for (int qc = l; qc < cpr; qc += 32) {
-                        const int mt = qc >> 4, c16 = qc & 15;
-                        const int col = m0 + qc * 8;
-                        const bool v = rcur[j] >= 0 && col < p.m_total;
-                        const bf16* src = v ? A + (long long)rcur[j] * p.lda + col : A;
-                        const uint32_t off = (uint32_t)(mt * kTileA + (c16 >> 3) * 8192 + (kr >> 3) * 1024 +
-                                                        (kr & 7) * 128 + (((c16 & 7) ^ (kr & 7)) << 4));
-                        cp16(sA + off, src, v ? 16u : 0u, pol_w);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) rcur[j] = rnxt[j];
-            }
-            // B: nb rows, KS*128 contiguous bytes each
-            {
-                const int sub = chunk >> 3, c = chunk & 7;
-                const int k = k0 + chunk * 8;
-                for (int r = w * RPI + rsub; r < p.nb; r += 4 * RPI) {
-                    const bool v = r < p.b_rows && k < p.b_cols;
-                    const bf16* src = v ? B + (long long)r * p.ldb + k : B;
-                    cp16(sB + sub * (uint32_t)p.nb * 128u + kmaj_off(r, c), src, v ? 16u : 0u, pol_b);
-                }
-            }
-            cp_commit();
-            if (g >= LAG) {
-                cp_wait<LAG>();
-                fence_proxy_async();
-                mbar_arrive(&sh->full[(int)((g - LAG) % S)]);
+                tma_tile(sA, &p.ta, kb * kBK, m0, &sh->full[st], pol_w);
+                tma_tile(sB, &p.tb, kb * kBK, 0, &sh->full[st], pol_b);
             }
         }
     }
-    // every copy lands before the CTA can retire; arrive for the stages not yet signalled
-    cp_wait<0>();
-    fence_proxy_async();
-    if (ok)
-        for (long long h = (g >= LAG ? g - LAG : 0); h < g; ++h) mbar_arrive(&sh->full[(int)(h % S)]);
 }
 
 // ---- MMA issuer --------------------------------------------------------------
@@ -348,8 +270,6 @@ __device__ void run_mma(const TcParams& p, const Problem& q, unsigned char* stag
     const int S = p.stages;
     const bool down = p.mode == kTcDown;
     const uint32_t idesc = mma_idesc(p.nb, down ? 1 : 0);
-    const uint32_t b_off = (uint32_t)a_subtiles(p) * kTileA;
-    const int acc_cols = q.MT * p.nb;
     long long it = q.it0, g = 0;
     int segi = 0;
     Seg s;
@@ -362,7 +282,7 @@ __device__ void run_mma(const TcParams& p, const Problem& q, unsigned char* stag
             break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(acc * acc_cols);
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * p.nb);
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++g) {
             const int st = (int)(g % S);
             if (!mbar_wait_one(&sh->full[st], (uint32_t)((g / S) & 1))) {
@@ -371,20 +291,12 @@ __device__ void run_mma(const TcParams& p, const Problem& q, unsigned char* stag
             }
             tc_fence_after();
             const uint32_t sA = smem_addr(stages + (size_t)st * stage_bytes);
-            const uint32_t sB = sA + b_off;
-            if (down) {
-                for (int mt = 0; mt < q.MT; ++mt)
+            const uint32_t sB = sA + kTileA;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma(d_tmem + mt * p.nb, sw128_desc(sA + mt * kTileA + kk * 2048, 8192, 1024),
-                               sw128_desc(sB + kk * 32, 16, 1024), idesc, (kb > s.kb0 || kk > 0) ? 1u : 0u);
-            } else {
-                for (int sub = 0; sub < p.ks; ++sub)
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma(d_tmem, sw128_desc(sA + sub * kTileA + kk * 32, 16, 1024),
-                               sw128_desc(sB + sub * p.nb * 128 + kk * 32, 16, 1024), idesc,
-                               (kb > s.kb0 || sub > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint64_t ad =
+                    down ? sw128_desc(sA + kk * 2048, 8192, 1024) : sw128_desc(sA + kk * 32, 16, 1024);
+                tc_mma(d_tmem, ad, sw128_desc(sB + kk * 32, 16, 1024), idesc, (kb > s.kb0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(&sh->empty[st]);
         }
@@ -403,10 +315,9 @@ __device__ void run_mma(const TcParams& p, const Problem& q, unsigned char* stag
 
 // ---- epilogue ----------------------------------------------------------------
 
-// Final values v[0..15] of columns c0..c0+15 (combined hi+lo when paired) for
+// Final values v[0..15] of columns c0..c0+15 (hi+lo combined when paired) of
 // output row m.  `act` collects the gate's activity flag.
-__device__ __forceinline__ void emit16(const TcParams& p, const Problem& q, int m, int c0, const float* v,
-                                       bool& act) {
+__device__ __forceinline__ void emit16(const TcParams& p, int m, int c0, const float* v, bool& act) {
     if (p.mode == kTcGateZ) {
         if (m >= p.m_total) return;
 #pragma unroll
@@ -429,15 +340,15 @@ __device__ __forceinline__ void emit16(const TcParams& p, const Problem& q, int 
             o[(long long)(p.npad + tok) * p.ldo + m] = lo;
         }
     } else if (p.mode == kTcUp) {
+        // m is the channel; channels past d_ff (the last block's tail) write zeros
         bf16* o = static_cast<bf16*>(p.out);
-        const int ch = m < q.U ? __ldg(p.a_rows + m) : -1;
         float gv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int tok = c0 + i;
             gv[i] = 0.f;
-            if (ch >= 0 && tok < p.n) {
-                const long long zi = (long long)tok * p.ldsel + ch;
+            if (m < p.m_total && tok < p.n) {
+                const long long zi = (long long)tok * p.ldsel + m;
                 gv[i] = p.topk ? p.gsel[zi] : fmaxf(p.zsel[zi] - p.tau, 0.f);
             }
         }
@@ -460,15 +371,86 @@ __device__ __forceinline__ void emit16(const TcParams& p, const Problem& q, int 
     }
 }
 
-__device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, uint32_t tmem) {
-    const int ew = (threadIdx.x >> 5) & 3;            // TMEM lane quarter of this warp
+// Sum of the parts of 32-row quarter `quarter` of a cut tile, in CTA order,
+// once every part has arrived; the last of the tile's four quarter sums resets
+// its counters for the next launch.
+__device__ void sum_quarter(const TcParams& p, int t, int m0, int c_first, int c_last, int quarter, int row,
+                            int cols, size_t slot_floats) {
     const int lane = threadIdx.x & 31;
-    const int row = ew * 32 + lane;
-    const int etid = threadIdx.x - kProd * 32;        // 0..127
+    const int parts = c_last - c_first + 1;
+    unsigned* arrivals = p.tickets + 2 * t;
+    unsigned* finished = arrivals + 1;
+    bool ready = true;
+    if (lane == 0) {
+        const unsigned long long t0 = globaltimer_ns();
+        unsigned backoff = 64;
+        while (ld_acquire(arrivals) < (unsigned)parts) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                ready = false;
+                break;
+            }
+            __nanosleep(backoff);
+            if (backoff < 1024) backoff <<= 1;
+        }
+    }
+    ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
+    if (!ready) {
+        set_status(p.status, kStatusWaitTimeout);
+        return;
+    }
+    __threadfence();
+    const int m = m0 + row;
+    bool act = false;
+    for (int c0 = 0; c0 < cols; c0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        for (int c = c_first; c <= c_last; ++c) {
+            const float* pp =
+                p.part + ((size_t)c * 2 + (c == c_first ? 0 : 1)) * slot_floats + (size_t)row * p.nb + c0;
+            float4 a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(pp) + i);
+            if (p.paired) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) b[i] = __ldcg(reinterpret_cast<const float4*>(pp + p.npad) + i);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                v[4 * i] += a[i].x + b[i].x;
+                v[4 * i + 1] += a[i].y + b[i].y;
+                v[4 * i + 2] += a[i].z + b[i].z;
+                v[4 * i + 3] += a[i].w + b[i].w;
+            }
+        }
+        emit16(p, m, c0, v, act);
+    }
+    if (p.mode == kTcGateZ && p.ubits) {
+        const unsigned bits = __ballot_sync(0xffffffffu, act && !p.topk && m < p.m_total);
+        if (lane == 0) p.ubits[(m0 + quarter * 32) >> 5] = bits;
+    }
+    __syncwarp();
+    if (lane == 0 && atomicAdd(finished, 1u) == 3u) {
+        *arrivals = 0u;
+        *finished = 0u;
+    }
+}
+
+__device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, uint32_t tmem) {
+    const int warp = threadIdx.x >> 5;
+    const int quarter = warp & 3;                     // TMEM lanes this warp may access
+    const int lane = threadIdx.x & 31;
+    const int row = quarter * 32 + lane;
+    const int etid = threadIdx.x - kEpiWarp0 * 32;    // 0..127
     const int cols = p.paired ? p.npad : p.nb;        // final columns
     const int C = q.C;
-    const int acc_cols = q.MT * p.nb;
-    const size_t slot_floats = (size_t)acc_cols * kBM;
+    const size_t slot_floats = (size_t)p.nb * kBM;
+    // cut tiles this CTA takes part in (its first and last segments at most)
+    int cut_t[2], cut_m0[2], cut_first[2], cut_last[2];
+    int ncut = 0;
     long long it = q.it0;
     int segi = 0;
     Seg s;
@@ -482,88 +464,77 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
             return;
         }
         tc_fence_after();
-        const uint32_t taddr = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * acc_cols);
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.nb);
         const bool whole = s.kb0 == 0 && s.kb1 == q.KB;
-        const int mbase = s.t * kBM * q.MT + row;
-        bool act = false;
+        const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
+        const int m = m0 + row;
         if (whole) {
-            for (int mt = 0; mt < q.MT; ++mt)
-                for (int c0 = 0; c0 < cols; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(taddr + mt * p.nb + c0, v);
-                    if (p.paired) {
-                        float x[16];
-                        tmem_ld16(taddr + mt * p.nb + p.npad + c0, x);
+            bool act = false;
+            for (int c0 = 0; c0 < cols; c0 += 16) {
+                float v[16];
+                tmem_ld16(taddr + c0, v);
+                if (p.paired) {
+                    float x[16];
+                    tmem_ld16(taddr + p.npad + c0, x);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] += x[i];
-                    }
-                    emit16(p, q, mbase + mt * kBM, c0, v, act);
+                    for (int i = 0; i < 16; ++i) v[i] += x[i];
                 }
+                emit16(p, m, c0, v, act);
+            }
             tc_fence_before();
             mbar_arrive(&sh->tempty[acc]);
+            if (p.mode == kTcGateZ && p.ubits) {
+                // union bitmap words of this tile: one word per warp (32 channels)
+                const unsigned bits = __ballot_sync(0xffffffffu, act && !p.topk && m < p.m_total);
+                if (lane == 0) p.ubits[(m0 + quarter * 32) >> 5] = bits;
+            }
         } else {
-            // partial tile: park it, the CTA completing the tile sums all parts in CTA order
+            // cut tile: park this CTA's part (row-major, each thread's row contiguous)
             const int c_first = cta_of((long long)s.t * q.KB, q.I, C);
+            const int c_last = cta_of((long long)(s.t + 1) * q.KB - 1, q.I, C);
             const int slot = c_first == (int)blockIdx.x ? 0 : 1;
-            float* mine = p.part + ((size_t)blockIdx.x * 2 + slot) * slot_floats;
-            for (int c0 = 0; c0 < acc_cols; c0 += 16) {
+            float* mine = p.part + ((size_t)blockIdx.x * 2 + slot) * slot_floats + (size_t)row * p.nb;
+            for (int c0 = 0; c0 < p.nb; c0 += 16) {
                 float v[16];
                 tmem_ld16(taddr + c0, v);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) mine[(size_t)(c0 + i) * kBM + row] = v[i];
+                for (int i = 0; i < 16; i += 4)
+                    *reinterpret_cast<float4*>(mine + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
             }
             tc_fence_before();
             mbar_arrive(&sh->tempty[acc]);
             __threadfence();
             named_sync(1, kEpi * 32);
-            const int c_last = cta_of((long long)(s.t + 1) * q.KB - 1, q.I, C);
-            if (etid == 0) {
-                const unsigned done = atomicAdd(p.tickets + s.t, 1u);
-                sh->reducer = done == (unsigned)(c_last - c_first);
-                if (sh->reducer) p.tickets[s.t] = 0;   // every part has arrived: reset for the next launch
+            if (etid == 0) atomicAdd(p.tickets + 2 * s.t, 1u);
+            if (ncut < 2) {
+                cut_t[ncut] = s.t;
+                cut_m0[ncut] = m0;
+                cut_first[ncut] = c_first;
+                cut_last[ncut] = c_last;
+                ++ncut;
             }
-            named_sync(1, kEpi * 32);
-            const bool red = sh->reducer != 0;
-            named_sync(1, kEpi * 32);
-            if (!red) continue;
-            __threadfence();
-            for (int mt = 0; mt < q.MT; ++mt)
-                for (int c0 = 0; c0 < cols; c0 += 16) {
-                    float v[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
-                    for (int c = c_first; c <= c_last; ++c) {
-                        const float* pp = p.part + ((size_t)c * 2 + (c == c_first ? 0 : 1)) * slot_floats +
-                                          (size_t)mt * p.nb * kBM;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float x = __ldcg(pp + (size_t)(c0 + i) * kBM + row);
-                            if (p.paired) x += __ldcg(pp + (size_t)(p.npad + c0 + i) * kBM + row);
-                            v[i] += x;
-                        }
-                    }
-                    emit16(p, q, mbase + mt * kBM, c0, v, act);
-                }
         }
-        if (p.mode == kTcGateZ && p.ubits) {
-            // union bitmap words of this tile: one word per warp (32 channels)
-            const unsigned bits = __ballot_sync(0xffffffffu, act && !p.topk && mbase < p.m_total);
-            if (lane == 0) p.ubits[(s.t * kBM + ew * 32) >> 5] = bits;
-        }
+    }
+    // Every part of this CTA is out; now the quarter sums it owns: quarter j of
+    // a cut tile is summed by CTA c_first + j mod parts (one warp each).
+    for (int i = 0; i < ncut; ++i) {
+        const int parts = cut_last[i] - cut_first[i] + 1;
+        if (quarter % parts == (int)blockIdx.x - cut_first[i])
+            sum_quarter(p, cut_t[i], cut_m0[i], cut_first[i], cut_last[i], quarter, row, cols, slot_floats);
     }
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const TcParams p) {
+__global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant__ TcParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* stages = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                              ~static_cast<uintptr_t>(1023));
-    const uint32_t stage_bytes = (uint32_t)a_subtiles(p) * kTileA + (uint32_t)(p.ks * p.nb) * 128u;
+    const uint32_t stage_bytes = kTileA + (uint32_t)p.nb * 128u;
     TcShared* sh = reinterpret_cast<TcShared*>(stages + (size_t)p.stages * stage_bytes);
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; ++i) {
-            mbar_init(&sh->full[i], kProd * 32);
+            mbar_init(&sh->full[i], 1);
             mbar_init(&sh->empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -584,15 +555,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const TcParams p) {
     griddep_launch_dependents();
     griddep_wait();
     const Problem q = make_problem(p);
+    if (p.mode == kTcUp || p.mode == kTcDown) {
+        for (int i = threadIdx.x; i < q.nblk; i += kTcThreads) sh->blk[i] = __ldg(p.blk_list + i);
+        __syncthreads();
+    }
 
-    if (warp < kProd) {
-        if (p.stages >= 8) run_producer<6>(p, q, stages, stage_bytes, sh);
-        else if (p.stages >= 6) run_producer<4>(p, q, stages, stage_bytes, sh);
-        else run_producer<2>(p, q, stages, stage_bytes, sh);
-    } else if (warp < kProd + kEpi) {
+    if (warp == kProdWarp) {
+        if ((threadIdx.x & 31) == 0) run_producer(p, q, stages, stage_bytes, sh);
+    } else if (warp == kMmaWarp) {
+        if ((threadIdx.x & 31) == 0) run_mma(p, q, stages, stage_bytes, sh, tmem);
+    } else {
         run_epilogue(p, q, sh, tmem);
-    } else if ((threadIdx.x & 31) == 0) {
-        run_mma(p, q, stages, stage_bytes, sh, tmem);
     }
     tc_fence_before();
     __syncthreads();
@@ -602,84 +575,95 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const TcParams p) {
 
 // ---- union list ----------------------------------------------------------------
 // Ordered list of the channels any token selected (bit k of the bitmap), the
-// per-channel token masks, and the union size.
+// per-channel token masks, the union size, and the ordered list of 128-channel
+// blocks that hold at least one listed channel.
 
 constexpr int kUnionThreads = 1024;
 
+__device__ __forceinline__ int block_sum(int v, int* red) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int x = red[threadIdx.x];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (threadIdx.x == 0) red[32] = x;
+    }
+    __syncthreads();
+    const int r = red[32];
+    __syncthreads();
+    return r;
+}
+
+// Word w of the union bitmap (every channel when force_all), masked to d_ff.
+__device__ __forceinline__ uint32_t union_word(const UnionParams& p, int w, int nwords) {
+    const uint32_t tail = (w == nwords - 1 && (p.d_ff & 31)) ? (1u << (p.d_ff & 31)) - 1u : 0xffffffffu;
+    return (p.force_all ? 0xffffffffu : p.ubits[w]) & tail;
+}
+
 __global__ void __launch_bounds__(kUnionThreads) k_union(const UnionParams p) {
     __shared__ int sh[40];
-    __shared__ int s_red[32];
+    __shared__ int red[33];
     griddep_launch_dependents();
     griddep_wait();
     const int base = blockIdx.x * kUnionThreads;
     const int words_before = base >> 5;
     const int nwords = (p.d_ff + 31) >> 5;
-    // channels listed before this block: popcount of the bitmap words before it
-    int before = 0, total = 0;
-    if (p.force_all) {
-        before = base;
-        total = p.d_ff;
-    } else {
-        int a = 0, b = 0;
-        for (int w = threadIdx.x; w < nwords; w += kUnionThreads) {
-            const uint32_t bits = p.ubits[w];
-            const int c = __popc(w == nwords - 1 && (p.d_ff & 31) ? bits & ((1u << (p.d_ff & 31)) - 1u) : bits);
-            b += c;
-            if (w < words_before) a += c;
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            a += __shfl_xor_sync(0xffffffffu, a, o);
-            b += __shfl_xor_sync(0xffffffffu, b, o);
-        }
-        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = a;
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            int x = s_red[threadIdx.x];
-#pragma unroll
-            for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            if (threadIdx.x == 0) s_red[0] = x;
-        }
-        __syncthreads();
-        before = s_red[0];
-        __syncthreads();
-        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = b;
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            int x = s_red[threadIdx.x];
-#pragma unroll
-            for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            if (threadIdx.x == 0) s_red[1] = x;
-        }
-        __syncthreads();
-        total = s_red[1];
+    // channels listed before this block, and in all
+    int a = 0, b = 0;
+    for (int w = threadIdx.x; w < nwords; w += kUnionThreads) {
+        const int c = __popc(union_word(p, w, nwords));
+        b += c;
+        if (w < words_before) a += c;
     }
+    const int before = block_sum(a, red);
+    const int total = block_sum(b, red);
     const int k = base + threadIdx.x;
-    const bool in = k < p.d_ff && (p.force_all || ((p.ubits[k >> 5] >> (k & 31)) & 1u));
+    const bool in = k < p.d_ff && ((union_word(p, k >> 5, nwords) >> (k & 31)) & 1u);
     int tot = 0;
     const int rank = block_exclusive_scan(in ? 1 : 0, &tot, sh);
     if (in) {
         p.lst[before + rank] = k;
         for (int w = 0; w < p.mw; ++w) {
-            uint32_t m = 0;
+            uint32_t msk = 0;
             const int t1 = min(p.n, 32 * w + 32);
             for (int t = 32 * w; t < t1; ++t) {
                 const long long zi = (long long)t * p.d_ff + k;
                 const bool s = p.topk ? p.sel[zi] != 0 : p.z[zi] > p.tau;
-                m |= (s ? 1u : 0u) << (t - 32 * w);
+                msk |= (s ? 1u : 0u) << (t - 32 * w);
             }
-            p.lst_mask[(size_t)k * p.mw + w] = m;
+            p.lst_mask[(size_t)k * p.mw + w] = msk;
         }
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) *p.u_count = total;
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0) *p.u_count = total;
+        // 128-channel blocks with a listed channel, in order
+        const int nblk = (p.d_ff + 127) / 128;
+        int prior = 0;
+        for (int b0 = 0; b0 < nblk; b0 += kUnionThreads) {
+            const int bi = b0 + threadIdx.x;
+            bool act = false;
+            if (bi < nblk)
+                for (int w = 4 * bi; w < min(4 * bi + 4, nwords); ++w) act |= union_word(p, w, nwords) != 0;
+            int cnt = 0;
+            const int r = block_exclusive_scan(act ? 1 : 0, &cnt, sh);
+            if (act) p.blk_list[prior + r] = bi;
+            prior += cnt;
+        }
+        if (threadIdx.x == 0) *p.blk_count = prior;
+    }
 }
 
 SmemAttrCache g_tc_smem;
+std::once_flag g_enc_once;
+PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
 
 }  // namespace
 
-size_t tc_smem_bytes(int a_sub, int ks, int nb, int* stages) {
-    const size_t stage = (size_t)a_sub * kTileA + (size_t)ks * nb * 128;
+size_t tc_smem_bytes(int nb, int* stages) {
+    const size_t stage = kTileA + (size_t)nb * 128;
     int s = (int)((kMaxSmemPerCta - 1024 - sizeof(TcShared)) / stage);
     if (s > kMaxStages) s = kMaxStages;
     if (stages) *stages = s;
@@ -690,31 +674,49 @@ size_t tc_smem_bytes(int a_sub, int ks, int nb, int* stages) {
 cudaError_t launch_tc(const TcParams& p_in, int grid, cudaStream_t s, bool pdl) {
     TcParams p = p_in;
     if (p.nb < 16 || p.nb > 256 || p.nb % 16 || (p.paired && 2 * p.npad != p.nb)) return cudaErrorInvalidValue;
-    // One 64-wide k-block and one 128-row accumulator tile per iteration: the
-    // deepest ring of the smallest stages keeps the most bytes in flight.
-    p.ks = 1;
-    p.mt = 1;
+    if ((p.mode == kTcUp || p.mode == kTcDown) && p.blk_cap > kMaxBlocks) return cudaErrorInvalidValue;
     int st = 0;
-    size_t smem = 0;
-    for (;;) {
-        smem = tc_smem_bytes(p.mode == kTcDown ? p.mt : p.ks, p.ks, p.nb, &st);
-        if (smem || (p.ks == 1 && p.mt == 1)) break;
-        if (p.ks > 1) p.ks >>= 1; else p.mt >>= 1;
-    }
+    const size_t smem = tc_smem_bytes(p.nb, &st);
     if (!smem) return cudaErrorInvalidValue;
     p.stages = st;
     p.tmem_cols = 32;
-    const int acc_cols = (p.mode == kTcDown ? p.mt : 1) * p.nb;
-    while ((int)p.tmem_cols < 2 * acc_cols) p.tmem_cols <<= 1;
-    if (p.tmem_cols > 512) return cudaErrorInvalidValue;
+    while ((int)p.tmem_cols < 2 * p.nb) p.tmem_cols <<= 1;
     cudaError_t e = ensure_smem(k_tc_gemm, smem, g_tc_smem);
     if (e != cudaSuccess) return e;
     return launch_ex(k_tc_gemm, dim3(grid), dim3(kTcThreads), smem, s, pdl, p);
 }
 
 cudaError_t launch_union(const UnionParams& p, cudaStream_t s, bool pdl) {
+    if ((p.d_ff + 127) / 128 > kMaxBlocks) return cudaErrorInvalidValue;
     const int grid = (p.d_ff + kUnionThreads - 1) / kUnionThreads;
     return launch_ex(k_union, dim3(grid), dim3(kUnionThreads), 0, s, pdl, p);
+}
+
+// 2-D bf16 tensor map (row-major, `cols` contiguous elements per row) with a
+// box of box_cols x box_rows elements and the 128-byte swizzle; elements
+// outside the tensor read as zero.  The driver's encoder is fetched once
+// through the runtime.
+cudaError_t encode_tile_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                            uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows) {
+    std::call_once(g_enc_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_enc) return cudaErrorNotSupported;
+    if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_stride_bytes & 15) || cols == 0 || rows == 0 ||
+        box_cols * 2 > 128 || box_rows > 256)
+        return cudaErrorInvalidValue;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 }  // namespace sffn
