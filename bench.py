@@ -117,16 +117,17 @@ def kernel_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel: str, workload: str):
+def traffic_for(kernel: str, workload: str, tokens: int):
     """Per-launch DRAM bytes from a committed ncu capture, if it was taken on
-    the current kernel sources."""
+    the current kernel sources (keyed by workload and token count)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             data = json.load(f)
     except (OSError, ValueError):
         return None
-    ent = data.get(workload, {}).get(kernel)
+    ent = (data.get(f"{workload}:n{tokens}") or data.get(workload, {}) if tokens > 1 else
+           data.get(workload, {})).get(kernel)
     if not ent or ent.get("kernel_hash") != kernel_hash():
         return None
     return ent.get("dram_bytes_per_launch")
@@ -452,7 +453,7 @@ def main():
     roofline = {"bound": "hbm", "kernel": dom_name, "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic_for(dom_name, a.workload),
+                "traffic": traffic_for(dom_name, a.workload, wl.n),
                 "algorithmic_bytes_per_launch": int(dom_bytes),
                 "avg_launch_us": round(avg_launch_ms * 1e3, 3),
                 "kernel_timing": (f"timed region per step x the kernel's share of the step; shares from "
