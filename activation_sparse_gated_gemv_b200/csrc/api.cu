@@ -89,7 +89,7 @@ struct sffn_ctx {
     int* seg_count = nullptr;
     float* u = nullptr;
     float* dpart = nullptr;
-    float* fpart = nullptr;
+    float* fpart = nullptr;      // fused decode: [g1][min(max_tokens, 4)][d] partials of y
     unsigned* tickets = nullptr;
     int* status = nullptr;
     void* xdev = nullptr;
@@ -310,7 +310,8 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     size_t dec_smem = 0;
     const int dec_nt = pick_nt(n);
     const bool fused = sel->kind == SFFN_SELECT_THRESHOLD && !dense && n <= kDecodeMaxTokens &&
-                       decode_geometry(dec_nt, c.d, lopa ? c.lopa_rank : 0, gk, P.cpb, P.mw, &dec_sb, &dec_nb,
+                       decode_geometry(dec_nt, c.d, lopa ? c.lopa_rank : 0, gk, P.cpb, P.mw,
+                                       c.wdtype == SFFN_BF16 ? 8 : 4, P.g1, &dec_sb, &dec_nb,
                                        &dec_smem);
 
     h->last_tc = false;
@@ -335,8 +336,6 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
         dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.part = h->fpart;
         dp.tickets = h->tickets; dp.y = out;
-        dp.reducers = 32;
-        while (dp.reducers > 1 && (c.d % (4 * dp.reducers) || dp.reducers > P.g1)) dp.reducers /= 2;
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
         h->last_names[launches] = "decode_fused";
         record(h, ++launches, s);

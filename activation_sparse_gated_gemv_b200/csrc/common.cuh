@@ -104,6 +104,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -253,15 +258,14 @@ struct DecodeParams {
     const void* wdn;        // [d_ff][d]
     float tau;
     int cpb, mw;
-    int* lst_idx;
-    float* lst_h;           // [d_ff][n]
+    int* lst_idx;           // [CTAs][cpb] each CTA's active channels, ascending
+    float* lst_h;           // unused by the fused kernel
     uint32_t* lst_mask;     // [d_ff][mw]
     int* seg_count;         // [CTAs]
     int sb, nb;             // streamed piece bytes, pieces in flight per streaming warp
     int* status;
     float* part;            // [CTAs][n][d] per-CTA partials of y
-    unsigned* tickets;      // [2] zero between forwards
-    int reducers;           // CTAs that sum the partials (d / reducers a multiple of 4)
+    unsigned* tickets;      // [2] grid-barrier counters, zero between forwards
     void* y;                // [n][d] T
 };
 
@@ -375,7 +379,8 @@ size_t down_smem_bytes(int wdtype, int nt, int nseg, int cpb);
 int down_slice_cols(int wdtype);
 cudaError_t launch_transpose(int wdtype, const void* src, void* dst, int rows, int cols,
                              cudaStream_t s);
-bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* sb, int* nb, size_t* smem);
+bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int vec, int grid, int* sb, int* nb,
+                     size_t* smem);
 cudaError_t launch_decode(int wdtype, const DecodeParams& p, int nt, int gate_kind, int grid, size_t smem,
                           cudaStream_t s, bool pdl);
 constexpr int kDecodeMaxTokens = 4;   // the fused decode path takes up to this many tokens

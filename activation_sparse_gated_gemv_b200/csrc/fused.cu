@@ -1,6 +1,6 @@
 // Fused decode path (threshold selection, a few tokens): one kernel streams
 // the gate, selects, takes the up dots, adds the CTA's share of the down
-// projection and sums the per-CTA partials.
+// projection and sums the per-CTA partials, one column slice per CTA.
 //
 // "Model Casting and Low-Parameter Gating" (abstract): the gating matrix is
 // evaluated first and the two other matrices are touched only for channels
@@ -17,10 +17,10 @@
 //     their pieces are done), so the W_up rows are read while the gate streams;
 //   * after a barrier the active channels are compacted in ascending order
 //     and every thread adds, for its 8 (or 4) output columns, h_k W_down[k,:]
-//     over that ordered list (rows mostly in L2 by now), and stores the CTA's
-//     fp32 partial of y.
-//   * each CTA writes its partial and takes a ticket; the last few CTAs sum
-//     the partials of a column slice each, in CTA order, and store y.
+//     over that ordered list (whole rows, mostly in L2 by now), and stores the
+//     CTA's fp32 partial of y;
+//   * a grid-wide barrier, then every CTA sums one column slice of y over all
+//     CTAs' partials (in L2) in a fixed order and stores it.
 // Every sum has a fixed order, so y is bitwise reproducible.
 #include "common.cuh"
 #include "dot.cuh"
@@ -35,8 +35,20 @@ constexpr int kQueueTail = 0, kQueueHead = 1, kGateDone = 2, kAbort = 3;
 struct DecodeSmem {
     size_t xs, us, zpart, zfin, hs, done, queue, ctr, wl, mask, flag, scan, bars, bufs, total;
 };
+
+// Chunks (16 bytes of `vec` elements) per column slice of the down pass: the
+// smallest power of two covering d with `grid` slices.
+__host__ __device__ inline int decode_slice_chunks(int d, int vec, int grid) {
+    int cps = 1;
+    while (cps * vec * grid < d) cps <<= 1;
+    return cps;
+}
+// Bytes the cross-CTA sum keeps in the (then idle) streaming ring.
+__host__ __device__ inline size_t decode_tail_bytes(int, int, int, int) {
+    return (size_t)kDecThreads * 16;                     // one float4 per thread for the partial sums
+}
 __host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, int gate_kind, int cpb, int mw,
-                                                         int sb, int nb) {
+                                                         int sb, int nb, int vec, int grid) {
     DecodeSmem L;
     const int glen = gate_kind == kGateLopa ? r : d;
     const int rb = glen * 4;                      // fp32 rows: an upper bound on the part count
@@ -57,7 +69,9 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, i
     o = (o + 15) & ~(size_t)15;
     L.bars = o;  o += (size_t)kDecStreamWarps * nb * sizeof(uint64_t);
     o = (o + 127) & ~(size_t)127;
-    L.bufs = o;  o += (size_t)kDecStreamWarps * nb * sb;
+    L.bufs = o;
+    const size_t ring = (size_t)kDecStreamWarps * nb * sb, tail = decode_tail_bytes(nt, d, vec, grid);
+    o += ring > tail ? ring : tail;
     L.total = o;
     return L;
 }
@@ -70,7 +84,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     const int c0 = blockIdx.x * p.cpb;
     const int nslots = max(0, min(p.cpb, p.d_ff - c0));
     const int n = p.n;                                  // n <= NT
-    const DecodeSmem L = decode_smem_layout(NT, p.d, p.r, GATE, p.cpb, p.mw, p.sb, p.nb);
+    const DecodeSmem L = decode_smem_layout(NT, p.d, p.r, GATE, p.cpb, p.mw, p.sb, p.nb, V, gridDim.x);
     float* xs = reinterpret_cast<float*>(smem + L.xs);
     float* us = reinterpret_cast<float*>(smem + L.us);
     float* zpart = reinterpret_cast<float*>(smem + L.zpart);
@@ -301,7 +315,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             if (lane == t && t < n) {
                 const float h = ((tokmask >> t) & 1u) ? (zfin[s * NT + t] - p.tau) * u[t] : 0.f;
                 hs[s * NT + t] = h;
-                p.lst_h[(size_t)k * n + t] = h;
             }
     }
     __syncthreads();
@@ -327,6 +340,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     }
     if (threadIdx.x == 0) p.seg_count[blockIdx.x] = tot;
 
+    // ---- the CTA's share of the down projection: h_k W_down[k, :] over its
+    // active channels in list order (whole rows, mostly in L2 by now), as an
+    // fp32 partial of y.
     constexpr int UB = 8;
     const int cpd = p.d / V;                              // 16-byte chunks per output row
     for (int cch = threadIdx.x; cch < cpd; cch += kDecThreads) {
@@ -369,87 +385,82 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         }
     }
 
-    // ---- cross-CTA sum.  Each CTA takes a ticket once its partial is out; the
-    // last `reducers` CTAs wait (bounded) until every partial is written, then
-    // each adds a column slice over all CTAs in CTA order and stores y.  They
-    // wait only on CTAs that are already running, so this cannot deadlock.
+    // ---- grid barrier: every CTA's partial is out.  All CTAs are resident
+    // (one per SM, grid <= SMs, and a dependent launch waits until every CTA of
+    // this grid has started), so the wait ends; it is bounded all the same.
+    // A CTA without a column slice only arrives.
+    const int G = gridDim.x;
+    const int cps = decode_slice_chunks(p.d, V, G);       // 16-byte chunks per column slice
+    const int col0 = blockIdx.x * cps * V;
     __threadfence();
     __syncthreads();
-    const int parts = gridDim.x;
-    const int reducers = p.reducers;
-    if (threadIdx.x == 0) scan_sh[1] = (int)atomicAdd(p.tickets, 1u);
-    __syncthreads();
-    const int rank = scan_sh[1] - (parts - reducers);
-    if (rank < 0) return;
     if (threadIdx.x == 0) {
-        const unsigned long long t0 = globaltimer_ns();
+        atomicAdd(p.tickets, 1u);
         int ok = 1;
-        while (*reinterpret_cast<volatile unsigned*>(p.tickets) < (unsigned)parts) {
-            __nanosleep(128);
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                atomicOr(p.status, (int)kStatusWaitTimeout);
-                ok = 0;
-                break;
+        if (col0 < p.d) {
+            const unsigned long long t0 = globaltimer_ns();
+            unsigned backoff = 32;
+            while (ld_acquire_u32(p.tickets) < (unsigned)G) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(backoff);
+                if (backoff < 256) backoff <<= 1;
             }
         }
         scan_sh[2] = ok;
-        __threadfence();
     }
     __syncthreads();
-    if (scan_sh[2]) {
-        const int cols = p.d / reducers;                    // a multiple of 4
-        const int col0 = rank * cols;
-        const int c4n = cols / 4;
-        const int items = n * c4n;
-        const int G = items >= kDecThreads ? 1 : kDecThreads / items;
-        const int per_round = kDecThreads / G;
-        float4* gsum = reinterpret_cast<float4*>(smem + L.bufs);   // the streaming ring, idle now
-        const size_t stride = (size_t)n * p.d / 4;
-        T* y = static_cast<T*>(p.y);
-        for (int base = 0; base < items; base += per_round) {
-            const int item = base + (int)threadIdx.x % per_round;
-            const int grp = (int)threadIdx.x / per_round;
-            const int t = item / c4n, c = col0 + (item - t * c4n) * 4;
-            const bool ok = item < items && grp < G;
+    if (scan_sh[2] && col0 < p.d) {
+        __threadfence();
+        // y[:, col0 : col0 + cps V] = sum over the G partials.  Thread (g, item)
+        // adds partials g, g + GR, ... in order; then the GR sums in order.
+        const int q4 = min(cps * V, p.d - col0) / 4;     // float4 per token
+        const int items = n * q4;
+        const int GR = max(1, kDecThreads / items);
+        float4* red = reinterpret_cast<float4*>(smem + L.bufs);          // the idle ring
+        const int g = (int)threadIdx.x / items, item = (int)threadIdx.x - g * items;
+        if (g < GR) {
+            const int t = item / q4, c = col0 + (item - t * q4) * 4;
             float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (ok) {
-                const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)t * p.d + c);
-                for (int b = grp; b < parts; b += 16 * G) {
-                    float4 v[16];
+            constexpr int UB = 16;
+            for (int b0 = g; b0 < G; b0 += UB * GR) {
+                float4 v[UB];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int b2 = b + q * G;
-                        v[q] = b2 < parts ? __ldcg(src + (size_t)b2 * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        if (b + q * G < parts) {
-                            sum.x += v[q].x; sum.y += v[q].y; sum.z += v[q].z; sum.w += v[q].w;
-                        }
+                for (int u2 = 0; u2 < UB; ++u2) {
+                    const int b = b0 + u2 * GR;
+                    v[u2] = b < G ? __ldcg(reinterpret_cast<const float4*>(p.part + ((size_t)b * n + t) * p.d + c))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-            }
-            if (G > 1) {
-                __syncthreads();
-                gsum[threadIdx.x] = sum;
-                __syncthreads();
-                if (grp == 0 && ok)
-                    for (int q = 1; q < G; ++q) {
-                        const float4 v = gsum[q * per_round + (int)threadIdx.x % per_round];
-                        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+#pragma unroll
+                for (int u2 = 0; u2 < UB; ++u2)
+                    if (b0 + u2 * GR < G) {
+                        sum.x += v[u2].x; sum.y += v[u2].y; sum.z += v[u2].z; sum.w += v[u2].w;
                     }
             }
-            if (grp == 0 && ok) {
-                T* dst = y + (size_t)t * p.d + c;
-                dst[0] = from_f32<T>(sum.x);
-                dst[1] = from_f32<T>(sum.y);
-                dst[2] = from_f32<T>(sum.z);
-                dst[3] = from_f32<T>(sum.w);
+            red[g * items + item] = sum;
+        }
+        __syncthreads();
+        if ((int)threadIdx.x < items) {
+            float4 sum = red[threadIdx.x];
+            for (int q = 1; q < GR; ++q) {
+                const float4 v = red[q * items + threadIdx.x];
+                sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
             }
+            const int t = (int)threadIdx.x / q4, c = col0 + ((int)threadIdx.x - t * q4) * 4;
+            T* dst = static_cast<T*>(p.y) + (size_t)t * p.d + c;
+            dst[0] = from_f32<T>(sum.x);
+            dst[1] = from_f32<T>(sum.y);
+            dst[2] = from_f32<T>(sum.z);
+            dst[3] = from_f32<T>(sum.w);
         }
     }
-    // The last reducer to finish resets the tickets for the next forward.
+    // The last CTA through resets the barrier counters for the next forward
+    // (every CTA has left the barrier by then).
     __syncthreads();
-    if (threadIdx.x == 0 && atomicAdd(p.tickets + 1, 1u) == (unsigned)reducers - 1u) {
+    if (threadIdx.x == 0 && atomicAdd(p.tickets + 1, 1u) == gridDim.x - 1u) {
         p.tickets[0] = 0u;
         p.tickets[1] = 0u;
         __threadfence();
@@ -458,15 +469,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
 
 // ---------------------------------------------------------------------------
 
-size_t decode_smem_bytes(int nt, int d, int r, int gate_kind, int cpb, int mw, int sb, int nb) {
-    return decode_smem_layout(nt, d, r, gate_kind, cpb, mw, sb, nb).total;
+size_t decode_smem_bytes(int nt, int d, int r, int gate_kind, int cpb, int mw, int sb, int nb, int vec, int grid) {
+    return decode_smem_layout(nt, d, r, gate_kind, cpb, mw, sb, nb, vec, grid).total;
 }
 
-bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* sb, int* nb, size_t* smem) {
+bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int vec, int grid, int* sb, int* nb,
+                     size_t* smem) {
+    // the cross-CTA sum gives one thread to each (token, 4 columns) of a slice
+    if (grid < 1 || (long)nt * decode_slice_chunks(d, vec, grid) * vec / 4 > kDecThreads) return false;
     int best_sb = 0, best_nb = 0;
     for (int cand_sb : {8192, 4096, 2048})
         for (int cand_nb = 2; cand_nb <= 4; ++cand_nb) {
-            if (decode_smem_bytes(nt, d, r, gate_kind, cpb, mw, cand_sb, cand_nb) > kMaxSmemPerCta) continue;
+            if (decode_smem_bytes(nt, d, r, gate_kind, cpb, mw, cand_sb, cand_nb, vec, grid) > kMaxSmemPerCta)
+                continue;
             const long cur = (long)cand_sb * cand_nb, best = (long)best_sb * best_nb;
             if (cur > best || (cur == best && cand_nb > best_nb)) {
                 best_sb = cand_sb;
@@ -476,7 +491,7 @@ bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int* 
     if (!best_sb) return false;
     *sb = best_sb;
     *nb = best_nb;
-    *smem = decode_smem_bytes(nt, d, r, gate_kind, cpb, mw, best_sb, best_nb);
+    *smem = decode_smem_bytes(nt, d, r, gate_kind, cpb, mw, best_sb, best_nb, vec, grid);
     return true;
 }
 
