@@ -4,7 +4,7 @@
 // weight repacking, and the kernel sequence of one forward:
 //   threshold, n <= 4:  [LoPA x A] -> one fused decode kernel
 //   n > 4, bf16 (tensor cores):
-//               gate GEMM (z) [-> top-K] -> union list -> up GEMM -> down GEMM
+//               gate GEMM (z, union bitmap) [-> top-K] -> up GEMM -> down GEMM
 //               (LoPA: x A GEMM, then the z GEMM)
 //   otherwise:  [LoPA x A] -> gate+select+up -> down, or for top-K
 //               [LoPA x A] -> gate (z) -> top-K -> preselected up -> down
@@ -99,16 +99,16 @@ struct sffn_ctx {
     int tc_npad_max = 0;
     long long tc_ldh = 0;
     uint32_t* ubits = nullptr;
-    int* u_count = nullptr;
+
     void* h2 = nullptr;          // [2 npad][tc_ldh] bf16: h as hi/lo rows
     void* u2 = nullptr;          // [2 npad][r] bf16: LoPA x A as hi/lo rows
     float* tc_part = nullptr;    // [sms][2][128][256]
     unsigned* tc_tickets = nullptr;
-    int* blk_list = nullptr;     // 128-channel blocks holding a selected channel
-    int* blk_count = nullptr;
     bool maps_ok = false;        // weight tensor maps encoded
     CUtensorMap map_wg{}, map_at{}, map_bcm{}, map_wup{}, map_wdn{};
-    bool last_tc = false;
+    bool last_tc = false;        // the last forward took the tensor-core path
+    bool last_topk = false;
+    float last_tau = 0.f;
     Plan plan;
     int last_n = -1;
     cudaStream_t last_stream = nullptr;
@@ -195,8 +195,9 @@ int check_forward(const sffn_ctx* h, const void* x, int n, int gate_mode, const 
     return SFFN_OK;
 }
 
-// Batched forward on the tensor cores: gate GEMM -> [top-K] -> union list ->
-// up GEMM -> down GEMM, every GEMM one stream-K tcgen05 kernel over all SMs.
+// Batched forward on the tensor cores: gate GEMM -> [top-K] -> up GEMM ->
+// down GEMM, every GEMM one stream-K tcgen05 kernel over all SMs; the up and
+// down kernels find the active channel blocks in the gate's union bitmap.
 // Returns SFFN_ERR_UNSUPPORTED (nothing launched) when a tensor map cannot be
 // made for this call; the caller then takes the CUDA-core path.
 int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel, void* out, cudaStream_t s,
@@ -256,20 +257,10 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
         record(h, ++launches, s);
     }
 
-    UnionParams up{};
-    up.ubits = h->ubits; up.d_ff = c.d_ff; up.n = n; up.mw = h->plan.mw;
-    up.z = h->zbuf; up.sel = h->sel; up.tau = tau; up.topk = topk ? 1 : 0; up.force_all = dense ? 1 : 0;
-    up.lst = h->lst_idx; up.u_count = h->u_count; up.lst_mask = h->lst_mask;
-    up.blk_list = h->blk_list; up.blk_count = h->blk_count;
-    SFFN_CUDA(launch_union(up, s, true), "union list launch");
-    h->last_names[launches] = "union";
-    record(h, ++launches, s);
-
-    const int nblk = (c.d_ff + 127) / 128;
     TcParams w = base;                          // h = g * <x, W_up[ch]> over the active channel blocks
     w.mode = kTcUp;
     w.ta = h->map_wup; w.tb = map_x;
-    w.blk_list = h->blk_list; w.blk_count = h->blk_count; w.blk_cap = nblk;
+    w.ubits = h->ubits; w.d_ff = c.d_ff; w.force_all = dense ? 1 : 0;
     w.m_total = c.d_ff; w.k_total = c.d; w.nb = npad;
     w.out = h->h2; w.ldo = h->tc_ldh; w.h_pairs = 1;
     w.zsel = h->zbuf; w.gsel = h->gbuf; w.ldsel = c.d_ff;
@@ -280,7 +271,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     TcParams dn = base;                         // y = sum over the active blocks of h W_down[ch]
     dn.mode = kTcDown;
     dn.ta = h->map_wdn; dn.tb = map_h2;
-    dn.blk_list = h->blk_list; dn.blk_count = h->blk_count; dn.blk_cap = nblk;
+    dn.ubits = h->ubits; dn.d_ff = c.d_ff; dn.force_all = dense ? 1 : 0;
     dn.m_total = c.d; dn.nb = 2 * npad; dn.paired = 1;
     dn.out = out; dn.ldo = c.d;
     SFFN_CUDA(launch_tc(dn, h->sms, s, true), "tensor-core down launch");
@@ -291,6 +282,8 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     h->last_stream = s;
     h->last_launches = launches;
     h->last_tc = true;
+    h->last_topk = topk;
+    h->last_tau = tau;
     return SFFN_OK;
 }
 
@@ -492,11 +485,10 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t NP = h->tc ? (size_t)h->tc_npad_max : 0;
     const size_t FDR = F > D ? (F > R ? F : R) : (D > R ? D : R);
     const size_t tiles = round_up(FDR, 128) / 128 + 1;
-    const size_t o_ub = take(h->tc ? tiles * 4 * 4 : 0), o_uc = take(h->tc ? 4 : 0);
+    const size_t o_ub = take(h->tc ? tiles * 4 * 4 : 0);
     const size_t o_h2 = take(2 * NP * (size_t)h->tc_ldh * 2), o_u2 = take(2 * NP * R * 2);
     // stream-K partial tiles: two slots per CTA of up to 256 accumulator columns x 128 rows
     const size_t o_tp = take(h->tc ? (size_t)h->sms * 2 * 256 * 128 * 4 : 0), o_tt = take(h->tc ? tiles * 8 : 0);
-    const size_t o_bl = take(h->tc ? (round_up(F, 128) / 128 + 1) * 4 : 0), o_bc = take(h->tc ? 4 : 0);
     e = cudaMalloc(&h->ws, off);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "workspace allocation"); }
     char* b = static_cast<char*>(h->ws);
@@ -516,13 +508,10 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->ydev = b + o_y;
     if (h->tc) {
         h->ubits = reinterpret_cast<uint32_t*>(b + o_ub);
-        h->u_count = reinterpret_cast<int*>(b + o_uc);
         h->h2 = b + o_h2;
         h->u2 = b + o_u2;
         h->tc_part = reinterpret_cast<float*>(b + o_tp);
         h->tc_tickets = reinterpret_cast<unsigned*>(b + o_tt);
-        h->blk_list = reinterpret_cast<int*>(b + o_bl);
-        h->blk_count = reinterpret_cast<int*>(b + o_bc);
     }
     e = cudaMemset(h->ws, 0, off);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -665,26 +654,31 @@ int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union
     std::vector<int> seg(P.g1), lidx(F);
     std::vector<uint32_t> mask((size_t)F * P.mw);
     if (h->last_tc) {
-        // one ordered union list of u_count entries
-        int U = 0;
-        SFFN_CUDA(cudaMemcpy(&U, h->u_count, 4, cudaMemcpyDeviceToHost), "list copy");
-        if (U < 0 || U > F) return fail(SFFN_ERR_DEVICE_CHECK, "union size %d", U);
-        SFFN_CUDA(cudaMemcpy(lidx.data(), h->lst_idx, (size_t)U * 4, cudaMemcpyDeviceToHost), "list copy");
-        SFFN_CUDA(cudaMemcpy(mask.data(), h->lst_mask, mask.size() * 4, cudaMemcpyDeviceToHost), "list copy");
+        // the tensor-core path keeps the gate's decisions, not lists: z (threshold,
+        // the same fp32 comparison the kernels make) or the top-K mask
         for (int t = 0; t < n; ++t) counts[t] = 0;
-        int uni = 0, prev = -1;
-        for (int i = 0; i < U; ++i) {
-            const int k = lidx[i];
-            if (k <= prev || k >= F) return fail(SFFN_ERR_DEVICE_CHECK, "union list entry %d = %d", i, k);
-            prev = k;
-            bool any = false;
+        std::vector<uint8_t> any(F, 0);
+        if (h->last_topk) {
+            std::vector<uint8_t> selv((size_t)n * F);
+            SFFN_CUDA(cudaMemcpy(selv.data(), h->sel, selv.size(), cudaMemcpyDeviceToHost), "mask copy");
             for (int t = 0; t < n; ++t)
-                if ((mask[(size_t)k * P.mw + (t >> 5)] >> (t & 31)) & 1u) {
-                    idx[(size_t)t * F + counts[t]++] = k;
-                    any = true;
-                }
-            uni += any;
+                for (int k = 0; k < F; ++k)
+                    if (selv[(size_t)t * F + k]) {
+                        idx[(size_t)t * F + counts[t]++] = k;
+                        any[k] = 1;
+                    }
+        } else {
+            std::vector<float> z((size_t)n * F);
+            SFFN_CUDA(cudaMemcpy(z.data(), h->zbuf, z.size() * 4, cudaMemcpyDeviceToHost), "gate copy");
+            for (int t = 0; t < n; ++t)
+                for (int k = 0; k < F; ++k)
+                    if (z[(size_t)t * F + k] > h->last_tau) {
+                        idx[(size_t)t * F + counts[t]++] = k;
+                        any[k] = 1;
+                    }
         }
+        int uni = 0;
+        for (int k = 0; k < F; ++k) uni += any[k];
         if (union_size) *union_size = uni;
         return SFFN_OK;
     }

@@ -283,9 +283,8 @@ struct alignas(64) TcParams {
     int mode;
     int m_total;            // output rows: gate rows, d_ff (up), d (down)
     int k_total;            // contraction length of gate and up
-    const int* blk_list;    // up, down: 128-channel blocks holding a selected channel, ascending
-    const int* blk_count;
-    int blk_cap;
+    int d_ff;               // up, down: channels (bits of the union bitmap)
+    int force_all;          // up, down: every channel block (the dense FFN)
     int n, npad, nb;        // tokens, tokens padded to 16, MMA N (npad or 2 npad)
     int paired;             // accumulator columns t and npad+t are hi and lo parts
     int h_pairs;            // up: also write the lo rows of h (B of a paired down)
@@ -298,7 +297,7 @@ struct alignas(64) TcParams {
     long long ldsel;
     float tau;
     int topk;
-    uint32_t* ubits;        // gate: union bitmap out (threshold), zeroed (top-K)
+    uint32_t* ubits;        // gate: union bitmap out (threshold), zeroed (top-K); up, down: read
     float* part;            // [CTAs][2][128][nb] stream-K partial tiles
     unsigned* tickets;      // two counters per tile (parts arrived, quarters summed), zero between launches
     int* status;
@@ -306,19 +305,6 @@ struct alignas(64) TcParams {
     uint32_t tmem_cols;     // set by the launcher
 };
 
-struct UnionParams {
-    const uint32_t* ubits;  // [ceil(d_ff/32)]
-    int d_ff, n, mw;
-    const float* z;         // threshold: [n][d_ff]
-    const uint8_t* sel;     // top-K: [n][d_ff]
-    float tau;
-    int topk, force_all;
-    int* lst;               // [d_ff] ordered union
-    int* u_count;
-    uint32_t* lst_mask;     // [d_ff][mw] tokens that selected each listed channel
-    int* blk_list;          // [ceil(d_ff/128)] 128-channel blocks holding a listed channel
-    int* blk_count;
-};
 
 // Bits of the device status word.
 enum StatusBits { kStatusWaitTimeout = 2 };
@@ -388,7 +374,6 @@ size_t tc_smem_bytes(int nb, int* stages);
 cudaError_t encode_tile_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                             uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
 cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_union(const UnionParams& p, cudaStream_t s, bool pdl);
 constexpr int kTcMaxTokens = 128;     // token columns of one tensor-core pass (hi/lo pairs fill N = 256)
 
 }  // namespace sffn

@@ -17,7 +17,7 @@
 //
 // Rows are skipped at the granularity of 128-channel blocks: the up and down
 // passes read every block holding at least one channel that some token of the
-// batch selected (a channel of such a block that a token did not select gets
+// batch selected (each CTA finds them from the gate's union bitmap) (a channel of such a block that a token did not select gets
 // g = 0 for it).  With several independent tokens nearly every block holds one
 // (a block is skipped only if all its 128 channels stay inactive for every
 // token), so the batched passes read what a per-channel gather would, in whole
@@ -62,7 +62,8 @@ constexpr int kTcThreads = (kEpiWarp0 + kEpi) * 32;
 constexpr uint32_t kTileA = kBM * kBK * 2;   // 16 KB
 constexpr int kMaxStages = 12;
 constexpr int kMaxBlocks = 1024;    // 128-channel blocks (d_ff <= 131072)
-constexpr int kMinIters = 16;       // iterations per CTA at least, so few tiles are cut many ways
+constexpr int kMinIters = 8;        // iterations per CTA at least
+constexpr int kMaxParts = 8;        // CTAs sharing one tile at most
 
 struct TcShared {
     uint64_t full[kMaxStages];
@@ -73,6 +74,7 @@ struct TcShared {
     uint32_t tmem_base;
     int abort;
     int reducer;
+    int wcount[kTcThreads / 32];
     int blk[kMaxBlocks];    // up/down: the active 128-channel blocks
 };
 
@@ -195,9 +197,9 @@ struct Problem {
     long long I, it0, it1;
 };
 
-__device__ __forceinline__ Problem make_problem(const TcParams& p) {
+__device__ __forceinline__ Problem make_problem(const TcParams& p, int nblk) {
     Problem q;
-    q.nblk = p.blk_count ? min(max(*p.blk_count, 0), min(p.blk_cap, kMaxBlocks)) : 0;
+    q.nblk = nblk;
     if (p.mode == kTcUp) {
         q.T = q.nblk;
         q.KB = (p.k_total + kBK - 1) / kBK;
@@ -209,7 +211,7 @@ __device__ __forceinline__ Problem make_problem(const TcParams& p) {
         q.KB = (p.k_total + kBK - 1) / kBK;
     }
     q.I = (long long)q.T * q.KB;
-    q.C = (int)min((long long)gridDim.x, (q.I + kMinIters - 1) / kMinIters);
+    q.C = (int)min(min((long long)gridDim.x, (q.I + kMinIters - 1) / kMinIters), (long long)q.T * kMaxParts);
     if ((int)blockIdx.x < q.C) {
         q.it0 = q.I * blockIdx.x / q.C;
         q.it1 = q.I * (blockIdx.x + 1) / q.C;
@@ -554,11 +556,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
 
     griddep_launch_dependents();
     griddep_wait();
-    const Problem q = make_problem(p);
+    int nblk = 0;
     if (p.mode == kTcUp || p.mode == kTcDown) {
-        for (int i = threadIdx.x; i < q.nblk; i += kTcThreads) sh->blk[i] = __ldg(p.blk_list + i);
-        __syncthreads();
+        // the 128-channel blocks holding a channel some token selected, from the union bitmap
+        const int nbk = (p.d_ff + 127) / 128, nwords = (p.d_ff + 31) >> 5;
+        const int lane = threadIdx.x & 31;
+        for (int b0 = 0; b0 < nbk; b0 += kTcThreads) {
+            const int bi = b0 + threadIdx.x;
+            bool act = false;
+            if (bi < nbk) {
+                if (p.force_all) {
+                    act = true;
+                } else {
+                    for (int w = 4 * bi; w < min(4 * bi + 4, nwords); ++w) {
+                        uint32_t bits = __ldcg(p.ubits + w);
+                        if (w == nwords - 1 && (p.d_ff & 31)) bits &= (1u << (p.d_ff & 31)) - 1u;
+                        act |= bits != 0u;
+                    }
+                }
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, act);
+            if (lane == 0) sh->wcount[warp] = __popc(m);
+            __syncthreads();
+            int before = nblk;
+            for (int w2 = 0; w2 < warp; ++w2) before += sh->wcount[w2];
+            if (act) sh->blk[before + __popc(m & ((1u << lane) - 1u))] = bi;
+            for (int w2 = 0; w2 < kTcThreads / 32; ++w2) nblk += sh->wcount[w2];
+            __syncthreads();
+        }
     }
+    const Problem q = make_problem(p, nblk);
 
     if (warp == kProdWarp) {
         if ((threadIdx.x & 31) == 0) run_producer(p, q, stages, stage_bytes, sh);
@@ -571,89 +598,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, p.tmem_cols);
-}
-
-// ---- union list ----------------------------------------------------------------
-// Ordered list of the channels any token selected (bit k of the bitmap), the
-// per-channel token masks, the union size, and the ordered list of 128-channel
-// blocks that hold at least one listed channel.
-
-constexpr int kUnionThreads = 1024;
-
-__device__ __forceinline__ int block_sum(int v, int* red) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        int x = red[threadIdx.x];
-#pragma unroll
-        for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (threadIdx.x == 0) red[32] = x;
-    }
-    __syncthreads();
-    const int r = red[32];
-    __syncthreads();
-    return r;
-}
-
-// Word w of the union bitmap (every channel when force_all), masked to d_ff.
-__device__ __forceinline__ uint32_t union_word(const UnionParams& p, int w, int nwords) {
-    const uint32_t tail = (w == nwords - 1 && (p.d_ff & 31)) ? (1u << (p.d_ff & 31)) - 1u : 0xffffffffu;
-    return (p.force_all ? 0xffffffffu : p.ubits[w]) & tail;
-}
-
-__global__ void __launch_bounds__(kUnionThreads) k_union(const UnionParams p) {
-    __shared__ int sh[40];
-    __shared__ int red[33];
-    griddep_launch_dependents();
-    griddep_wait();
-    const int base = blockIdx.x * kUnionThreads;
-    const int words_before = base >> 5;
-    const int nwords = (p.d_ff + 31) >> 5;
-    // channels listed before this block, and in all
-    int a = 0, b = 0;
-    for (int w = threadIdx.x; w < nwords; w += kUnionThreads) {
-        const int c = __popc(union_word(p, w, nwords));
-        b += c;
-        if (w < words_before) a += c;
-    }
-    const int before = block_sum(a, red);
-    const int total = block_sum(b, red);
-    const int k = base + threadIdx.x;
-    const bool in = k < p.d_ff && ((union_word(p, k >> 5, nwords) >> (k & 31)) & 1u);
-    int tot = 0;
-    const int rank = block_exclusive_scan(in ? 1 : 0, &tot, sh);
-    if (in) {
-        p.lst[before + rank] = k;
-        for (int w = 0; w < p.mw; ++w) {
-            uint32_t msk = 0;
-            const int t1 = min(p.n, 32 * w + 32);
-            for (int t = 32 * w; t < t1; ++t) {
-                const long long zi = (long long)t * p.d_ff + k;
-                const bool s = p.topk ? p.sel[zi] != 0 : p.z[zi] > p.tau;
-                msk |= (s ? 1u : 0u) << (t - 32 * w);
-            }
-            p.lst_mask[(size_t)k * p.mw + w] = msk;
-        }
-    }
-    if (blockIdx.x == 0) {
-        if (threadIdx.x == 0) *p.u_count = total;
-        // 128-channel blocks with a listed channel, in order
-        const int nblk = (p.d_ff + 127) / 128;
-        int prior = 0;
-        for (int b0 = 0; b0 < nblk; b0 += kUnionThreads) {
-            const int bi = b0 + threadIdx.x;
-            bool act = false;
-            if (bi < nblk)
-                for (int w = 4 * bi; w < min(4 * bi + 4, nwords); ++w) act |= union_word(p, w, nwords) != 0;
-            int cnt = 0;
-            const int r = block_exclusive_scan(act ? 1 : 0, &cnt, sh);
-            if (act) p.blk_list[prior + r] = bi;
-            prior += cnt;
-        }
-        if (threadIdx.x == 0) *p.blk_count = prior;
-    }
 }
 
 SmemAttrCache g_tc_smem;
@@ -674,7 +618,8 @@ size_t tc_smem_bytes(int nb, int* stages) {
 cudaError_t launch_tc(const TcParams& p_in, int grid, cudaStream_t s, bool pdl) {
     TcParams p = p_in;
     if (p.nb < 16 || p.nb > 256 || p.nb % 16 || (p.paired && 2 * p.npad != p.nb)) return cudaErrorInvalidValue;
-    if ((p.mode == kTcUp || p.mode == kTcDown) && p.blk_cap > kMaxBlocks) return cudaErrorInvalidValue;
+    if ((p.mode == kTcUp || p.mode == kTcDown) && ((p.d_ff + 127) / 128 > kMaxBlocks || (!p.ubits && !p.force_all)))
+        return cudaErrorInvalidValue;
     int st = 0;
     const size_t smem = tc_smem_bytes(p.nb, &st);
     if (!smem) return cudaErrorInvalidValue;
@@ -686,11 +631,6 @@ cudaError_t launch_tc(const TcParams& p_in, int grid, cudaStream_t s, bool pdl) 
     return launch_ex(k_tc_gemm, dim3(grid), dim3(kTcThreads), smem, s, pdl, p);
 }
 
-cudaError_t launch_union(const UnionParams& p, cudaStream_t s, bool pdl) {
-    if ((p.d_ff + 127) / 128 > kMaxBlocks) return cudaErrorInvalidValue;
-    const int grid = (p.d_ff + kUnionThreads - 1) / kUnionThreads;
-    return launch_ex(k_union, dim3(grid), dim3(kUnionThreads), 0, s, pdl, p);
-}
 
 // 2-D bf16 tensor map (row-major, `cols` contiguous elements per row) with a
 // box of box_cols x box_rows elements and the 128-byte swizzle; elements

@@ -6,8 +6,9 @@
 // order-preserving uint32; a 4-pass MSB-first radix select (8-bit digits,
 // warp-aggregated shared-memory histograms) finds the K-th largest key, then a
 // block-wide prefix sum over channel order takes the ties at that key from the
-// lowest channel index up.  Outputs: sel[t][k] (1 = selected) and
-// gbuf[t][k] = SiLU(z) on selected channels, 0 elsewhere; optionally the
+// lowest channel index up.  The keys are computed once into shared memory.
+// Outputs: sel[t][k] (1 = selected) and gbuf[t][k] = SiLU(z) on selected
+// channels, 0 elsewhere; optionally the
 // selected channels are OR-ed into a union bitmap (bit k of word k/32).
 #include "common.cuh"
 
@@ -21,9 +22,19 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-constexpr int kTopkThreads = 1024;
+// Inverse of order_key (exact, except that -0 comes back as +0).
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
 
+constexpr int kTopkThreads = 1024;
+constexpr size_t kTopkSmemKeys = 200 * 1024;   // keys staged in shared memory up to this many bytes
+
+// SMEM: the token's keys are computed once into shared memory; otherwise every
+// pass recomputes them from z (rows too long for shared memory).
+template <bool SMEM>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
+    extern __shared__ uint32_t skeys[];
     __shared__ unsigned hist[256];
     __shared__ int sh[40];
     __shared__ uint32_t s_prefix;
@@ -34,6 +45,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
 
     griddep_wait();
     griddep_launch_dependents();
+    if (SMEM) {
+        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) skeys[k] = order_key(silu_f(z[k]));
+        __syncthreads();
+    }
+    auto key_at = [&](int k) -> uint32_t { return SMEM ? skeys[k] : order_key(silu_f(z[k])); };
 
     const int K = p.k;
     const bool partial = K > 0 && K < p.d_ff;
@@ -48,7 +64,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
                 const int k = base + lane;
                 uint32_t digit = 0xFFFFFFFFu;
                 if (k < p.d_ff) {
-                    const uint32_t key = order_key(silu_f(z[k]));
+                    const uint32_t key = key_at(k);
                     if ((key & pmask) == prefix) digit = (key >> shift) & 0xFFu;
                 }
                 const unsigned peers = __match_any_sync(0xffffffffu, digit);
@@ -76,16 +92,16 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     const int k0 = threadIdx.x * per, k1 = min(p.d_ff, k0 + per);
     int ties = 0;
     if (partial)
-        for (int k = k0; k < k1; ++k) ties += order_key(silu_f(z[k])) == prefix;
+        for (int k = k0; k < k1; ++k) ties += key_at(k) == prefix;
     int tot = 0;
     int rank = block_exclusive_scan(ties, &tot, sh);
     for (int k = k0; k < k1; ++k) {
-        const float gv = silu_f(z[k]);
+        const uint32_t key = key_at(k);
+        const float gv = SMEM ? key_value(key) : silu_f(z[k]);
         bool s;
         if (!partial) {
             s = K > 0;
         } else {
-            const uint32_t key = order_key(gv);
             if (key == prefix) {
                 s = rank < remaining;
                 ++rank;
@@ -100,7 +116,14 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s, bool pdl) {
-    return launch_ex(k_topk, dim3(p.n), dim3(kTopkThreads), 0, s, pdl, p);
+    const size_t keys = (size_t)p.d_ff * sizeof(uint32_t);
+    if (keys <= kTopkSmemKeys) {
+        static SmemAttrCache cache;
+        cudaError_t e = ensure_smem(k_topk<true>, keys, cache);
+        if (e != cudaSuccess) return e;
+        return launch_ex(k_topk<true>, dim3(p.n), dim3(kTopkThreads), keys, s, pdl, p);
+    }
+    return launch_ex(k_topk<false>, dim3(p.n), dim3(kTopkThreads), 0, s, pdl, p);
 }
 
 }  // namespace sffn
