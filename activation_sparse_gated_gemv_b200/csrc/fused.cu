@@ -333,12 +333,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     }
     __syncthreads();
     const int tot = scan_sh[0];
-    for (int i = threadIdx.x; i < tot; i += kDecThreads) {
-        const int sl = wl[i];
-        p.lst_idx[c0 + i] = c0 + sl;
-        for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + sl) * p.mw + w] = smask[sl * p.mw + w];
-    }
-    if (threadIdx.x == 0) p.seg_count[blockIdx.x] = tot;
 
     // ---- the CTA's share of the down projection: h_k W_down[k, :] over its
     // active channels in list order (whole rows, mostly in L2 by now), as an
@@ -392,10 +386,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     const int G = gridDim.x;
     const int cps = decode_slice_chunks(p.d, V, G);       // 16-byte chunks per column slice
     const int col0 = blockIdx.x * cps * V;
-    __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
+        // release: the CTA's partial (ordered before this thread by the barrier) is visible first
+        __threadfence();
         atomicAdd(p.tickets, 1u);
+    }
+    // the CTA's list, for sffn_get_active only: off the path to the barrier
+    for (int i = threadIdx.x; i < tot; i += kDecThreads) {
+        const int sl = wl[i];
+        p.lst_idx[c0 + i] = c0 + sl;
+        for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + sl) * p.mw + w] = smask[sl * p.mw + w];
+    }
+    if (threadIdx.x == 0) {
+        p.seg_count[blockIdx.x] = tot;
         int ok = 1;
         if (col0 < p.d) {
             const unsigned long long t0 = globaltimer_ns();
