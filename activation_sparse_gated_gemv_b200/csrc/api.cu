@@ -94,7 +94,7 @@ struct sffn_ctx {
     int* status = nullptr;
     void* xdev = nullptr;
     void* ydev = nullptr;
-    // tensor-core batched path (bf16 handles with max_tokens > kDecodeMaxTokens)
+    // tensor-core batched path (bf16 handles with max_tokens > kFusedMaxTokens)
     bool tc = false;
     int tc_npad_max = 0;
     long long tc_ldh = 0;
@@ -308,7 +308,11 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
                                        &dec_smem);
 
     h->last_tc = false;
-    if (h->tc && n > kDecodeMaxTokens && n <= kTcMaxTokens) {
+    // Three or more tokens: the tensor-core path (measured faster than the fused
+    // decode kernel from n = 3 on every shape but one, and the only fast path
+    // where the decode kernel's shared memory does not fit); one or two: the
+    // fused decode kernel.
+    if (h->tc && n > kFusedMaxTokens && n <= kTcMaxTokens) {
         const int rc = run_tc(h, x, n, lopa, sel, out, s, dense, launches);
         if (rc != SFFN_ERR_UNSUPPORTED) return rc;
     }
@@ -479,7 +483,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_tk = take((size_t)(P.down_slices > 2 ? P.down_slices : 2) * 4), o_st = take(4);
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
     // tensor-core path buffers
-    h->tc = c.wdtype == SFFN_BF16 && c.max_tokens > kDecodeMaxTokens;
+    h->tc = c.wdtype == SFFN_BF16 && c.max_tokens > kFusedMaxTokens;
     h->tc_npad_max = (int)round_up(c.max_tokens < kTcMaxTokens ? c.max_tokens : kTcMaxTokens, 16);
     h->tc_ldh = (long long)round_up(F, 128);
     const size_t NP = h->tc ? (size_t)h->tc_npad_max : 0;

@@ -369,7 +369,8 @@ bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int v
                      size_t* smem);
 cudaError_t launch_decode(int wdtype, const DecodeParams& p, int nt, int gate_kind, int grid, size_t smem,
                           cudaStream_t s, bool pdl);
-constexpr int kDecodeMaxTokens = 4;   // the fused decode path takes up to this many tokens
+constexpr int kDecodeMaxTokens = 4;   // the fused decode kernel takes up to this many tokens
+constexpr int kFusedMaxTokens = 2;    // ... and is preferred to the tensor-core path up to this many
 size_t tc_smem_bytes(int nb, int* stages);
 cudaError_t encode_tile_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                             uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);

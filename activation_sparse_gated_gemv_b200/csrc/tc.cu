@@ -586,6 +586,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
         }
     }
     const Problem q = make_problem(p, nblk);
+    if (p.mode == kTcDown && q.KB == 0) {
+        // no channel is active for any token: y = 0
+        bf16* y = static_cast<bf16*>(p.out);
+        const long long total = (long long)p.n * p.m_total;
+        for (long long i = (long long)blockIdx.x * kTcThreads + threadIdx.x; i < total;
+             i += (long long)gridDim.x * kTcThreads) {
+            const long long t = i / p.m_total;
+            y[t * p.ldo + (i - t * p.m_total)] = __float2bfloat16_rn(0.f);
+        }
+    }
 
     if (warp == kProdWarp) {
         if ((threadIdx.x & 31) == 0) run_producer(p, q, stages, stage_bytes, sh);
