@@ -94,7 +94,7 @@ struct sffn_ctx {
     int* status = nullptr;
     void* xdev = nullptr;
     void* ydev = nullptr;
-    // tensor-core batched path (bf16 handles with max_tokens > kFusedMaxTokens)
+    // tensor-core batched path (bf16 handles with max_tokens > 1)
     bool tc = false;
     int tc_npad_max = 0;
     long long tc_ldh = 0;
@@ -309,15 +309,15 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
 
     h->last_tc = false;
     // Three or more tokens: the tensor-core path (measured faster than the fused
-    // decode kernel from n = 3 on every shape but one, and the only fast path
-    // where the decode kernel's shared memory does not fit); one or two: the
-    // fused decode kernel.
-    if (h->tc && n > kFusedMaxTokens && n <= kTcMaxTokens) {
+    // decode kernel from n = 3 on every shape but one); one or two: the fused
+    // decode kernel, or the tensor-core path for two tokens where the decode
+    // kernel's shared memory does not fit.
+    if (h->tc && n <= kTcMaxTokens && (n > kFusedMaxTokens || (n > 1 && !fused))) {
         const int rc = run_tc(h, x, n, lopa, sel, out, s, dense, launches);
         if (rc != SFFN_ERR_UNSUPPORTED) return rc;
     }
 
-    if (lopa) {
+    if (lopa && !fused) {
         LopaUParams lp{};
         lp.x = x; lp.at = h->a; lp.n = n; lp.d = c.d; lp.r = c.lopa_rank; lp.u = h->u;
         SFFN_CUDA(launch_lopa_u(c.wdtype, lp, pick_nt(n), s, pdl), "LoPA x*A launch");
@@ -328,7 +328,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     if (fused) {
         DecodeParams dp{};
         dp.x = x; dp.n = n; dp.d = c.d; dp.d_ff = c.d_ff; dp.r = c.lopa_rank;
-        dp.wg = h->wg; dp.bcm = h->bcm; dp.u = h->u; dp.wup = h->wup; dp.wdn = h->wdn;
+        dp.wg = h->wg; dp.bcm = h->bcm; dp.at = h->a; dp.u = h->u; dp.wup = h->wup; dp.wdn = h->wdn;
         dp.tau = sel->tau; dp.cpb = P.cpb; dp.mw = P.mw;
         dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
         dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.part = h->fpart;
@@ -480,10 +480,10 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_u = take(T * R * 4);
     const size_t o_dp = take((size_t)P.down_chunks * T * D * 4);
     const size_t o_fp = take((size_t)P.g1 * (T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * D * 4);
-    const size_t o_tk = take((size_t)(P.down_slices > 2 ? P.down_slices : 2) * 4), o_st = take(4);
+    const size_t o_tk = take((size_t)(P.down_slices > 4 ? P.down_slices : 4) * 4), o_st = take(4);
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
     // tensor-core path buffers
-    h->tc = c.wdtype == SFFN_BF16 && c.max_tokens > kFusedMaxTokens;
+    h->tc = c.wdtype == SFFN_BF16 && c.max_tokens > 1;
     h->tc_npad_max = (int)round_up(c.max_tokens < kTcMaxTokens ? c.max_tokens : kTcMaxTokens, 16);
     h->tc_ldh = (long long)round_up(F, 128);
     const size_t NP = h->tc ? (size_t)h->tc_npad_max : 0;

@@ -253,7 +253,8 @@ struct DecodeParams {
     int n, d, d_ff, r;
     const void* wg;         // [d_ff][d]   dense gate rows
     const void* bcm;        // [d_ff][r]   LoPA B rows
-    const float* u;         // [n][r]      LoPA x A
+    const void* at;         // [r][d]      LoPA A^T rows (stage 1 inside the kernel)
+    float* u;               // [n][r]      LoPA x A, written and read inside the kernel
     const void* wup;        // [d_ff][d]
     const void* wdn;        // [d_ff][d]
     float tau;
@@ -265,7 +266,7 @@ struct DecodeParams {
     int sb, nb;             // streamed piece bytes, pieces in flight per streaming warp
     int* status;
     float* part;            // [CTAs][n][d] per-CTA partials of y
-    unsigned* tickets;      // [2] grid-barrier counters, zero between forwards
+    unsigned* tickets;      // [3] grid-barrier counters, zero between forwards
     void* y;                // [n][d] T
 };
 

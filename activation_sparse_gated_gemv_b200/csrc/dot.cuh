@@ -50,7 +50,7 @@ __device__ __forceinline__ void chunk_dot(const uint4& w, const float* xrow, int
 // nt..NT-1 are zero.  16-byte loads, all of a thread's loads issued before any
 // store (a handful of round trips at most).  All threads of the block take part.
 template <class WT, class XT, int NT>
-__device__ __forceinline__ void stage_rows(float* dst, const XT* src, int len, int t0, int nt) {
+__device__ __forceinline__ void stage_rows(float* dst, const XT* src, int len, int t0, int nt, bool l2_only = false) {
     constexpr int V = Elem<WT>::kVec;
     constexpr int XV = 16 / sizeof(XT);                 // elements per 16-byte load
     constexpr int U = 4;
@@ -62,9 +62,8 @@ __device__ __forceinline__ void stage_rows(float* dst, const XT* src, int len, i
         for (int u = 0; u < U; ++u) {
             const int i = base + u * blockDim.x;
             const int t = i / per_row;
-            v[u] = (i < total && t < nt)
-                       ? *reinterpret_cast<const uint4*>(src + (size_t)(t0 + t) * len + (size_t)(i - t * per_row) * XV)
-                       : make_uint4(0u, 0u, 0u, 0u);
+            const uint4* q = reinterpret_cast<const uint4*>(src + (size_t)(t0 + t) * len + (size_t)(i - t * per_row) * XV);
+            v[u] = (i < total && t < nt) ? (l2_only ? __ldcg(q) : *q) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {

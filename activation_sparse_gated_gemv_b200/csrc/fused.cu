@@ -6,7 +6,9 @@
 // evaluated first and the two other matrices are touched only for channels
 // whose activation is non-zero.  Here those touches overlap the gate stream:
 //
-// k_decode, one CTA per SM over its channel range [c0, c0 + cpb), 16 warps:
+// k_decode, one CTA per SM over its channel range [c0, c0 + cpb), 16 warps
+// (LoPA: first each CTA computes its rows of u = x A, and a grid barrier
+// publishes u to all CTAs):
 //   * warps 0..13 stream the CTA's gate rows (dense W_gate, or LoPA's B) through
 //     per-warp rings of bulk copies (TMA engine, mbarriers) and leave per-piece
 //     dot products in shared memory.  When a row's last piece is in, the warp
@@ -164,6 +166,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         while (issued < min(p.nb, wcount)) issue_next();
         __syncwarp();
     }
+    // LoPA: this CTA's rows of A^T (stage 1) into L2 as well
+    const int u0 = GATE == kGateLopa ? (int)((long long)p.r * blockIdx.x / gridDim.x) : 0;
+    const int u1 = GATE == kGateLopa ? (int)((long long)p.r * (blockIdx.x + 1) / gridDim.x) : 0;
+    if (GATE == kGateLopa && lane == 0)
+        for (int j = u0 + warp; j < u1; j += kDecWarps)
+            bulk_prefetch_l2(static_cast<const T*>(p.at) + (size_t)j * p.d, (uint32_t)(p.d * sizeof(T)));
 
     griddep_wait();
     griddep_launch_dependents();
@@ -176,12 +184,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     for (int i = threadIdx.x; i < p.cpb * p.mw; i += kDecThreads) smask[i] = 0u;
     if (threadIdx.x < 4) ctr[threadIdx.x] = 0;
     stage_rows<T, T, NT>(xs, static_cast<const T*>(p.x), p.d, 0, n);
-    if (GATE == kGateLopa) stage_rows<T, float, NT>(us, p.u, p.r, 0, n);
     if (streamer) {
         while (issued < min(p.nb, wcount)) issue_next();
         __syncwarp();
     }
     __syncthreads();
+    if (GATE == kGateLopa) {
+        // LoPA stage 1 inside the launch: this CTA's rows of u = x A (one per
+        // warp), published; a grid barrier; then every CTA stages all of u.
+        // The wait is bounded and cannot deadlock: all CTAs are resident.
+        for (int j = u0 + warp; j < u1; j += kDecWarps) {
+            float acc[NT];
+            warp_dot_global<T, NT>(static_cast<const T*>(p.at) + (size_t)j * p.d, p.d / V, xs, p.d, acc);
+            if (lane == 0)
+                for (int t = 0; t < n; ++t) p.u[(size_t)t * p.r + j] = acc[t];
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(p.tickets + 2, 1u);
+            const unsigned long long t0 = globaltimer_ns();
+            unsigned backoff = 32;
+            int ok = 1;
+            while (ld_acquire_u32(p.tickets + 2) < gridDim.x) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                    atomicExch(ctr + kAbort, 1);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(backoff);
+                if (backoff < 256) backoff <<= 1;
+            }
+            scan_sh[3] = ok;
+        }
+        __syncthreads();
+        __threadfence();
+        stage_rows<T, float, NT>(us, p.u, p.r, 0, n, true);
+        __syncthreads();
+    }
 
     // Row s is complete: z from its parts in order, select, queue it.
     auto finalize = [&](int s) {                         // lane 0 only
@@ -467,6 +508,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     if (threadIdx.x == 0 && atomicAdd(p.tickets + 1, 1u) == gridDim.x - 1u) {
         p.tickets[0] = 0u;
         p.tickets[1] = 0u;
+        p.tickets[2] = 0u;                                // the LoPA stage-1 barrier
         __threadfence();
     }
 }

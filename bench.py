@@ -421,9 +421,9 @@ def main():
     dom_name = kernel_names[dominant] if dominant < len(kernel_names) else f"k{dominant}"
     w = bytes_per_elem(wl.dtype)
     if dom_name == "decode_fused":
-        # everything but A, which the separate stage-1 LoPA kernel reads
+        # everything (LoPA's stage 1 runs inside the same launch)
         dom_bytes = algorithmic_bytes(wl, union) - (
-            wl.d * wl.r * bytes_per_elem(wl.dtype) if wl.gate == "lopa" else 0)
+            wl.d * wl.r * bytes_per_elem(wl.dtype) if "lopa_u" in kernel_names else 0)
     elif dom_name == "gate_select_up":
         dom_bytes = algorithmic_bytes(wl, union, gate_kernel_only=True)
     elif dom_name == "down":
