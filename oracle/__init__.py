@@ -41,7 +41,7 @@ _SRC = os.path.join(_HERE, "sffn_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 ODT_BF16, ODT_F32, ODT_F64 = 0, 1, 2
-SEL_THRESHOLD, SEL_TOPK = 0, 1
+SEL_THRESHOLD, SEL_TOPK, SEL_TOPP = 0, 1, 2
 
 _lib = None
 
@@ -69,6 +69,8 @@ def _load():
     lib.oracle_select_threshold.argtypes = [P, L, L, D, P, P, P]
     lib.oracle_select_topk.argtypes = [P, L, L, L, P, P, P]
     lib.oracle_select_topk.restype = I
+    lib.oracle_select_topp.argtypes = [P, L, L, D, P, P, P]
+    lib.oracle_select_topp.restype = I
     lib.oracle_sparse_ffn.argtypes = [P, I, P, P, I, L, L, L, P, P, P, P, P]
     lib.oracle_dense_ffn.argtypes = [P, I, P, P, I, L, L, L, P, P]
     lib.oracle_num_threads.restype = I
@@ -194,13 +196,27 @@ def select_topk(z: np.ndarray, k: int):
     return _lists(idx, cnt), g
 
 
+def select_topp(z: np.ndarray, p: float):
+    """(sets, g): per token the shortest prefix of channels by descending z
+    (ties: lower index) whose softmax mass reaches p, listed ascending;
+    g = SiLU(z) on S_t, else 0."""
+    z = np.ascontiguousarray(z, np.float64)
+    n, d_ff = z.shape
+    idx = np.zeros((n, max(d_ff, 1)), np.int32)
+    cnt = np.zeros(n, np.int32)
+    g = np.empty((n, d_ff), np.float64)
+    if _load().oracle_select_topp(_ptr(z), n, d_ff, float(p), _ptr(idx), _ptr(cnt), _ptr(g)) != 0:
+        raise ValueError(f"bad top-p p={p}")
+    return _lists(idx, cnt), g
+
+
 def gate_values(z: np.ndarray, sets: Sequence[np.ndarray], kind: str, tau: float = 0.0):
     """g = act(z) on the given per-token sets (z - tau or SiLU(z)), 0 elsewhere."""
     z = np.ascontiguousarray(z, np.float64)
     n, d_ff = z.shape
     idx, cnt = _packed(sets, d_ff)
     g = np.empty((n, d_ff), np.float64)
-    code = SEL_THRESHOLD if kind == "threshold" else SEL_TOPK
+    code = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "topp": SEL_TOPP}[kind]
     _load().oracle_gate_values(_ptr(z), n, d_ff, _ptr(idx), _ptr(cnt), code, float(tau), _ptr(g))
     return g
 
@@ -253,13 +269,15 @@ def gate(x, weights: dict, gate_mode: str = "dense"):
 
 
 def forward(x, weights: dict, gate_mode: str, select: str, tau: float = 0.0, k: int = 0,
-            dense: bool = False) -> Result:
+            dense: bool = False, p: float = 0.0) -> Result:
     """The whole path: gate, select, then the sparse (or the dense) FFN."""
     z, u = gate(x, weights, gate_mode)
     if select == "threshold":
         sets, g = select_threshold(z, tau)
-    else:
+    elif select == "topk":
         sets, g = select_topk(z, k)
+    else:
+        sets, g = select_topp(z, p)
     if dense:
         y = dense_ffn(x, weights["w_up"], weights["w_down"], g)
     else:

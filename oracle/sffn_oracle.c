@@ -17,6 +17,10 @@
  *     (a shifted ReLU, the "sparsity inducing activation" of model casting)
  *   top-K select       S_t = the K channels with the largest SiLU(z[t,k]),
  *                      ties to the lower index;  g = SiLU(z) on S_t
+ *   top-p select       S_t = the shortest prefix, by descending z (ties to the
+ *                      lower index), whose softmax mass reaches p;  g = SiLU(z)
+ *     "PrunePath" (abstract: softmax-normalised routing distribution,
+ *     cumulative-mass threshold, token-level probability budget).
  *     "Mixture-of-Channels" (sections "Dentro il mixture", "Dentro MoC": Top-K
  *     channels per token, ranked by the SwiGLU gate).
  *   sparse FFN         y[t,:] = sum over k in S_t, ascending, of
@@ -40,7 +44,7 @@
 #endif
 
 enum { ODT_BF16 = 0, ODT_F32 = 1, ODT_F64 = 2 };
-enum { OSEL_THRESHOLD = 0, OSEL_TOPK = 1 };
+enum { OSEL_THRESHOLD = 0, OSEL_TOPK = 1, OSEL_TOPP = 2 };
 
 /* Exact widening of one stored element to double.  A bf16 value is the upper
  * half of an IEEE binary32, so its bits shifted left by 16 are that binary32. */
@@ -174,6 +178,47 @@ int oracle_select_topk(const double* z, int64_t n, int64_t d_ff, int64_t K,
     }
     free(items);
     oracle_gate_values(z, n, d_ff, idx, cnt, OSEL_TOPK, 0.0, g);
+    return 0;
+}
+
+/* Top-p selection ("PrunePath", abstract: a softmax-normalised routing
+ * distribution and a cumulative-mass threshold, i.e. a per-token probability
+ * budget).  Per token: P_k = exp(z_k - max z) / sum_j exp(z_j - max z); rank
+ * the channels by z (the order of P), ties to the lower index; keep the
+ * shortest prefix whose mass reaches p; list it ascending.  p = 0 keeps none.
+ * Activation SiLU(z) on the kept channels, as for top-K.  Returns -1 on p
+ * outside [0, 1] or an allocation failure. */
+int oracle_select_topp(const double* z, int64_t n, int64_t d_ff, double p,
+                       int32_t* idx, int32_t* cnt, double* g) {
+    if (!(p >= 0.0 && p <= 1.0)) return -1;
+    rank_item* items = (rank_item*)malloc(sizeof(rank_item) * (size_t)(d_ff > 0 ? d_ff : 1));
+    if (!items) return -1;
+    for (int64_t t = 0; t < n; t++) {
+        const double* zt = z + t * d_ff;
+        int32_t c = 0;
+        if (d_ff > 0 && p > 0.0) {
+            double m = zt[0];
+            for (int64_t k = 1; k < d_ff; k++) if (zt[k] > m) m = zt[k];
+            double total = 0.0;
+            for (int64_t k = 0; k < d_ff; k++) total += exp(zt[k] - m);
+            for (int64_t k = 0; k < d_ff; k++) {
+                items[k].key = zt[k];
+                items[k].k = (int32_t)k;
+            }
+            qsort(items, (size_t)d_ff, sizeof(rank_item), by_key_desc);
+            const double target = p * total;
+            double cum = 0.0;
+            for (int64_t q = 0; q < d_ff; q++) {
+                idx[t * d_ff + c++] = items[q].k;
+                cum += exp(items[q].key - m);
+                if (cum >= target) break;
+            }
+            qsort(idx + t * d_ff, (size_t)c, sizeof(int32_t), by_int_asc);
+        }
+        cnt[t] = c;
+    }
+    free(items);
+    oracle_gate_values(z, n, d_ff, idx, cnt, OSEL_TOPP, 0.0, g);
     return 0;
 }
 

@@ -107,6 +107,81 @@ def test_topk_ranks_by_silu_not_by_z():
     assert list(sets[0]) == [1, 2]
 
 
+# top-p ("PrunePath", abstract: a softmax-normalised routing distribution and a
+# cumulative-mass threshold, i.e. a per-token probability budget)
+
+def _softmax_exact(z):
+    m = max(z)
+    w = [math.exp(v - m) for v in z]
+    tot = math.fsum(w)
+    return [v / tot for v in w]
+
+
+@pytest.mark.parametrize("seed,d,d_ff,p", [(7, 4, 9, 0.5), (8, 6, 11, 0.8), (9, 3, 12, 0.3), (10, 5, 10, 0.95)])
+def test_topp_set_by_brute_force(seed, d, d_ff, p):
+    """The kept set is the smallest set of channels whose softmax mass reaches
+    p, and among sets of that size the one of largest mass (found over every
+    subset)."""
+    n = 2
+    w, x = _tiny_weights(d, d_ff, n, seed)
+    res = oracle.forward(x, w, "dense", "topp", p=p)
+    X, WG = _exact(x), _exact(w["w_gate"])
+    for t in range(n):
+        z = [float(sum(X[t][j] * WG[j][k] for j in range(d))) for k in range(d_ff)]
+        P = _softmax_exact(z)
+        best_size, best, best_set = None, None, None
+        for size in range(1, d_ff + 1):
+            for S in itertools.combinations(range(d_ff), size):
+                mass = math.fsum(P[k] for k in S)
+                if mass >= p * (1 - 1e-12) and (best is None or mass > best):
+                    best, best_set = mass, S
+            if best_set is not None:
+                best_size = size
+                break
+        assert tuple(res.sets[t]) == best_set and len(best_set) == best_size
+        for k in range(d_ff):
+            expect = z[k] / (1.0 + math.exp(-z[k])) if k in best_set else 0.0
+            assert res.g[t, k] == pytest.approx(expect, rel=1e-12, abs=1e-300)
+
+
+@pytest.mark.parametrize("d_ff,p", [(10, 0.35), (64, 0.5001), (1000, 0.9004), (37, 0.01)])
+def test_topp_uniform_gate_keeps_ceil_p_dff_lowest(d_ff, p):
+    """Equal gate values: every channel carries 1/d_ff, so exactly ceil(p d_ff)
+    channels are kept, the lowest indices first (ties to the lower index)."""
+    z = np.full((1, d_ff), 0.25)
+    sets, _ = oracle.select_topp(z, p)
+    m = math.ceil(p * d_ff)
+    assert list(sets[0]) == list(range(m))
+
+
+def test_topp_extremes_and_monotone():
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((3, 200))
+    for t in range(3):
+        top = int(np.argmax(z[t]))
+        assert list(oracle.select_topp(z[t:t + 1], 1e-9)[0][0]) == [top]      # tiny budget: the arg max
+    assert all(len(s) == 0 for s in oracle.select_topp(z, 0.0)[0])             # no budget: nothing
+    assert all(len(s) == 200 for s in oracle.select_topp(z, 1.0)[0])           # the whole mass: all
+    prev = [set() for _ in range(3)]
+    for p in (0.1, 0.3, 0.5, 0.7, 0.9, 0.99):                                   # nested as p grows
+        sets, _ = oracle.select_topp(z, p)
+        for t in range(3):
+            cur = set(sets[t].tolist())
+            assert prev[t] <= cur
+            prev[t] = cur
+
+
+def test_topp_equals_topk_by_z_of_the_same_size():
+    """For positive gate values SiLU orders like z, so the kept set is the
+    top-K set of the same size."""
+    rng = np.random.default_rng(4)
+    z = np.abs(rng.standard_normal((2, 300))) + 0.1
+    sets, _ = oracle.select_topp(z, 0.6)
+    for t in range(2):
+        ks, _ = oracle.select_topk(z[t:t + 1], len(sets[t]))
+        assert list(ks[0]) == list(sets[t])
+
+
 # --------------------------------------------------------------------------
 # special cases against an independent numpy product chain
 
