@@ -8,10 +8,11 @@ library's CUDA kernels.  PyTorch is used for device memory and streams only.
     y = W_down^T ( act(x W_gate) (*) (x W_up) )
 
 with the gate evaluated first (dense, or LoPA's rank-r ``A B``), channels
-selected by a threshold (``z > tau``, act = ``z - tau``) or per-token top-K of
-``SiLU(z)``, and only the active channels' ``W_up``/``W_down`` rows read
-("Model Casting and Low-Parameter Gating", abstract; "Mixture-of-Channels",
-sections "Dentro il mixture" and "Dentro MoC").
+selected by a threshold (``z > tau``, act = ``z - tau``), per-token top-K of
+``SiLU(z)``, or per-token top-p of the softmax mass of z, and only the active
+channels' ``W_up``/``W_down`` rows read ("Model Casting and Low-Parameter
+Gating", abstract; "Mixture-of-Channels", sections "Dentro il mixture" and
+"Dentro MoC"; "PrunePath", abstract).
 
 There is no fallback: importing this package fails if ``libsffn.so`` is
 missing, and every call that needs a GPU fails if there is none.
@@ -38,7 +39,7 @@ SFFN_ERR_DEVICE_CHECK = 7
 
 SFFN_BF16, SFFN_F32 = 0, 1
 SFFN_GATE_DENSE, SFFN_GATE_LOPA = 0, 1
-SFFN_SELECT_THRESHOLD, SFFN_SELECT_TOPK = 0, 1
+SFFN_SELECT_THRESHOLD, SFFN_SELECT_TOPK, SFFN_SELECT_TOPP = 0, 1, 2
 
 
 class sffn_config(ctypes.Structure):
@@ -47,7 +48,7 @@ class sffn_config(ctypes.Structure):
 
 
 class sffn_select(ctypes.Structure):
-    _fields_ = [("kind", ctypes.c_int32), ("tau", ctypes.c_float), ("k", ctypes.c_int32)]
+    _fields_ = [("kind", ctypes.c_int32), ("tau", ctypes.c_float), ("k", ctypes.c_int32), ("p", ctypes.c_float)]
 
 
 if not os.path.exists(LIB_PATH):
@@ -121,9 +122,9 @@ def _stream_ptr(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def make_select(select: str = "threshold", tau: float = 0.0, k: int = 0) -> sffn_select:
-    kind = {"threshold": SFFN_SELECT_THRESHOLD, "topk": SFFN_SELECT_TOPK}[select]
-    return sffn_select(kind, float(tau), int(k))
+def make_select(select: str = "threshold", tau: float = 0.0, k: int = 0, p: float = 0.0) -> sffn_select:
+    kind = {"threshold": SFFN_SELECT_THRESHOLD, "topk": SFFN_SELECT_TOPK, "topp": SFFN_SELECT_TOPP}[select]
+    return sffn_select(kind, float(tau), int(k), float(p))
 
 
 def gate_code(gate: str) -> int:
@@ -171,26 +172,26 @@ class SparseFFN:
                                _stream_ptr(stream) if on_dev else None), "sffn_set_weights")
 
     def forward(self, x, gate: str = "dense", select: str = "threshold", tau: float = 0.0, k: int = 0,
-                out=None, stream=None, dense: bool = False):
+                out=None, stream=None, dense: bool = False, p: float = 0.0):
         """y for device tokens x (n x d); asynchronous on the stream."""
         torch = _torch()
         n = x.shape[0]
         if out is None:
             out = torch.empty((n, self.d), dtype=x.dtype, device=x.device)
-        sel = make_select(select, tau, k)
+        sel = make_select(select, tau, k, p)
         fn = sffn_forward_dense if dense else sffn_forward
         check(fn(self._h, x.data_ptr(), n, gate_code(gate), ctypes.byref(sel), out.data_ptr(),
                  _stream_ptr(stream)), "sffn_forward_dense" if dense else "sffn_forward")
         return out
 
     def forward_host(self, x, gate: str = "dense", select: str = "threshold", tau: float = 0.0, k: int = 0,
-                     out=None, stream=None):
+                     out=None, stream=None, p: float = 0.0):
         """y for host tokens x (n x d, CPU tensor; pinned for async copies); synchronous."""
         torch = _torch()
         n = x.shape[0]
         if out is None:
             out = torch.empty((n, self.d), dtype=x.dtype, pin_memory=x.is_pinned())
-        sel = make_select(select, tau, k)
+        sel = make_select(select, tau, k, p)
         check(sffn_forward_host(self._h, x.data_ptr(), n, gate_code(gate), ctypes.byref(sel),
                                 out.data_ptr(), _stream_ptr(stream)), "sffn_forward_host")
         return out

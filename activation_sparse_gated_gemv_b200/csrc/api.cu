@@ -167,6 +167,9 @@ int check_select(const sffn_ctx* h, const sffn_select* sel) {
     } else if (sel->kind == SFFN_SELECT_TOPK) {
         if (sel->k < 0 || sel->k > h->cfg.d_ff)
             return fail(SFFN_ERR_INVALID_ARG, "top-K k=%d outside [0, d_ff=%d]", sel->k, h->cfg.d_ff);
+    } else if (sel->kind == SFFN_SELECT_TOPP) {
+        if (!(sel->p >= 0.f && sel->p <= 1.f))
+            return fail(SFFN_ERR_INVALID_ARG, "top-p p=%g outside [0, 1]", (double)sel->p);
     } else {
         return fail(SFFN_ERR_INVALID_ARG, "unknown select kind %d", sel->kind);
     }
@@ -203,7 +206,7 @@ int check_forward(const sffn_ctx* h, const void* x, int n, int gate_mode, const 
 int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel, void* out, cudaStream_t s,
            bool dense, int& launches) {
     const sffn_config& c = h->cfg;
-    const bool topk = sel->kind == SFFN_SELECT_TOPK;
+    const bool topk = sel->kind != SFFN_SELECT_THRESHOLD;   // a top-K or top-p mask decides
     const int npad = (int)round_up(n, 16);
     const float tau = topk ? 0.f : sel->tau;
     if (!h->maps_ok || (lopa && c.lopa_rank < 64)) return SFFN_ERR_UNSUPPORTED;
@@ -252,8 +255,10 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
         TopkParams tp{};
         tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
         tp.ubits = h->ubits;
-        SFFN_CUDA(launch_topk(tp, s, true), "top-K launch");
-        h->last_names[launches] = "topk";
+        tp.mode = sel->kind == SFFN_SELECT_TOPP ? 1 : 0;
+        tp.p = sel->p;
+        SFFN_CUDA(launch_topk(tp, s, true), "top-K / top-p launch");
+        h->last_names[launches] = tp.mode ? "topp" : "topk";
         record(h, ++launches, s);
     }
 
@@ -368,8 +373,10 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         record(h, ++launches, s);
         TopkParams tp{};
         tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
-        SFFN_CUDA(launch_topk(tp, s, pdl), "top-K launch");
-        h->last_names[launches] = "topk";
+        tp.mode = sel->kind == SFFN_SELECT_TOPP ? 1 : 0;
+        tp.p = sel->p;
+        SFFN_CUDA(launch_topk(tp, s, pdl), "top-K / top-p launch");
+        h->last_names[launches] = tp.mode ? "topp" : "topk";
         record(h, ++launches, s);
         gp.out = kOutSelectUp;
         const int nt = presel_nt(h, n);

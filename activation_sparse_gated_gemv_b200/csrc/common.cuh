@@ -232,6 +232,8 @@ struct TopkParams {
     float* gbuf;            // [n][d_ff]
     uint8_t* sel;           // [n][d_ff]
     uint32_t* ubits;        // [d_ff/32] union bitmap, OR-ed into (NULL: none)
+    int mode;               // 0: top-K (k channels), 1: top-p (softmax mass p)
+    float p;
 };
 
 struct DownParams {

@@ -1,6 +1,8 @@
 // Per-token top-K channel selection ("Mixture-of-Channels", sections "Dentro il
 // mixture" and "Dentro MoC": per token only the K channels ranked highest by the
-// SwiGLU gate stay active, as a binary mask with no threshold heuristics).
+// SwiGLU gate stay active, as a binary mask with no threshold heuristics), and
+// per-token top-p selection ("PrunePath", abstract: a softmax-normalised
+// routing distribution with a cumulative-mass threshold).
 //
 // One CTA per token.  The key of channel k is SiLU(z[t,k]) mapped to an
 // order-preserving uint32; a 4-pass MSB-first radix select (8-bit digits,
@@ -30,8 +32,20 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 constexpr int kTopkThreads = 1024;
 constexpr size_t kTopkSmemKeys = 200 * 1024;   // keys staged in shared memory up to this many bytes
 
+// Fixed-point scale 2^S of the top-p masses: a token's total stays below 2^31.
+__host__ __device__ inline int topp_scale_bits(int d_ff) {
+    int s = 0;
+    while (s < 24 && ((long long)d_ff << (s + 1)) < (1ll << 31)) ++s;
+    return s;
+}
+
 // SMEM: the token's keys are computed once into shared memory; otherwise every
 // pass recomputes them from z (rows too long for shared memory).
+// Top-K (p.mode 0): key = order of SiLU(z); each channel counts 1; keep K.
+// Top-p (p.mode 1): key = order of z; each channel weighs
+//   m_k = round(exp(z_k - max z) 2^S) (integer, so sums are exact and the
+//   choice reproducible); keep the shortest prefix by descending key whose
+//   mass reaches ceil(p sum_k m_k).
 template <bool SMEM>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     extern __shared__ uint32_t skeys[];
@@ -39,22 +53,65 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     __shared__ int sh[40];
     __shared__ uint32_t s_prefix;
     __shared__ int s_remaining;
+    __shared__ unsigned s_red[33];
     const int lane = threadIdx.x & 31;
     const size_t row = (size_t)blockIdx.x * p.d_ff;
     const float* z = p.zbuf + row;
+    const bool topp = p.mode == 1;
 
     griddep_wait();
     griddep_launch_dependents();
+    auto make_key = [&](int k) -> uint32_t { return order_key(topp ? z[k] : silu_f(z[k])); };
     if (SMEM) {
-        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) skeys[k] = order_key(silu_f(z[k]));
+        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) skeys[k] = make_key(k);
         __syncthreads();
     }
-    auto key_at = [&](int k) -> uint32_t { return SMEM ? skeys[k] : order_key(silu_f(z[k])); };
+    auto key_at = [&](int k) -> uint32_t { return SMEM ? skeys[k] : make_key(k); };
 
-    const int K = p.k;
-    const bool partial = K > 0 && K < p.d_ff;
+    // top-p: the largest gate value, the masses and their total
+    float zmax = 0.f, scale = 0.f;
+    if (topp) {
+        uint32_t mk = 0u;
+        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) mk = max(mk, key_at(k));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) mk = max(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+        if (lane == 0) s_red[threadIdx.x >> 5] = mk;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            uint32_t v = s_red[threadIdx.x];
+#pragma unroll
+            for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (threadIdx.x == 0) s_red[32] = v;
+        }
+        __syncthreads();
+        zmax = key_value(s_red[32]);
+        scale = (float)(1 << topp_scale_bits(p.d_ff));
+        __syncthreads();
+    }
+    auto mass_of = [&](uint32_t key) -> unsigned { return __float2uint_rn(expf(key_value(key) - zmax) * scale); };
+
+    int target = p.k;                                     // top-K: channels; top-p: mass
+    if (topp) {
+        unsigned tm = 0u;
+        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) tm += mass_of(key_at(k));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) tm += __shfl_xor_sync(0xffffffffu, tm, o);
+        if (lane == 0) s_red[threadIdx.x >> 5] = tm;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            unsigned v = s_red[threadIdx.x];
+#pragma unroll
+            for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (threadIdx.x == 0) s_red[32] = v;
+        }
+        __syncthreads();
+        const unsigned total = s_red[32];
+        target = (int)min((double)total, ceil((double)p.p * (double)total));
+        __syncthreads();
+    }
+    const bool partial = topp ? target > 0 : (target > 0 && target < p.d_ff);
     uint32_t prefix = 0u, pmask = 0u;
-    int remaining = K;
+    int remaining = target;
     if (partial) {
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass;
@@ -63,19 +120,24 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
             for (int base = (threadIdx.x & ~31); base < p.d_ff; base += kTopkThreads) {
                 const int k = base + lane;
                 uint32_t digit = 0xFFFFFFFFu;
+                unsigned w = 0u;
                 if (k < p.d_ff) {
                     const uint32_t key = key_at(k);
-                    if ((key & pmask) == prefix) digit = (key >> shift) & 0xFFu;
+                    if ((key & pmask) == prefix) {
+                        digit = (key >> shift) & 0xFFu;
+                        w = topp ? mass_of(key) : 1u;
+                    }
                 }
                 const unsigned peers = __match_any_sync(0xffffffffu, digit);
-                if (digit != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+                const unsigned sum = __reduce_add_sync(peers, w);
+                if (digit != 0xFFFFFFFFu && lane == __ffs(peers) - 1 && sum) atomicAdd(&hist[digit], sum);
             }
             __syncthreads();
-            // thread i < 256 takes bin 255 - i; `before` = candidates in higher bins
+            // thread i < 256 takes bin 255 - i; `before` = weight in higher bins
             const int c = threadIdx.x < 256 ? (int)hist[255 - threadIdx.x] : 0;
             int tot = 0;
             const int before = block_exclusive_scan(c, &tot, sh);
-            if (threadIdx.x < 256 && before < remaining && before + c >= remaining) {
+            if (threadIdx.x < 256 && c > 0 && before < remaining && before + c >= remaining) {
                 s_prefix = prefix | ((uint32_t)(255 - threadIdx.x) << shift);
                 s_remaining = remaining - before;
             }
@@ -86,8 +148,14 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
             __syncthreads();
         }
     }
-    // Keys above `prefix` are all selected; `remaining` keys equal to it are
-    // taken in ascending channel order.
+    // Keys above `prefix` are all selected; of the keys equal to it, taken in
+    // ascending channel order: `remaining` (top-K) or enough to cover the
+    // remaining mass (top-p: equal keys weigh the same).
+    int take = remaining;
+    if (topp && partial) {
+        const unsigned m_tie = mass_of(prefix);
+        take = m_tie ? (int)((remaining + m_tie - 1) / m_tie) : 0;
+    }
     const int per = (p.d_ff + kTopkThreads - 1) / kTopkThreads;
     const int k0 = threadIdx.x * per, k1 = min(p.d_ff, k0 + per);
     int ties = 0;
@@ -97,13 +165,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     int rank = block_exclusive_scan(ties, &tot, sh);
     for (int k = k0; k < k1; ++k) {
         const uint32_t key = key_at(k);
-        const float gv = SMEM ? key_value(key) : silu_f(z[k]);
+        const float gv = topp ? silu_f(key_value(key)) : (SMEM ? key_value(key) : silu_f(z[k]));
         bool s;
         if (!partial) {
-            s = K > 0;
+            s = !topp && target > 0;
         } else {
             if (key == prefix) {
-                s = rank < remaining;
+                s = rank < take;
                 ++rank;
             } else {
                 s = key > prefix;

@@ -57,6 +57,8 @@ def parse():
                     choices=["llama7b-decode", "lopa7b", "moc-topk", "llama70b", "llama70b-lopa", "tiny"])
     ap.add_argument("--sparsity", type=float, default=0.9)
     ap.add_argument("--tokens", type=int, default=0, help="batch size (0: the workload's)")
+    ap.add_argument("--top-p", type=float, default=0.0,
+                    help="select by top-p with this softmax-mass budget instead of the workload's rule")
     ap.add_argument("--graph-steps", type=int, default=256, help="steps per captured graph")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
@@ -81,6 +83,8 @@ def make_workload(a) -> workloads.Workload:
         wl = workloads.tiny()
     if a.tokens:
         wl.n = a.tokens
+    if a.top_p:
+        wl.select, wl.p = "topp", a.top_p
     return wl
 
 
@@ -106,6 +110,8 @@ def dense_bytes(wl):
 def select_args(wl):
     if wl.select == "threshold":
         return dict(select="threshold", tau=wl.tau)
+    if wl.select == "topp":
+        return dict(select="topp", p=wl.p)
     return dict(select="topk", k=wl.k)
 
 
@@ -246,7 +252,7 @@ def cpu_oracle_run(wl, weights, budget_s: float, max_tokens: int = 4096):
     while t_total < budget_s and done < max_tokens:
         x = wl.x(tag=f"cpu{tag}")
         t0 = time.perf_counter()
-        oracle.forward(x, weights, wl.gate, wl.select, tau=wl.tau or 0.0, k=wl.k)
+        oracle.forward(x, weights, wl.gate, wl.select, tau=wl.tau or 0.0, k=wl.k, p=wl.p)
         t_total += time.perf_counter() - t0
         done += x.shape[0]
         tag += 1
@@ -269,11 +275,11 @@ def run_reference(a, world, rank):
     # each step is a bounded sample of the workload: one batch of tokens
     steps = min(steps, max(1, int(budget / 0.05)))
     for i in range(a.warmup and 1 or 0):
-        oracle.forward(wl.x(tag="refw"), weights, wl.gate, wl.select, tau=wl.tau or 0.0, k=wl.k)
+        oracle.forward(wl.x(tag="refw"), weights, wl.gate, wl.select, tau=wl.tau or 0.0, k=wl.k, p=wl.p)
     for i in range(steps):
         x = wl.x(tag=f"ref{i}")
         t0 = time.perf_counter()
-        oracle.forward(x, weights, wl.gate, wl.select, tau=wl.tau or 0.0, k=wl.k)
+        oracle.forward(x, weights, wl.gate, wl.select, tau=wl.tau or 0.0, k=wl.k, p=wl.p)
         per_step.append(time.perf_counter() - t0)
         if time.perf_counter() - t_all0 > budget:
             break
@@ -438,6 +444,8 @@ def main():
         dom_bytes = union * wl.d * w + wl.n * wl.d * w
     elif dom_name == "tc_down":
         dom_bytes = union * wl.d * w + wl.n * wl.d * w
+    elif dom_name in ("topk", "topp"):
+        dom_bytes = wl.n * wl.d_ff * 4                     # z read (the masks written are overhead)
     elif dom_name == "tc_lopa_u":
         dom_bytes = wl.d * wl.r * w + wl.n * wl.d * w
     else:

@@ -51,7 +51,7 @@ typedef enum {
 
 typedef enum { SFFN_BF16 = 0, SFFN_F32 = 1 } sffn_dtype;
 typedef enum { SFFN_GATE_DENSE = 0, SFFN_GATE_LOPA = 1 } sffn_gate_mode;
-typedef enum { SFFN_SELECT_THRESHOLD = 0, SFFN_SELECT_TOPK = 1 } sffn_select_kind;
+typedef enum { SFFN_SELECT_THRESHOLD = 0, SFFN_SELECT_TOPK = 1, SFFN_SELECT_TOPP = 2 } sffn_select_kind;
 
 /* Model shape.  d and lopa_rank must be multiples of 8 (16-byte weight rows);
  * lopa_rank = 0 means no LoPA gate; 1 <= max_tokens <= 1024; wdtype is the
@@ -69,11 +69,19 @@ typedef struct {
 /* Channel selection.  THRESHOLD: active iff z > tau, activation z - tau (a
  * shifted ReLU); tau = +inf selects nothing, NaN or -inf is rejected.
  * TOPK: per token the k channels with the largest SiLU(z) (ties to the lower
- * channel index), activation SiLU(z); 0 <= k <= d_ff. */
+ * channel index), activation SiLU(z); 0 <= k <= d_ff.
+ * TOPP ("PrunePath", abstract: a softmax-normalised routing distribution with
+ * a cumulative-mass threshold): per token the shortest run of channels by
+ * descending z (ties to the lower index) whose softmax mass reaches p,
+ * activation SiLU(z); 0 <= p <= 1 (0 selects nothing).  The masses are summed
+ * as integers, exp(z - max z) in units of 2^-S with d_ff 2^S < 2^30, so the
+ * choice is reproducible; it can differ from the exact one only where the
+ * cumulative mass lies within that rounding of the budget. */
 typedef struct {
     int32_t kind;        /* sffn_select_kind */
-    float tau;
-    int32_t k;
+    float tau;           /* THRESHOLD */
+    int32_t k;           /* TOPK */
+    float p;             /* TOPP */
 } sffn_select;
 
 /* Allocate a handle and its device workspace, sized for cfg->max_tokens.

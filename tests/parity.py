@@ -2,7 +2,9 @@
 
 * Active sets: identical per token, except channels whose oracle gate value
   lies within EXEMPT of the decision boundary (tau for threshold, the K-th
-  largest SiLU value for top-K), where fp32 and fp64 rounding may disagree.
+  largest SiLU value for top-K), where fp32 and fp64 rounding may disagree;
+  for top-p, channels whose cumulative softmax mass lies within EXEMPT of the
+  budget (the kernel sums the masses in fixed point).
 * Outputs: per token, max |y_gpu - y_ref| <= YTOL * max |y_ref| with y_ref the
   oracle evaluated on the GPU's own sets (and, for threshold, on its own sets
   too: the activation z - tau is continuous at the boundary).  A token whose
@@ -25,7 +27,24 @@ def to_np(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def assert_sets(gpu_sets, ref, select, tau=0.0, k=0, tokens=None):
+def topp_exempt(z, p, tol=EXEMPT):
+    """Channels the top-p decision may flip: where the oracle's cumulative
+    softmax mass (descending z, ties to the lower index) before or after the
+    channel lies within tol of the budget p, or whose z is within EXEMPT of
+    the boundary channel's."""
+    z = np.asarray(z, np.float64)
+    order = np.lexsort((np.arange(z.size), -z))
+    w = np.exp(z[order] - z.max())
+    total = w.sum()
+    cum_after = np.cumsum(w) / total
+    cum_before = cum_after - w / total
+    near = (np.abs(cum_before - p) <= tol) | (np.abs(cum_after - p) <= tol)
+    q = int(np.searchsorted(cum_after, p * (1 - 1e-12)))
+    zb = z[order[min(q, z.size - 1)]]
+    return set(order[near].tolist()) | set(np.nonzero(np.abs(z - zb) <= EXEMPT)[0].tolist())
+
+
+def assert_sets(gpu_sets, ref, select, tau=0.0, k=0, tokens=None, p=0.0):
     tokens = range(len(gpu_sets)) if tokens is None else tokens
     for i, t in enumerate(tokens):
         gs = np.asarray(gpu_sets[i])
@@ -35,6 +54,9 @@ def assert_sets(gpu_sets, ref, select, tau=0.0, k=0, tokens=None):
         z = ref.z[i]
         if select == "threshold":
             bad = [c for c in diff if abs(z[c] - tau) > EXEMPT]
+        elif select == "topp":
+            ex = topp_exempt(z, p) if diff else set()
+            bad = [c for c in diff if c not in ex]
         else:
             assert len(gs) == k, f"token {t}: {len(gs)} selected, expected {k}"
             s = silu(z)
@@ -57,19 +79,19 @@ def assert_y(y_gpu, y_ref, tol=YTOL, what=""):
             assert err <= tol * m, f"{what} token {t}: max err {err:.3e} > {tol} * {m:.3e}"
 
 
-def check_forward(ffn, w, x_cpu, gate, select, tau=0.0, k=0, dense=False, tokens=None, tol=YTOL):
+def check_forward(ffn, w, x_cpu, gate, select, tau=0.0, k=0, dense=False, tokens=None, tol=YTOL, p=0.0):
     """Run the CUDA path on all of x, compare the tokens listed (default all)
     with the oracle; returns (y_gpu, gpu_sets, union)."""
     x_dev = x_cpu.cuda()
-    y = ffn.forward(x_dev, gate=gate, select=select, tau=tau, k=k, dense=dense)
+    y = ffn.forward(x_dev, gate=gate, select=select, tau=tau, k=k, dense=dense, p=p)
     torch.cuda.synchronize()
     ffn.check_status()
     sets, union = ffn.active(x_cpu.shape[0])
     tok = list(range(x_cpu.shape[0])) if tokens is None else list(tokens)
     xs = x_cpu[tok]
-    ref = oracle.forward(xs, w, gate, select, tau=tau, k=k)
+    ref = oracle.forward(xs, w, gate, select, tau=tau, k=k, p=p)
     gsets = [sets[t] for t in tok]
-    assert_sets(gsets, ref, select, tau, k, tokens=tok)
+    assert_sets(gsets, ref, select, tau, k, tokens=tok, p=p)
     yg = to_np(y)[tok]
     y_on_gpu_sets = oracle.forward_on_sets(xs, w, gate, select, gsets, tau=tau)
     assert_y(yg, y_on_gpu_sets, tol, "vs oracle on the GPU's sets")

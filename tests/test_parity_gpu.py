@@ -138,6 +138,12 @@ SMALL = [
     (264, 1000, 32, 128, "bf16", "lopa", "topk"),
     (64, 300, 8, 6, "bf16", "lopa", "topk"),
     (1024, 640, 0, 100, "bf16", "dense", "threshold"),
+    # top-p: the batched path and the one-token path, dense and LoPA gates
+    (264, 1000, 0, 16, "bf16", "dense", "topp"),
+    (136, 4100, 0, 1, "bf16", "dense", "topp"),
+    (520, 3000, 64, 33, "bf16", "lopa", "topp"),
+    (512, 3000, 0, 9, "f32", "dense", "topp"),
+    (64, 1000, 8, 2, "bf16", "lopa", "topp"),
 ]
 
 
@@ -150,7 +156,7 @@ def test_small_ragged(sffn, d, d_ff, r, n, dtype, gate, select):
     tau = workloads.tau_for_sparsity(0.85)
     k = max(1, d_ff // 8)
     tokens = None if n <= 32 else [0, 1, n // 2, n - 1]
-    check_forward(ffn, w, x, gate, select, tau=tau, k=k, tokens=tokens)
+    check_forward(ffn, w, x, gate, select, tau=tau, k=k, tokens=tokens, p=0.7)
     ffn.close()
 
 
@@ -189,6 +195,30 @@ def test_tau_inf_and_k_zero_give_zero(sffn):
         assert union == 0 and all(len(s) == 0 for s in sets)
         y = ffn.forward(x.cuda(), gate=gate, select="topk", k=0)
         assert not to_np(y).any()
+    ffn.close()
+
+
+@pytest.mark.parametrize("n", [1, 6])
+def test_topp_extremes(sffn, n):
+    """p = 0 keeps nothing (y = 0); p = 1 keeps every channel with mass (the
+    dense SwiGLU FFN); a tiny p keeps each token's largest gate value."""
+    ffn, w, x = _small(sffn, n=n, d_ff=300)
+    y = ffn.forward(x.cuda(), gate="dense", select="topp", p=0.0)
+    assert not to_np(y).any()
+    sets, union = ffn.active(n)
+    assert union == 0
+    check_forward(ffn, w, x, "dense", "topp", p=1.0)
+    _, sets, _ = check_forward(ffn, w, x, "dense", "topp", p=1e-6)
+    z = oracle.forward(x, w, "dense", "topp", p=1e-6).z
+    assert [list(s) for s in sets] == [[int(np.argmax(z[t]))] for t in range(n)]
+    ffn.close()
+
+
+@pytest.mark.parametrize("p", [0.3, 0.9])
+def test_moc_shape_topp(sffn, p):
+    wl = workloads.moc_topk()
+    ffn, w = _ffn(sffn, wl)
+    check_forward(ffn, w, wl.x(), "dense", "topp", p=p)
     ffn.close()
 
 

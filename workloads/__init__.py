@@ -93,11 +93,12 @@ class Workload:
     n: int
     dtype: str
     gate: str                 # "dense" or "lopa"
-    select: str               # "threshold" or "topk"
+    select: str               # "threshold", "topk" or "topp"
     r: int = 0
     sparsity: Optional[float] = None
     tau: Optional[float] = None
     k: int = 0
+    p: float = 0.0            # top-p budget
     seed: int = 0
     extra: dict = field(default_factory=dict)
 
@@ -112,7 +113,8 @@ class Workload:
         return tokens(self.n if n is None else n, self.d, self.dtype, self.seed, tag)
 
     def describe(self) -> str:
-        sel = f"tau={self.tau:.5f}" if self.select == "threshold" else f"top-k k={self.k}"
+        sel = (f"tau={self.tau:.5f}" if self.select == "threshold" else
+               f"top-p p={self.p:g}" if self.select == "topp" else f"top-k k={self.k}")
         sp = f" sparsity={self.sparsity:g}" if self.sparsity is not None else ""
         rr = f" r={self.r}" if self.gate == "lopa" else ""
         return (f"{self.name}: d={self.d} d_ff={self.d_ff} n={self.n} {self.dtype} "
