@@ -6,7 +6,7 @@
 //
 // One CTA per token.  The key of channel k is SiLU(z[t,k]) mapped to an
 // order-preserving uint32; a 4-pass MSB-first radix select (8-bit digits,
-// warp-aggregated shared-memory histograms) finds the K-th largest key, then a
+// per-warp shared-memory histograms) finds the K-th largest key, then a
 // block-wide prefix sum over channel order takes the ties at that key from the
 // lowest channel index up.  The keys are computed once into shared memory.
 // Outputs: sel[t][k] (1 = selected) and gbuf[t][k] = SiLU(z) on selected
@@ -30,7 +30,7 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 }
 
 constexpr int kTopkThreads = 1024;
-constexpr size_t kTopkSmemKeys = 200 * 1024;   // keys staged in shared memory up to this many bytes
+constexpr size_t kTopkSmemKeys = 180 * 1024;   // keys staged in shared memory up to this many bytes
 
 // Fixed-point scale 2^S of the top-p masses: a token's total stays below 2^31.
 __host__ __device__ inline int topp_scale_bits(int d_ff) {
@@ -48,7 +48,9 @@ __host__ __device__ inline int topp_scale_bits(int d_ff) {
 //   mass reaches ceil(p sum_k m_k).
 template <bool SMEM>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
-    extern __shared__ uint32_t skeys[];
+    extern __shared__ uint32_t dyn[];
+    unsigned* whist = dyn;                                // [32 warps][256 bins]
+    uint32_t* skeys = dyn + 32 * 256;                     // [d_ff] (SMEM)
     __shared__ unsigned hist[256];
     __shared__ int sh[40];
     __shared__ uint32_t s_prefix;
@@ -113,24 +115,22 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     uint32_t prefix = 0u, pmask = 0u;
     int remaining = target;
     if (partial) {
+        unsigned* mine = whist + (threadIdx.x >> 5) * 256;
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass;
-            if (threadIdx.x < 256) hist[threadIdx.x] = 0u;
+            for (int i = threadIdx.x; i < 32 * 256; i += kTopkThreads) whist[i] = 0u;
             __syncthreads();
-            for (int base = (threadIdx.x & ~31); base < p.d_ff; base += kTopkThreads) {
-                const int k = base + lane;
-                uint32_t digit = 0xFFFFFFFFu;
-                unsigned w = 0u;
-                if (k < p.d_ff) {
-                    const uint32_t key = key_at(k);
-                    if ((key & pmask) == prefix) {
-                        digit = (key >> shift) & 0xFFu;
-                        w = topp ? mass_of(key) : 1u;
-                    }
-                }
-                const unsigned peers = __match_any_sync(0xffffffffu, digit);
-                const unsigned sum = __reduce_add_sync(peers, w);
-                if (digit != 0xFFFFFFFFu && lane == __ffs(peers) - 1 && sum) atomicAdd(&hist[digit], sum);
+            // per-warp histograms (integer weights: the sums are exact in any order)
+            for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) {
+                const uint32_t key = key_at(k);
+                if ((key & pmask) == prefix) atomicAdd(&mine[(key >> shift) & 0xFFu], topp ? mass_of(key) : 1u);
+            }
+            __syncthreads();
+            if (threadIdx.x < 256) {
+                unsigned h = 0u;
+#pragma unroll 8
+                for (int w = 0; w < 32; ++w) h += whist[w * 256 + threadIdx.x];
+                hist[threadIdx.x] = h;
             }
             __syncthreads();
             // thread i < 256 takes bin 255 - i; `before` = weight in higher bins
@@ -156,11 +156,31 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
         const unsigned m_tie = mass_of(prefix);
         take = m_tie ? (int)((remaining + m_tie - 1) / m_tie) : 0;
     }
+    // Channels tied at the boundary key: when all of them are kept (the usual
+    // case) the choice needs no ranks and the writes stream in channel order.
+    int nties = 0;
+    if (partial) {
+        int c = 0;
+        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) c += key_at(k) == prefix;
+        int tot0 = 0;
+        block_exclusive_scan(c, &tot0, sh);
+        nties = tot0;
+    }
+    if (!partial || nties <= take) {
+        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) {
+            const uint32_t key = key_at(k);
+            const float gv = topp ? silu_f(key_value(key)) : (SMEM ? key_value(key) : silu_f(z[k]));
+            const bool s = partial ? key >= prefix : (!topp && target > 0);
+            p.sel[row + k] = s ? 1 : 0;
+            p.gbuf[row + k] = s ? gv : 0.f;
+            if (s && p.ubits) atomicOr(&p.ubits[k >> 5], 1u << (k & 31));
+        }
+        return;
+    }
     const int per = (p.d_ff + kTopkThreads - 1) / kTopkThreads;
     const int k0 = threadIdx.x * per, k1 = min(p.d_ff, k0 + per);
     int ties = 0;
-    if (partial)
-        for (int k = k0; k < k1; ++k) ties += key_at(k) == prefix;
+    for (int k = k0; k < k1; ++k) ties += key_at(k) == prefix;
     int tot = 0;
     int rank = block_exclusive_scan(ties, &tot, sh);
     for (int k = k0; k < k1; ++k) {
@@ -184,14 +204,18 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s, bool pdl) {
+    const size_t whist = 32 * 256 * sizeof(unsigned);
     const size_t keys = (size_t)p.d_ff * sizeof(uint32_t);
     if (keys <= kTopkSmemKeys) {
         static SmemAttrCache cache;
-        cudaError_t e = ensure_smem(k_topk<true>, keys, cache);
+        cudaError_t e = ensure_smem(k_topk<true>, whist + keys, cache);
         if (e != cudaSuccess) return e;
-        return launch_ex(k_topk<true>, dim3(p.n), dim3(kTopkThreads), keys, s, pdl, p);
+        return launch_ex(k_topk<true>, dim3(p.n), dim3(kTopkThreads), whist + keys, s, pdl, p);
     }
-    return launch_ex(k_topk<false>, dim3(p.n), dim3(kTopkThreads), 0, s, pdl, p);
+    static SmemAttrCache cache2;
+    cudaError_t e = ensure_smem(k_topk<false>, whist, cache2);
+    if (e != cudaSuccess) return e;
+    return launch_ex(k_topk<false>, dim3(p.n), dim3(kTopkThreads), whist, s, pdl, p);
 }
 
 }  // namespace sffn
