@@ -91,6 +91,7 @@ struct sffn_ctx {
     float* dpart = nullptr;
     float* fpart = nullptr;      // fused decode: [g1][min(max_tokens, 4)][d] partials of y
     unsigned* tickets = nullptr;
+    unsigned* dbar = nullptr;    // fused decode: grid-barrier arrival counters
     int* status = nullptr;
     void* xdev = nullptr;
     void* ydev = nullptr;
@@ -337,7 +338,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         dp.tau = sel->tau; dp.cpb = P.cpb; dp.mw = P.mw;
         dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
         dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.part = h->fpart;
-        dp.tickets = h->tickets; dp.y = out;
+        dp.tickets = h->dbar; dp.y = out;
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
         h->last_names[launches] = "decode_fused";
         record(h, ++launches, s);
@@ -487,7 +488,8 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_u = take(T * R * 4);
     const size_t o_dp = take((size_t)P.down_chunks * T * D * 4);
     const size_t o_fp = take((size_t)P.g1 * (T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * D * 4);
-    const size_t o_tk = take((size_t)(P.down_slices > 4 ? P.down_slices : 4) * 4), o_st = take(4);
+    const size_t o_tk = take((size_t)(P.down_slices > 2 ? P.down_slices : 2) * 4), o_st = take(4);
+    const size_t o_db = take(16);   // the decode kernel's two grid-barrier counters (64-bit, never reset)
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
     // tensor-core path buffers
     h->tc = c.wdtype == SFFN_BF16 && c.max_tokens > 1;
@@ -514,6 +516,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->dpart = reinterpret_cast<float*>(b + o_dp);
     h->fpart = reinterpret_cast<float*>(b + o_fp);
     h->tickets = reinterpret_cast<unsigned*>(b + o_tk);
+    h->dbar = reinterpret_cast<unsigned*>(b + o_db);
     h->status = reinterpret_cast<int*>(b + o_st);
     h->xdev = b + o_x;
     h->ydev = b + o_y;

@@ -268,7 +268,7 @@ struct DecodeParams {
     int sb, nb;             // streamed piece bytes, pieces in flight per streaming warp
     int* status;
     float* part;            // [CTAs][n][d] per-CTA partials of y
-    unsigned* tickets;      // [3] grid-barrier counters, zero between forwards
+    unsigned* tickets;      // two 64-bit grid-barrier arrival counters (8-byte aligned), zero at creation
     void* y;                // [n][d] T
 };
 

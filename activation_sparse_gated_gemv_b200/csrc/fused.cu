@@ -21,8 +21,9 @@
 //     and every thread adds, for its 8 (or 4) output columns, h_k W_down[k,:]
 //     over that ordered list (whole rows, mostly in L2 by now), and stores the
 //     CTA's fp32 partial of y;
-//   * a grid-wide barrier, then every CTA sums one column slice of y over all
-//     CTAs' partials (in L2) in a fixed order and stores it.
+//   * a grid-wide barrier (a counter that only grows, so nothing resets it),
+//     then every CTA sums one column slice of y over all CTAs' partials (in
+//     L2) in a fixed order and stores it.
 // Every sum has a fixed order, so y is bitwise reproducible.
 #include "common.cuh"
 #include "dot.cuh"
@@ -78,6 +79,19 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, i
     return L;
 }
 
+// Arrival at a grid barrier on a counter that only grows: the barrier of a
+// launch is complete when the counter reaches the next multiple of the grid
+// size, so it never needs resetting (64 bits: no wrap in practice).
+__device__ __forceinline__ unsigned long long grid_arrive(unsigned long long* ctr, unsigned grid) {
+    const unsigned long long old = atomicAdd(ctr, 1ull);
+    return (old / grid + 1) * grid;
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 template <class T, int NT, int GATE>
 __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p) {
     constexpr int V = Elem<T>::kVec;
@@ -99,6 +113,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     uint32_t* smask = reinterpret_cast<uint32_t*>(smem + L.mask);
     uint8_t* flag = reinterpret_cast<uint8_t*>(smem + L.flag);
     int* scan_sh = reinterpret_cast<int*>(smem + L.scan);
+    // grid-barrier arrival counters: [0] the partials of y, [1] LoPA's stage 1
+    unsigned long long* bar = reinterpret_cast<unsigned long long*>(p.tickets);
     const bool streamer = warp < kDecStreamWarps;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + (streamer ? warp : 0) * p.nb;
     unsigned char* bufs = smem + L.bufs + (size_t)(streamer ? warp : 0) * p.nb * p.sb;
@@ -202,11 +218,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         __syncthreads();
         if (threadIdx.x == 0) {
             __threadfence();
-            atomicAdd(p.tickets + 2, 1u);
+            const unsigned long long target = grid_arrive(bar + 1, gridDim.x);
             const unsigned long long t0 = globaltimer_ns();
             unsigned backoff = 32;
             int ok = 1;
-            while (ld_acquire_u32(p.tickets + 2) < gridDim.x) {
+            while (ld_acquire_u64(bar + 1) < target) {
                 if (globaltimer_ns() - t0 > kWaitLimitNs) {
                     atomicOr(p.status, (int)kStatusWaitTimeout);
                     atomicExch(ctr + kAbort, 1);
@@ -428,10 +444,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     const int cps = decode_slice_chunks(p.d, V, G);       // 16-byte chunks per column slice
     const int col0 = blockIdx.x * cps * V;
     __syncthreads();
+    unsigned long long target = 0ull;
     if (threadIdx.x == 0) {
         // release: the CTA's partial (ordered before this thread by the barrier) is visible first
         __threadfence();
-        atomicAdd(p.tickets, 1u);
+        if (col0 < p.d) target = grid_arrive(bar, G);
+        else atomicAdd(bar, 1ull);                        // arrives only, waits for no one
     }
     // the CTA's list, for sffn_get_active only: off the path to the barrier
     for (int i = threadIdx.x; i < tot; i += kDecThreads) {
@@ -445,7 +463,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         if (col0 < p.d) {
             const unsigned long long t0 = globaltimer_ns();
             unsigned backoff = 32;
-            while (ld_acquire_u32(p.tickets) < (unsigned)G) {
+            while (ld_acquire_u64(bar) < target) {
                 if (globaltimer_ns() - t0 > kWaitLimitNs) {
                     atomicOr(p.status, (int)kStatusWaitTimeout);
                     ok = 0;
@@ -501,15 +519,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             dst[2] = from_f32<T>(sum.z);
             dst[3] = from_f32<T>(sum.w);
         }
-    }
-    // The last CTA through resets the barrier counters for the next forward
-    // (every CTA has left the barrier by then).
-    __syncthreads();
-    if (threadIdx.x == 0 && atomicAdd(p.tickets + 1, 1u) == gridDim.x - 1u) {
-        p.tickets[0] = 0u;
-        p.tickets[1] = 0u;
-        p.tickets[2] = 0u;                                // the LoPA stage-1 barrier
-        __threadfence();
     }
 }
 
