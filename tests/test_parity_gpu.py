@@ -262,6 +262,23 @@ def test_deterministic_bitwise(sffn):
     ffn.close()
 
 
+def test_paths_alternate_on_one_handle(sffn):
+    """One handle takes the fused decode kernel (grid-barrier counters), the
+    unfused top-K path (per-forward tickets), the tensor-core path and the
+    fused LoPA kernel in turn; every forward still matches the oracle."""
+    d, d_ff, r = 256, 2048, 64
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=31, gate="both", r=r)
+    ffn = sffn.SparseFFN(d, d_ff, r, 8, "bf16")
+    ffn.set_weights(**w)
+    tau, k = workloads.tau_for_sparsity(0.9), d_ff // 8
+    plan = [(1, "dense", "threshold"), (1, "dense", "topk"), (8, "dense", "threshold"), (1, "lopa", "threshold"),
+            (2, "dense", "topp"), (1, "dense", "threshold"), (8, "lopa", "topk"), (2, "lopa", "threshold")]
+    for i, (n, gate, select) in enumerate(plan * 2):
+        x = workloads.tokens(n, d, "bf16", seed=100 + i)
+        check_forward(ffn, w, x, gate, select, tau=tau, k=k, p=0.6)
+    ffn.close()
+
+
 def test_forward_host_matches_device_forward(sffn):
     ffn, w, x = _small(sffn)
     tau = workloads.tau_for_sparsity(0.8)
