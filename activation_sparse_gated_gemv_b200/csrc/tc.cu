@@ -341,27 +341,6 @@ __device__ __forceinline__ void emit16(const TcParams& p, int m, int c0, const f
             o[(long long)tok * p.ldo + m] = hi;
             o[(long long)(p.npad + tok) * p.ldo + m] = lo;
         }
-    } else if (p.mode == kTcUp) {
-        // m is the channel; channels past d_ff (the last block's tail) write zeros
-        bf16* o = static_cast<bf16*>(p.out);
-        float gv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int tok = c0 + i;
-            gv[i] = 0.f;
-            if (m < p.m_total && tok < p.n) {
-                const long long zi = (long long)tok * p.ldsel + m;
-                gv[i] = p.topk ? p.gsel[zi] : fmaxf(p.zsel[zi] - p.tau, 0.f);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int tok = c0 + i;
-            const float h = gv[i] * v[i];
-            const bf16 hi = __float2bfloat16_rn(h);
-            o[(long long)tok * p.ldo + m] = hi;
-            if (p.h_pairs) o[(long long)(p.npad + tok) * p.ldo + m] = __float2bfloat16_rn(h - __bfloat162float(hi));
-        }
     } else {  // down
         if (m >= p.m_total) return;
         bf16* o = static_cast<bf16*>(p.out);
@@ -373,6 +352,79 @@ __device__ __forceinline__ void emit16(const TcParams& p, int m, int c0, const f
     }
 }
 
+// ---- up epilogue ---------------------------------------------------------------
+// h(token, m) = g(token, m) * acc, g the gate activation of channel m for the
+// token (ReLU(z - tau), or the selected SiLU value; zero past n and d_ff).
+// The gate values of a tile are loaded into registers before its accumulator
+// is ready, so their latency hides behind the mainloop instead of costing one
+// round trip per 16 tokens after it.
+
+constexpr int kUpChunks = kTcMaxTokens / 16;
+
+struct UpG {
+    float raw[kUpChunks * 16];
+};
+
+// Issue the loads of the gate source (z or the selected g) of channel m for the
+// first `cols` token columns.
+__device__ __forceinline__ void up_g_load(const TcParams& p, int m, int cols, UpG& g) {
+    const float* src = p.topk ? p.gsel : p.zsel;
+    const bool row_ok = m < p.m_total;
+#pragma unroll
+    for (int j = 0; j < kUpChunks; ++j) {
+        if (16 * j < cols) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int tok = 16 * j + i;
+                g.raw[16 * j + i] = (row_ok && tok < p.n) ? __ldcg(src + (long long)tok * p.ldsel + m) : 0.f;
+            }
+        }
+    }
+}
+
+// Columns 16j..16j+15 of channel m: h = g * v, written as bf16 hi (and lo) rows.
+__device__ __forceinline__ void up_emit16(const TcParams& p, int m, int j, const float* v, const UpG& g) {
+    bf16* o = static_cast<bf16*>(p.out);
+    const bool row_ok = m < p.m_total;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int tok = 16 * j + i;
+        const float raw = g.raw[16 * j + i];
+        const float gv = (row_ok && tok < p.n) ? (p.topk ? raw : fmaxf(raw - p.tau, 0.f)) : 0.f;
+        const float h = gv * v[i];
+        const bf16 hi = __float2bfloat16_rn(h);
+        o[(long long)tok * p.ldo + m] = hi;
+        if (p.h_pairs) o[(long long)(p.npad + tok) * p.ldo + m] = __float2bfloat16_rn(h - __bfloat162float(hi));
+    }
+}
+
+// Columns c0..c0+15 of row `row` of a cut tile: the sum of its parts in CTA order.
+__device__ __forceinline__ void part_sum16(const TcParams& p, int c_first, int c_last, int row, int c0,
+                                           size_t slot_floats, float* v) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+        const float* pp = p.part + ((size_t)c * 2 + (c == c_first ? 0 : 1)) * slot_floats + (size_t)row * p.nb + c0;
+        float4 a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(pp) + i);
+        if (p.paired) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) b[i] = __ldcg(reinterpret_cast<const float4*>(pp + p.npad) + i);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[4 * i] += a[i].x + b[i].x;
+            v[4 * i + 1] += a[i].y + b[i].y;
+            v[4 * i + 2] += a[i].z + b[i].z;
+            v[4 * i + 3] += a[i].w + b[i].w;
+        }
+    }
+}
+
 // Sum of the parts of 32-row quarter `quarter` of a cut tile, in CTA order,
 // once every part has arrived; the last of the tile's four quarter sums resets
 // its counters for the next launch.
@@ -380,8 +432,11 @@ __device__ void sum_quarter(const TcParams& p, int t, int m0, int c_first, int c
                             int cols, size_t slot_floats) {
     const int lane = threadIdx.x & 31;
     const int parts = c_last - c_first + 1;
+    const int m = m0 + row;
     unsigned* arrivals = p.tickets + 2 * t;
     unsigned* finished = arrivals + 1;
+    UpG g;
+    if (p.mode == kTcUp) up_g_load(p, m, cols, g);   // in flight while the parts arrive
     bool ready = true;
     if (lane == 0) {
         const unsigned long long t0 = globaltimer_ns();
@@ -401,34 +456,21 @@ __device__ void sum_quarter(const TcParams& p, int t, int m0, int c_first, int c
         return;
     }
     __threadfence();
-    const int m = m0 + row;
     bool act = false;
-    for (int c0 = 0; c0 < cols; c0 += 16) {
-        float v[16];
+    if (p.mode == kTcUp) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.f;
-        for (int c = c_first; c <= c_last; ++c) {
-            const float* pp =
-                p.part + ((size_t)c * 2 + (c == c_first ? 0 : 1)) * slot_floats + (size_t)row * p.nb + c0;
-            float4 a[4], b[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(pp) + i);
-            if (p.paired) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) b[i] = __ldcg(reinterpret_cast<const float4*>(pp + p.npad) + i);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[4 * i] += a[i].x + b[i].x;
-                v[4 * i + 1] += a[i].y + b[i].y;
-                v[4 * i + 2] += a[i].z + b[i].z;
-                v[4 * i + 3] += a[i].w + b[i].w;
-            }
+        for (int j = 0; j < kUpChunks; ++j) {
+            if (16 * j >= cols) break;
+            float v[16];
+            part_sum16(p, c_first, c_last, row, 16 * j, slot_floats, v);
+            up_emit16(p, m, j, v, g);
         }
-        emit16(p, m, c0, v, act);
+    } else {
+        for (int c0 = 0; c0 < cols; c0 += 16) {
+            float v[16];
+            part_sum16(p, c_first, c_last, row, c0, slot_floats, v);
+            emit16(p, m, c0, v, act);
+        }
     }
     if (p.mode == kTcGateZ && p.ubits) {
         const unsigned bits = __ballot_sync(0xffffffffu, act && !p.topk && m < p.m_total);
@@ -460,6 +502,11 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
         const int acc = segi & 1;
         const uint32_t use = (uint32_t)(segi >> 1);
         ++segi;
+        const bool whole = s.kb0 == 0 && s.kb1 == q.KB;
+        const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
+        const int m = m0 + row;
+        UpG g;
+        if (p.mode == kTcUp && whole) up_g_load(p, m, cols, g);   // in flight during the mainloop
         if (!mbar_wait_warp(&sh->tfull[acc], use & 1u)) {
             sh->abort = 1;
             set_status(p.status, kStatusWaitTimeout);
@@ -467,10 +514,17 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
         }
         tc_fence_after();
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.nb);
-        const bool whole = s.kb0 == 0 && s.kb1 == q.KB;
-        const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
-        const int m = m0 + row;
-        if (whole) {
+        if (whole && p.mode == kTcUp) {
+#pragma unroll
+            for (int j = 0; j < kUpChunks; ++j) {
+                if (16 * j >= cols) break;
+                float v[16];
+                tmem_ld16(taddr + 16 * j, v);
+                up_emit16(p, m, j, v, g);
+            }
+            tc_fence_before();
+            mbar_arrive(&sh->tempty[acc]);
+        } else if (whole) {
             bool act = false;
             for (int c0 = 0; c0 < cols; c0 += 16) {
                 float v[16];
