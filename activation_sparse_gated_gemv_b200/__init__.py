@@ -14,8 +14,9 @@ channels' ``W_up``/``W_down`` rows read ("Model Casting and Low-Parameter
 Gating", abstract; "Mixture-of-Channels", sections "Dentro il mixture" and
 "Dentro MoC"; "PrunePath", abstract).
 
-There is no fallback: importing this package fails if ``libsffn.so`` is
-missing, and every call that needs a GPU fails if there is none.
+There is no fallback: importing this package builds ``libsffn.so`` if it is
+missing and fails if it cannot, and every call that needs a GPU fails if there
+is none.
 """
 from __future__ import annotations
 
@@ -52,8 +53,10 @@ class sffn_select(ctypes.Structure):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      f"`python -m activation_sparse_gated_gemv_b200.build` (needs nvcc)")
+    # a fresh checkout: compile the library in-tree first (nvcc, sm_100a); if
+    # that fails the import fails with it
+    from . import build as _build
+    _build.build()
 _lib = ctypes.CDLL(LIB_PATH)
 
 _P, _I = ctypes.c_void_p, ctypes.c_int

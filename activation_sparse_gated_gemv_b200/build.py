@@ -7,6 +7,7 @@ host process has already loaded.
 """
 from __future__ import annotations
 
+import fcntl
 import glob
 import os
 import shutil
@@ -54,6 +55,15 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = N
     if not force and up_to_date():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
+    # one build at a time (test workers and ranks may import together)
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        if not force and up_to_date():
+            return LIB
+        return _build_locked(verbose_ptxas, jobs)
+
+
+def _build_locked(verbose_ptxas: bool, jobs: int | None) -> str:
     exe = nvcc()
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
 
