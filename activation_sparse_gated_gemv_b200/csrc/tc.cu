@@ -31,14 +31,14 @@
 //              N = token columns, K = 16 per instruction, bf16 in, fp32
 //              accumulate in tensor memory) and tcgen05.commit;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
-//              lanes), the mode's epilogue, stores.
+//              lanes), the mode's epilogue, stores;
+//   warp 6     one thread: the second TMA producer (alternate k-blocks).
 // Work is split stream-K: the (tile, k-block) iterations are cut into one
 // contiguous range per CTA, so every SM streams the same number of weight
-// bytes.  A tile cut between CTAs is summed in a fixed order (by CTA index)
-// once all its parts have arrived, each 32-row quarter by one of the tile's
-// CTAs after it has written all of its own parts (so no wait can hold back a
-// part another CTA needs); results are deterministic and no single CTA
-// serialises the tail.
+// bytes.  A tile cut between CTAs is finished by the CTA holding its first
+// k-blocks (at the end of that CTA's range), which adds the other CTAs' parts,
+// parked early in their ranges, in CTA order: results are deterministic and
+// the end of a range waits only for parts written long before.
 //
 // fp32 intermediates that feed a later MMA (LoPA's u = x A, and h) are passed
 // as two bf16 rows, hi = bf16(v) and lo = bf16(v - hi); the MMA multiplies both
@@ -58,7 +58,9 @@ constexpr int kProdWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;        // epilogue warps 2..5
 constexpr int kEpi = 4;
-constexpr int kTcThreads = (kEpiWarp0 + kEpi) * 32;
+constexpr int kProdWarp2 = kEpiWarp0 + kEpi;   // second TMA producer (warp 6)
+constexpr int kProducers = 2;
+constexpr int kTcThreads = (kProdWarp2 + 1) * 32;
 constexpr uint32_t kTileA = kBM * kBK * 2;   // 16 KB
 constexpr int kMaxStages = 12;
 constexpr int kMaxBlocks = 1024;    // 128-channel blocks (d_ff <= 131072)
@@ -71,6 +73,7 @@ struct TcShared {
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
+    uint64_t fix;           // the owner's staged copy of the other parts of its cut tile
     uint32_t tmem_base;
     int abort;
     int reducer;
@@ -144,6 +147,12 @@ __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, i
         " [%0], [%1, {%2, %3}], [%4], %5;"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
+}
+// Ask the TMA engine to bring the box at (x, y) of the tensor map into L2.
+__device__ __forceinline__ void tma_prefetch_tile(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y)
+                 : "memory");
 }
 __device__ __forceinline__ uint64_t l2_evict_last() {
     uint64_t pol;
@@ -230,10 +239,42 @@ __device__ __forceinline__ bool next_seg(const Problem& q, long long& it, Seg& s
     return true;
 }
 
+// Before the wait for the previous kernel: the weight boxes of this CTA's first
+// `count` k-blocks into L2, so the ring fills from L2 once the wait ends.
+// Weights do not depend on earlier kernels.  The up and down passes do not know
+// their active blocks yet; they take the boxes of the case where every block
+// is active, which is the usual one with several tokens (a wrong guess costs
+// only the prefetched bytes).
+__device__ void prefetch_first_tiles(const TcParams& p, int count) {
+    const bool blocks = p.mode == kTcUp || p.mode == kTcDown;
+    const Problem q = make_problem(p, blocks ? (p.d_ff + 127) / 128 : 0);
+    long long it = q.it0;
+    int done = 0;
+    Seg s;
+    while (done < count && next_seg(q, it, s)) {
+        for (int kb = s.kb0; kb < s.kb1 && done < count; ++kb, ++done) {
+            if (p.mode == kTcDown) {
+                const int c0 = (kb >> 1) * kBM + (kb & 1) * kBK;
+                tma_prefetch_tile(&p.ta, s.t * kBM, c0);
+                tma_prefetch_tile(&p.ta, s.t * kBM + 64, c0);
+            } else {
+                tma_prefetch_tile(&p.ta, kb * kBK, s.t * kBM);
+            }
+        }
+    }
+}
+
 // ---- producer: one thread issues the TMA copies --------------------------------
 
+// Producer `pr` of kProducers fills the stages of the k-blocks g with
+// g % kProducers == pr.  One thread issuing every copy of an SM's stream keeps
+// only about three quarters of HBM bandwidth busy; two threads in different
+// warps, taking alternate k-blocks of the same ring, reach the copy peak.  The
+// ring stays one sequence for the MMA issuer.  (A producer waits for stage
+// g - S to be consumed; with kProducers <= S the parity wait cannot be a phase
+// behind.)
 __device__ void run_producer(const TcParams& p, const Problem& q, unsigned char* stages, uint32_t stage_bytes,
-                             TcShared* sh) {
+                             TcShared* sh, int pr) {
     const uint64_t pol_w = l2_evict_first(), pol_b = l2_evict_last();
     const int S = p.stages;
     const uint32_t tx = kTileA + (uint32_t)p.nb * 128u;
@@ -242,6 +283,7 @@ __device__ void run_producer(const TcParams& p, const Problem& q, unsigned char*
     while (next_seg(q, it, s)) {
         const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++g) {
+            if ((int)(g % kProducers) != pr) continue;
             const int st = (int)(g % S);
             if (!mbar_wait_one(&sh->empty[st], (uint32_t)(((g / S) & 1) ^ 1))) {
                 sh->abort = 1;
@@ -398,22 +440,43 @@ __device__ __forceinline__ void up_emit16(const TcParams& p, int m, int j, const
     }
 }
 
-// Columns c0..c0+15 of row `row` of a cut tile: the sum of its parts in CTA order.
-__device__ __forceinline__ void part_sum16(const TcParams& p, int c_first, int c_last, int row, int c0,
-                                           size_t slot_floats, float* v) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = 0.f;
-    for (int c = c_first; c <= c_last; ++c) {
-        const float* pp = p.part + ((size_t)c * 2 + (c == c_first ? 0 : 1)) * slot_floats + (size_t)row * p.nb + c0;
+// ---- stream-K fix-up ----------------------------------------------------------
+// A tile cut between CTAs c_first < ... < c_last: c_first holds the tile's first
+// k-blocks, at the end of its range (its last segment), and owns the tile.  Every
+// later CTA holds the tile in its first (or only) segment and parks its partial
+// accumulator in its part slot early in its run.  The owner adds those parts, in
+// CTA order, to its own accumulator and finishes the tile as it would a whole
+// one.  So the only wait at the end of a range is for parts that are normally
+// written long before, no CTA waits for a range that ends as late as its own,
+// and the owner's partial sum never goes through memory.  The waits point to
+// higher CTA indices only, so they cannot form a cycle.
+
+// Parts are parked row-major (row = TMEM lane, nb floats: the hi columns, then
+// the lo), with the 16-byte chunks of each row permuted by an XOR with the row
+// index, so the 32 rows a warp reads at one column sit in different banks once
+// staged in shared memory.
+__device__ __forceinline__ int part_swz_mask(int nb) {
+    const int q4 = nb >> 2;               // a multiple of 4
+    return min(q4 & -q4, 8) - 1;
+}
+
+// v[0..15] += the np parts at base, base + stride, ... (in that order) at
+// columns c0..c0+15 of row `row` (each part's hi + lo columns when paired).
+// `global` selects L2 loads (parts still in global memory) over plain loads
+// (parts staged in shared memory).
+__device__ __forceinline__ void add_parts16(const TcParams& p, const float* base, size_t stride, int np, int row,
+                                            int c0, bool global, float* v) {
+    const int mask = part_swz_mask(p.nb);
+    for (int k = 0; k < np; ++k) {
+        const float4* r4 = reinterpret_cast<const float4*>(base + (size_t)k * stride + (size_t)row * p.nb);
         float4 a[4], b[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(pp) + i);
-        if (p.paired) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) b[i] = __ldcg(reinterpret_cast<const float4*>(pp + p.npad) + i);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 4; ++i) {
+            const int ja = ((c0 >> 2) + i) ^ (row & mask);
+            const int jb = ((p.npad + c0) >> 2) + i;
+            a[i] = global ? __ldcg(r4 + ja) : r4[ja];
+            b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p.paired) b[i] = global ? __ldcg(r4 + (jb ^ (row & mask))) : r4[jb ^ (row & mask)];
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -425,65 +488,29 @@ __device__ __forceinline__ void part_sum16(const TcParams& p, int c_first, int c
     }
 }
 
-// Sum of the parts of 32-row quarter `quarter` of a cut tile, in CTA order,
-// once every part has arrived; the last of the tile's four quarter sums resets
-// its counters for the next launch.
-__device__ void sum_quarter(const TcParams& p, int t, int m0, int c_first, int c_last, int quarter, int row,
-                            int cols, size_t slot_floats) {
-    const int lane = threadIdx.x & 31;
-    const int parts = c_last - c_first + 1;
-    const int m = m0 + row;
-    unsigned* arrivals = p.tickets + 2 * t;
-    unsigned* finished = arrivals + 1;
-    UpG g;
-    if (p.mode == kTcUp) up_g_load(p, m, cols, g);   // in flight while the parts arrive
+// The owner's wait (bounded) until `want` parts of tile t have arrived.
+__device__ __forceinline__ bool wait_parts(const TcParams& p, int t, unsigned want) {
+    const unsigned* arrivals = p.tickets + 2 * t;
     bool ready = true;
-    if (lane == 0) {
+    if ((threadIdx.x & 31) == 0 && ld_acquire(arrivals) < want) {
         const unsigned long long t0 = globaltimer_ns();
-        unsigned backoff = 64;
-        while (ld_acquire(arrivals) < (unsigned)parts) {
+        unsigned backoff = 32;
+        while (ld_acquire(arrivals) < want) {
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 ready = false;
                 break;
             }
             __nanosleep(backoff);
-            if (backoff < 1024) backoff <<= 1;
+            if (backoff < 256) backoff <<= 1;
         }
     }
     ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-    if (!ready) {
-        set_status(p.status, kStatusWaitTimeout);
-        return;
-    }
     __threadfence();
-    bool act = false;
-    if (p.mode == kTcUp) {
-#pragma unroll
-        for (int j = 0; j < kUpChunks; ++j) {
-            if (16 * j >= cols) break;
-            float v[16];
-            part_sum16(p, c_first, c_last, row, 16 * j, slot_floats, v);
-            up_emit16(p, m, j, v, g);
-        }
-    } else {
-        for (int c0 = 0; c0 < cols; c0 += 16) {
-            float v[16];
-            part_sum16(p, c_first, c_last, row, c0, slot_floats, v);
-            emit16(p, m, c0, v, act);
-        }
-    }
-    if (p.mode == kTcGateZ && p.ubits) {
-        const unsigned bits = __ballot_sync(0xffffffffu, act && !p.topk && m < p.m_total);
-        if (lane == 0) p.ubits[(m0 + quarter * 32) >> 5] = bits;
-    }
-    __syncwarp();
-    if (lane == 0 && atomicAdd(finished, 1u) == 3u) {
-        *arrivals = 0u;
-        *finished = 0u;
-    }
+    return ready;
 }
 
-__device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, uint32_t tmem) {
+__device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, uint32_t tmem,
+                             unsigned char* ring, size_t ring_bytes) {
     const int warp = threadIdx.x >> 5;
     const int quarter = warp & 3;                     // TMEM lanes this warp may access
     const int lane = threadIdx.x & 31;
@@ -492,9 +519,6 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
     const int cols = p.paired ? p.npad : p.nb;        // final columns
     const int C = q.C;
     const size_t slot_floats = (size_t)p.nb * kBM;
-    // cut tiles this CTA takes part in (its first and last segments at most)
-    int cut_t[2], cut_m0[2], cut_first[2], cut_last[2];
-    int ncut = 0;
     long long it = q.it0;
     int segi = 0;
     Seg s;
@@ -503,10 +527,18 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
         const uint32_t use = (uint32_t)(segi >> 1);
         ++segi;
         const bool whole = s.kb0 == 0 && s.kb1 == q.KB;
+        const int c_first = whole ? (int)blockIdx.x : cta_of((long long)s.t * q.KB, q.I, C);
+        const int c_last = whole ? (int)blockIdx.x : cta_of((long long)(s.t + 1) * q.KB - 1, q.I, C);
+        const bool owner = c_first == (int)blockIdx.x;
         const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
         const int m = m0 + row;
         UpG g;
-        if (p.mode == kTcUp && whole) up_g_load(p, m, cols, g);   // in flight during the mainloop
+        if (p.mode == kTcUp && owner) up_g_load(p, m, cols, g);   // in flight during the mainloop
+        if (owner && !whole && !wait_parts(p, s.t, (unsigned)(c_last - c_first))) {
+            sh->abort = 1;
+            set_status(p.status, kStatusWaitTimeout);
+            return;
+        }
         if (!mbar_wait_warp(&sh->tfull[acc], use & 1u)) {
             sh->abort = 1;
             set_status(p.status, kStatusWaitTimeout);
@@ -514,28 +546,55 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
         }
         tc_fence_after();
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * p.nb);
-        if (whole && p.mode == kTcUp) {
-#pragma unroll
-            for (int j = 0; j < kUpChunks; ++j) {
-                if (16 * j >= cols) break;
-                float v[16];
-                tmem_ld16(taddr + 16 * j, v);
-                up_emit16(p, m, j, v, g);
-            }
-            tc_fence_before();
-            mbar_arrive(&sh->tempty[acc]);
-        } else if (whole) {
-            bool act = false;
-            for (int c0 = 0; c0 < cols; c0 += 16) {
-                float v[16];
-                tmem_ld16(taddr + c0, v);
-                if (p.paired) {
-                    float x[16];
-                    tmem_ld16(taddr + p.npad + c0, x);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] += x[i];
+        if (owner) {
+            // the other parts: staged into the (now idle) stage ring with bulk copies
+            // when they fit, else read from L2 chunk by chunk
+            const int np = c_last - c_first;
+            const float* pbase = p.part + (size_t)(c_first + 1) * slot_floats;
+            bool pglobal = true;
+            if (np > 0 && (size_t)np * slot_floats * 4 <= ring_bytes) {
+                // the last segment's accumulator is complete, so every MMA has read
+                // its stages and no copy into the ring is in flight
+                if (etid == 0) {
+                    const uint32_t bytes = (uint32_t)((size_t)np * slot_floats * 4);
+                    const uint64_t pol = l2_evict_first();
+                    fence_proxy_async_global();
+                    mbar_expect_tx(&sh->fix, bytes);
+                    for (uint32_t o = 0; o < bytes; o += 16384u)
+                        bulk_load(ring + o, reinterpret_cast<const unsigned char*>(pbase) + o,
+                                  min(16384u, bytes - o), &sh->fix, pol);
                 }
-                emit16(p, m, c0, v, act);
+                if (!mbar_wait_warp(&sh->fix, 0)) {
+                    sh->abort = 1;
+                    set_status(p.status, kStatusWaitTimeout);
+                    return;
+                }
+                pbase = reinterpret_cast<const float*>(ring);
+                pglobal = false;
+            }
+            bool act = false;
+            if (p.mode == kTcUp) {
+#pragma unroll
+                for (int j = 0; j < kUpChunks; ++j) {
+                    if (16 * j >= cols) break;
+                    float v[16];
+                    tmem_ld16(taddr + 16 * j, v);
+                    add_parts16(p, pbase, slot_floats, np, row, 16 * j, pglobal, v);
+                    up_emit16(p, m, j, v, g);
+                }
+            } else {
+                for (int c0 = 0; c0 < cols; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(taddr + c0, v);
+                    if (p.paired) {
+                        float x[16];
+                        tmem_ld16(taddr + p.npad + c0, x);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] += x[i];
+                    }
+                    add_parts16(p, pbase, slot_floats, np, row, c0, pglobal, v);
+                    emit16(p, m, c0, v, act);
+                }
             }
             tc_fence_before();
             mbar_arrive(&sh->tempty[acc]);
@@ -544,39 +603,34 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
                 const unsigned bits = __ballot_sync(0xffffffffu, act && !p.topk && m < p.m_total);
                 if (lane == 0) p.ubits[(m0 + quarter * 32) >> 5] = bits;
             }
+            if (!whole) {
+                // the last of the owner's four warps resets the tile's counters for the next launch
+                __syncwarp();
+                unsigned* arrivals = p.tickets + 2 * s.t;
+                if (lane == 0 && atomicAdd(arrivals + 1, 1u) == 3u) {
+                    arrivals[0] = 0u;
+                    arrivals[1] = 0u;
+                }
+            }
         } else {
-            // cut tile: park this CTA's part (row-major, each thread's row contiguous)
-            const int c_first = cta_of((long long)s.t * q.KB, q.I, C);
-            const int c_last = cta_of((long long)(s.t + 1) * q.KB - 1, q.I, C);
-            const int slot = c_first == (int)blockIdx.x ? 0 : 1;
-            float* mine = p.part + ((size_t)blockIdx.x * 2 + slot) * slot_floats + (size_t)row * p.nb;
+            // a later part of a cut tile: park it for the owner
+            float4* mine = reinterpret_cast<float4*>(p.part + (size_t)blockIdx.x * slot_floats + (size_t)row * p.nb);
+            const int mask = part_swz_mask(p.nb);
             for (int c0 = 0; c0 < p.nb; c0 += 16) {
                 float v[16];
                 tmem_ld16(taddr + c0, v);
 #pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    *reinterpret_cast<float4*>(mine + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                for (int i = 0; i < 4; ++i)
+                    mine[((c0 >> 2) + i) ^ (row & mask)] =
+                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
             tc_fence_before();
             mbar_arrive(&sh->tempty[acc]);
+            fence_proxy_async_global();   // the owner may read the part with bulk copies
             __threadfence();
             named_sync(1, kEpi * 32);
             if (etid == 0) atomicAdd(p.tickets + 2 * s.t, 1u);
-            if (ncut < 2) {
-                cut_t[ncut] = s.t;
-                cut_m0[ncut] = m0;
-                cut_first[ncut] = c_first;
-                cut_last[ncut] = c_last;
-                ++ncut;
-            }
         }
-    }
-    // Every part of this CTA is out; now the quarter sums it owns: quarter j of
-    // a cut tile is summed by CTA c_first + j mod parts (one warp each).
-    for (int i = 0; i < ncut; ++i) {
-        const int parts = cut_last[i] - cut_first[i] + 1;
-        if (quarter % parts == (int)blockIdx.x - cut_first[i])
-            sum_quarter(p, cut_t[i], cut_m0[i], cut_first[i], cut_last[i], quarter, row, cols, slot_floats);
     }
 }
 
@@ -598,6 +652,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
             mbar_init(&sh->tempty[i], kEpi * 32);
         }
         mbar_init(&sh->drain, 1);
+        mbar_init(&sh->fix, 1);
         sh->abort = 0;
         sh->reducer = 0;
         fence_mbar_init();
@@ -608,6 +663,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
 
+    if (warp == kProdWarp && (threadIdx.x & 31) == 0) prefetch_first_tiles(p, p.stages);
     griddep_launch_dependents();
     griddep_wait();
     int nblk = 0;
@@ -651,12 +707,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
         }
     }
 
-    if (warp == kProdWarp) {
-        if ((threadIdx.x & 31) == 0) run_producer(p, q, stages, stage_bytes, sh);
+    if (warp == kProdWarp || warp == kProdWarp2) {
+        if ((threadIdx.x & 31) == 0) run_producer(p, q, stages, stage_bytes, sh, warp == kProdWarp ? 0 : 1);
     } else if (warp == kMmaWarp) {
         if ((threadIdx.x & 31) == 0) run_mma(p, q, stages, stage_bytes, sh, tmem);
     } else {
-        run_epilogue(p, q, sh, tmem);
+        run_epilogue(p, q, sh, tmem, stages, (size_t)p.stages * stage_bytes);
     }
     tc_fence_before();
     __syncthreads();
