@@ -75,6 +75,7 @@ _sigs = {
     "sffn_last_error": ([], ctypes.c_char_p),
     "sffn_forward_noalloc": ([_P, _P, _P, _I, _I, _I, _P, _I, ctypes.c_float, _P, _P], _I),
     "sffn_last_kernel_name": ([_P, _I], ctypes.c_char_p),
+    "sffn_set_hot": ([_P, _P, _I], _I),
 }
 for _name, (_args, _res) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -96,6 +97,7 @@ sffn_strerror = _lib.sffn_strerror
 sffn_last_error = _lib.sffn_last_error
 sffn_forward_noalloc = _lib.sffn_forward_noalloc
 sffn_last_kernel_name = _lib.sffn_last_kernel_name
+sffn_set_hot = _lib.sffn_set_hot
 
 EXPORTED = tuple(_sigs)
 
@@ -207,6 +209,17 @@ class SparseFFN:
         check(sffn_get_active(self._h, idx.ctypes.data_as(ctypes.c_void_p),
                               cnt.ctypes.data_as(ctypes.c_void_p), ctypes.byref(uni)), "sffn_get_active")
         return [idx[t, :cnt[t]].copy() for t in range(n)], int(uni.value)
+
+    def set_hot(self, channels) -> None:
+        """Heavy-hitter channels (any int sequence; empty clears the set): the
+        fused decode kernel takes their up dots before the gate selects them.
+        y and the active lists do not change."""
+        a64 = np.asarray(channels, dtype=np.int64).reshape(-1)
+        if a64.size and (a64.min() < -2**31 or a64.max() >= 2**31):
+            raise SFFNError(SFFN_ERR_INVALID_ARG, "sffn_set_hot")
+        arr = np.ascontiguousarray(a64.astype(np.int32))
+        check(sffn_set_hot(self._h, arr.ctypes.data_as(ctypes.c_void_p) if arr.size else None, int(arr.size)),
+              "sffn_set_hot")
 
     def set_stage_events(self, events) -> None:
         arr = (ctypes.c_void_p * max(1, len(events)))(*[e.cuda_event for e in events])

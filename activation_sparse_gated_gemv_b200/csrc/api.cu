@@ -116,6 +116,8 @@ struct sffn_ctx {
     int last_launches = 0;
     const char* last_names[8] = {};
     std::vector<cudaEvent_t> events;
+    uint32_t* hot = nullptr;     // heavy-hitter channel bits [ceil(d_ff / 32)] (kept once allocated)
+    bool hot_on = false;         // a non-empty hot set is in force
 };
 
 namespace {
@@ -338,7 +340,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         dp.tau = sel->tau; dp.cpb = P.cpb; dp.mw = P.mw;
         dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
         dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.part = h->fpart;
-        dp.tickets = h->dbar; dp.y = out;
+        dp.tickets = h->dbar; dp.y = out; dp.hot = h->hot_on ? h->hot : nullptr;
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
         h->last_names[launches] = "decode_fused";
         record(h, ++launches, s);
@@ -720,6 +722,33 @@ int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union
     return SFFN_OK;
 }
 
+int sffn_set_hot(sffn_handle h, const int32_t* channels, int count) {
+    if (!h || count < 0 || (count > 0 && !channels)) return fail(SFFN_ERR_INVALID_ARG, "bad hot channel list");
+    const int d_ff = h->cfg.d_ff;
+    std::vector<uint32_t> bits(((size_t)d_ff + 31) / 32, 0u);
+    for (int i = 0; i < count; ++i) {
+        if (channels[i] < 0 || channels[i] >= d_ff) return fail(SFFN_ERR_INVALID_ARG, "hot channel out of range");
+        bits[(size_t)channels[i] >> 5] |= 1u << (channels[i] & 31);
+    }
+    DeviceGuard g(h->cfg.device);
+    if (count == 0 && !h->hot) return SFFN_OK;
+    // The buffer is never freed before the handle, so a graph captured with
+    // an earlier set keeps a valid (all-clear after a clear) bitmap.
+    if (!h->hot) {
+        void* p = nullptr;
+        if (cudaMalloc(&p, bits.size() * sizeof(uint32_t)) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(SFFN_ERR_OOM, "hot set allocation");
+        }
+        h->hot = static_cast<uint32_t*>(p);
+    }
+    // earlier forwards may still read the old set
+    SFFN_CUDA(cudaDeviceSynchronize(), "hot set update");
+    SFFN_CUDA(cudaMemcpy(h->hot, bits.data(), bits.size() * sizeof(uint32_t), cudaMemcpyHostToDevice), "hot set copy");
+    h->hot_on = count > 0;
+    return SFFN_OK;
+}
+
 int sffn_set_stage_events(sffn_handle h, void* const* events, int n_events) {
     if (!h || n_events < 0 || (n_events > 0 && !events)) return fail(SFFN_ERR_INVALID_ARG, "bad events");
     h->events.clear();
@@ -744,6 +773,7 @@ int sffn_destroy(sffn_handle h) {
         DeviceGuard g(h->cfg.device);
         free_weights(h);
         if (h->ws) cudaFree(h->ws);
+        if (h->hot) cudaFree(h->hot);
     }
     delete h;
     return SFFN_OK;

@@ -275,6 +275,7 @@ struct DecodeParams {
     float* part;            // [CTAs][n][d] per-CTA partials of y
     unsigned* tickets;      // two 64-bit grid-barrier arrival counters (8-byte aligned), zero at creation
     void* y;                // [n][d] T
+    const uint32_t* hot;    // [ceil(d_ff / 32)] heavy-hitter channel bits, or NULL
 };
 
 // Batched tensor-core GEMM (tcgen05): modes and parameters.

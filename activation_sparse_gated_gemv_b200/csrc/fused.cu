@@ -14,9 +14,12 @@
 //     dot products in shared memory.  When a row's last piece is in, the warp
 //     that finished it adds the pieces in order (z), selects (z > tau), and for
 //     an active channel pulls its W_down row into L2 and queues the channel;
+//   * with a heavy-hitter set, warps 14 and 15 first take the up dots of the
+//     CTA's hot channels, before and independent of the gate;
 //   * warps 14 and 15 take queued channels at once and compute the up dot
-//     <x, W_up[:,k]> and h = (z - tau) u (the streaming warps join them when
-//     their pieces are done), so the W_up rows are read while the gate streams;
+//     <x, W_up[:,k]> (a hot channel's is already in) and h = (z - tau) u (the
+//     streaming warps join them when their pieces are done), so the W_up rows
+//     are read while the gate streams;
 //   * after a barrier the active channels are compacted in ascending order
 //     and every thread adds, for its 8 (or 4) output columns, h_k W_down[k,:]
 //     over that ordered list (whole rows, mostly in L2 by now), and stores the
@@ -36,7 +39,7 @@ constexpr int kDecStreamWarps = 14;        // the other warps start as up worker
 constexpr int kQueueTail = 0, kQueueHead = 1, kGateDone = 2, kAbort = 3;
 
 struct DecodeSmem {
-    size_t xs, us, zpart, zfin, hs, done, queue, ctr, wl, mask, flag, scan, bars, bufs, total;
+    size_t xs, us, zpart, zfin, hs, hu, done, queue, ctr, wl, mask, flag, hrdy, scan, bars, bufs, total;
 };
 
 // Chunks (16 bytes of `vec` elements) per column slice of the down pass: the
@@ -62,12 +65,14 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, i
     L.zpart = o; o += (size_t)cpb * ppr * nt * sizeof(float);
     L.zfin = o;  o += (size_t)cpb * nt * sizeof(float);
     L.hs = o;    o += (size_t)cpb * nt * sizeof(float);
+    L.hu = o;    o += (size_t)cpb * nt * sizeof(float);
     L.done = o;  o += (size_t)cpb * sizeof(int);
     L.queue = o; o += (size_t)cpb * sizeof(int);
     L.ctr = o;   o += 4 * sizeof(int);
     L.wl = o;    o += (size_t)cpb * sizeof(int);
     L.mask = o;  o += (size_t)cpb * mw * sizeof(uint32_t);
     L.flag = o;  o += ((size_t)cpb + 15) & ~(size_t)15;
+    L.hrdy = o;  o += ((size_t)cpb + 15) & ~(size_t)15;
     L.scan = o;  o += 48 * sizeof(int);
     o = (o + 15) & ~(size_t)15;
     L.bars = o;  o += (size_t)kDecStreamWarps * nb * sizeof(uint64_t);
@@ -112,6 +117,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     int* wl = reinterpret_cast<int*>(smem + L.wl);
     uint32_t* smask = reinterpret_cast<uint32_t*>(smem + L.mask);
     uint8_t* flag = reinterpret_cast<uint8_t*>(smem + L.flag);
+    float* hu = reinterpret_cast<float*>(smem + L.hu);           // hot channels' up dots
+    uint8_t* hrdy = reinterpret_cast<uint8_t*>(smem + L.hrdy);   // ... and whether each is in
     int* scan_sh = reinterpret_cast<int*>(smem + L.scan);
     // grid-barrier arrival counters: [0] the partials of y, [1] LoPA's stage 1
     unsigned long long* bar = reinterpret_cast<unsigned long long*>(p.tickets);
@@ -194,8 +201,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
 
     for (int i = threadIdx.x; i < p.cpb; i += kDecThreads) {
         flag[i] = 0;
+        hrdy[i] = 0;
         done[i] = 0;
         queue[i] = 0;
+    }
+    // Heavy-hitter channels of this CTA, ascending, into the (still unused)
+    // list array: one idle warp, ballots.
+    if (warp == kDecStreamWarps) {
+        int cnt = 0;
+        if (p.hot) {
+            for (int base = 0; base < nslots; base += 32) {
+                const int sl = base + lane;
+                const bool hot = sl < nslots && ((__ldg(p.hot + ((c0 + sl) >> 5)) >> ((c0 + sl) & 31)) & 1u);
+                const unsigned m = __ballot_sync(0xffffffffu, hot);
+                if (hot) wl[cnt + __popc(m & ((1u << lane) - 1u))] = sl;
+                cnt += __popc(m);
+            }
+        }
+        if (lane == 0) scan_sh[4] = cnt;
     }
     for (int i = threadIdx.x; i < p.cpb * p.mw; i += kDecThreads) smask[i] = 0u;
     if (threadIdx.x < 4) ctr[threadIdx.x] = 0;
@@ -336,6 +359,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         }
     }
 
+    // ---- heavy hitters: the two warps that are not streaming take the up dots
+    // of the CTA's hot channels at once, independent of the gate (each is
+    // used if the gate selects its channel)
+    if (!streamer) {
+        const int nhot = scan_sh[4];
+        for (int j = warp - kDecStreamWarps; j < nhot; j += kDecWarps - kDecStreamWarps) {
+            const int sl = wl[j];
+            float u[NT];
+            warp_dot_global<T, NT>(wup + (size_t)(c0 + sl) * p.d, p.d / V, xs, p.d, u);
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+                if (lane == t) hu[sl * NT + t] = u[t];
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                reinterpret_cast<volatile uint8_t*>(hrdy)[sl] = 1;
+            }
+        }
+    }
+
     // ---- up workers (all warps once their streaming is done)
     for (;;) {
         int i = 0;
@@ -365,7 +408,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         __syncwarp();
         const int k = c0 + s;
         float u[NT];
-        warp_dot_global<T, NT>(wup + (size_t)k * p.d, p.d / V, xs, p.d, u);
+        int ready = 0;
+        if (lane == 0) ready = reinterpret_cast<volatile uint8_t*>(hrdy)[s];
+        if (__shfl_sync(0xffffffffu, ready, 0)) {
+            // a heavy hitter whose up dot is in (the same dot, so the same h)
+            __threadfence_block();
+#pragma unroll
+            for (int t = 0; t < NT; ++t) u[t] = hu[s * NT + t];
+        } else {
+            warp_dot_global<T, NT>(wup + (size_t)k * p.d, p.d / V, xs, p.d, u);
+        }
         const uint32_t tokmask = smask[s * p.mw];
 #pragma unroll
         for (int t = 0; t < NT; ++t)

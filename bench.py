@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=500)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b-decode",
-                    choices=["llama7b-decode", "lopa7b", "moc-topk", "llama70b", "llama70b-lopa", "tiny"])
+                    choices=["llama7b-decode", "lopa7b", "moc-topk", "llama70b", "llama70b-lopa", "heavy7b", "tiny"])
     ap.add_argument("--sparsity", type=float, default=0.9)
     ap.add_argument("--tokens", type=int, default=0, help="batch size (0: the workload's)")
     ap.add_argument("--top-p", type=float, default=0.0,
@@ -64,6 +64,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-hot", action="store_true", help="heavy7b: run without the heavy-hitter set")
     ap.add_argument("--json-out", default="")
     return ap.parse_args()
 
@@ -79,6 +80,8 @@ def make_workload(a) -> workloads.Workload:
         wl = workloads.llama70b(1, "dense", a.sparsity)
     elif a.workload == "llama70b-lopa":
         wl = workloads.llama70b(1, "lopa", a.sparsity)
+    elif a.workload == "heavy7b":
+        wl = workloads.heavy7b()
     else:
         wl = workloads.tiny()
     if a.tokens:
@@ -334,6 +337,9 @@ def main():
     # one probe handle to measure the active union for each pool batch
     probe = sffn.SparseFFN(wl.d, wl.d_ff, wl.r, wl.n, wl.dtype, device=local)
     probe.set_weights(**weights)
+    hot = wl.hot().numpy() if wl.hot_frac > 0.0 and not a.no_hot else None
+    if hot is not None:
+        probe.set_hot(hot)
     unions = []
     for i in range(P):
         probe.forward(xs[i], gate=wl.gate, out=ys[i], **sel)
@@ -347,6 +353,8 @@ def main():
     for i in range(R):
         f = sffn.SparseFFN(wl.d, wl.d_ff, wl.r, wl.n, wl.dtype, device=local)
         f.set_weights(**weights)
+        if hot is not None:
+            f.set_hot(hot)
         ffns.append(f)
 
     stream = torch.cuda.Stream(dev)
@@ -539,7 +547,8 @@ def main():
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": wl.describe(), "tokens_per_step": wl.n, "parallelism": f"replicas x{world}",
+            "config": {"workload": wl.describe() + (" (hot set off)" if wl.hot_frac > 0.0 and hot is None else ""),
+                       "tokens_per_step": wl.n, "parallelism": f"replicas x{world}",
                        "l2": f"{R} weight replicas rotated ({R * dense_bytes(wl) / 1e9:.2f} GB > L2 "
                              f"{l2 / 2**20:.0f} MiB), no step reuses L2-resident weights",
                        "mean_union": union, "timed_with": "CUDA graphs of "

@@ -129,6 +129,24 @@ int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_
  * forward's stream.  Errors: INVALID_ARG, NOT_READY (no forward yet), CUDA. */
 int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union_size);
 
+/* Heavy-hitter channels (the heavy-hitter split, an abstract in the "FFN
+ * modules" paper listing: a few FFN neurons carry a large output for every
+ * input while the rest fire sparsely, so the FFN is split into a part for
+ * those neurons and a sparse rest).  `channels` (host, `count` entries, each
+ * in [0, d_ff), duplicates allowed, NULL when count = 0) names the hot
+ * channels; count = 0 clears the set.  With a set, the fused decode kernel
+ * (threshold selection, one or two tokens) reads every hot channel's W_up
+ * row and takes its up dot products when the forward starts, alongside the
+ * gate stream rather than after the gate has selected the channel, and uses
+ * them for the hot channels the gate selects; the other channels stay
+ * gate-first.  Selection and activation are unchanged, so y and the active
+ * lists are bitwise those of the same forward without a hot set (a hot
+ * channel the gate does not select contributes nothing); the set changes
+ * which bytes are read and when.  Other paths ignore it.  Synchronous.
+ * Errors: INVALID_ARG (count < 0, channels NULL with count > 0, a channel
+ * outside [0, d_ff)), CUDA. */
+int sffn_set_hot(sffn_handle h, const int32_t* channels, int count);
+
 /* Record timing events around each kernel of later forwards (profiling):
  * events[0] before the first launch and events[i] after launch i; at most
  * n_events events are recorded (cudaEvent_t passed as void*, created by the

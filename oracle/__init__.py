@@ -285,6 +285,28 @@ def forward(x, weights: dict, gate_mode: str, select: str, tau: float = 0.0, k: 
     return Result(z, sets, g, y, u)
 
 
+def forward_hybrid(x, weights: dict, gate_mode: str, tau: float, hot) -> Result:
+    """The heavy-hitter split with threshold selection (an abstract in the "FFN
+    modules" paper listing: a few FFN neurons carry a large output for every
+    input while the others fire sparsely, so the FFN is split into a part for
+    those neurons and a sparse rest):
+
+        y = dense FFN over the hot channels H, act = ReLU(z - tau)
+          + sparse FFN over each token's selected channels outside H.
+
+    The active sets are the threshold sets, whatever H is."""
+    z, u = gate(x, weights, gate_mode)
+    sets, g = select_threshold(z, tau)
+    d_ff = z.shape[1]
+    in_h = np.zeros(d_ff, bool)
+    in_h[np.asarray(hot, dtype=np.int64).reshape(-1)] = True
+    g_hot = np.where(in_h[None, :], np.maximum(z - float(tau), 0.0), 0.0)
+    y_hot = dense_ffn(x, weights["w_up"], weights["w_down"], g_hot)
+    rest = [s[~in_h[s]] for s in sets]
+    y_rest = sparse_ffn(x, weights["w_up"], weights["w_down"], rest, np.where(in_h[None, :], 0.0, g))
+    return Result(z, sets, g, y_hot + y_rest, u)
+
+
 def forward_on_sets(x, weights: dict, gate_mode: str, select: str, sets, tau: float = 0.0):
     """The sparse FFN with the oracle's own gate values on caller-given sets."""
     z, _ = gate(x, weights, gate_mode)

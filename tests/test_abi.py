@@ -71,6 +71,7 @@ def test_null_handles_are_rejected(pkg):
     assert pkg.sffn_check_status(None) == pkg.SFFN_ERR_INVALID_ARG
     assert pkg.sffn_last_launches(None, None) == pkg.SFFN_ERR_INVALID_ARG
     assert pkg.sffn_set_stage_events(None, None, 0) == pkg.SFFN_ERR_INVALID_ARG
+    assert pkg.sffn_set_hot(None, None, 0) == pkg.SFFN_ERR_INVALID_ARG
     assert pkg.sffn_destroy(None) == pkg.SFFN_OK
 
 

@@ -358,3 +358,60 @@ def test_thread_count_does_not_change_results():
     finally:
         oracle.set_threads(n0)
     assert np.array_equal(a.y, b.y) and np.array_equal(a.z, b.z)
+
+
+# --------------------------------------------------------------------------
+# heavy-hitter split (the heavy-hitter abstract in the "FFN modules" paper
+# listing: a dense part for the neurons that fire for every input, a sparse
+# rest)
+
+def test_hybrid_split_regroups_the_sparse_sum():
+    wl = workloads.tiny()
+    w, x = wl.weights(), wl.x()
+    sp = oracle.forward(x, w, "dense", "threshold", tau=wl.tau)
+    for frac, seed in ((0.05, 3), (0.5, 4)):
+        hot = workloads.hot_channels(wl.d_ff, frac, seed=seed).numpy()
+        hy = oracle.forward_hybrid(x, w, "dense", wl.tau, hot)
+        assert all(np.array_equal(a, b) for a, b in zip(hy.sets, sp.sets))
+        # the same terms, grouped as (hot channels, dense) + (the rest, sparse)
+        np.testing.assert_allclose(hy.y, sp.y, rtol=0, atol=1e-12 * np.abs(sp.y).max())
+        assert not np.array_equal(hy.y, oracle.forward_on_sets(
+            x, w, "dense", "threshold", [s[~np.isin(s, hot)] for s in sp.sets], tau=wl.tau))
+
+
+def test_hybrid_extremes_reduce_to_sparse_and_dense():
+    wl = workloads.tiny()
+    w, x = wl.weights(), wl.x()
+    sp = oracle.forward(x, w, "dense", "threshold", tau=wl.tau)
+    de = oracle.forward(x, w, "dense", "threshold", tau=wl.tau, dense=True)
+    assert np.array_equal(oracle.forward_hybrid(x, w, "dense", wl.tau, []).y, sp.y)
+    assert np.array_equal(oracle.forward_hybrid(x, w, "dense", wl.tau, np.arange(wl.d_ff)).y, de.y)
+
+
+def test_hybrid_lopa_gate_matches_sparse():
+    wl = workloads.lopa7b()
+    d, d_ff, r = 64, 256, 16
+    w = workloads.ffn_weights(d, d_ff, "f32", 5, "lopa", r)
+    x = workloads.tokens(3, d, "f32", 5)
+    tau = wl.tau
+    sp = oracle.forward(x, w, "lopa", "threshold", tau=tau)
+    hy = oracle.forward_hybrid(x, w, "lopa", tau, workloads.hot_channels(d_ff, 0.1, 6).numpy())
+    np.testing.assert_allclose(hy.y, sp.y, rtol=0, atol=1e-12 * np.abs(sp.y).max())
+
+
+def test_heavy_hitter_workload_structure():
+    wl = workloads.heavy7b(n=4)
+    w, x = wl.weights(), wl.x()
+    z = oracle.gate_dense(x, w["w_gate"])
+    hot = wl.hot().numpy()
+    assert len(hot) == round(0.02 * wl.d_ff)
+    # hot channels: mean tau + 3 from the outlier feature, so active almost surely
+    assert (z[:, hot] > wl.tau).mean() >= 0.99
+    # the rest: z ~ N(0, |x|^2 / d) given x, the Gaussian closed form of the active count
+    rest = np.setdiff1d(np.arange(wl.d_ff), hot)
+    xs = x.double().numpy()
+    for t in range(wl.n):
+        sig = math.sqrt(float((xs[t] ** 2).sum()) / wl.d)
+        pr = 1.0 - _phi(wl.tau / sig)
+        m = int((z[t, rest] > wl.tau).sum())
+        assert abs(m - pr * len(rest)) <= 4.0 * math.sqrt(len(rest) * pr * (1 - pr))

@@ -322,3 +322,57 @@ def test_errors(sffn):
     rc = sffn.sffn_forward(ffn.handle, buf.data_ptr() + 2, 2, 0, ctypes.byref(sel), out.data_ptr(), None)
     assert rc == sffn.SFFN_ERR_INVALID_ARG
     ffn.close()
+
+
+# --------------------------------------------------------------------------
+# heavy-hitter channels (sffn_set_hot)
+
+@pytest.mark.parametrize("n", [1, 2])
+def test_heavy_hitter_workload_matches_hybrid_oracle(sffn, n):
+    wl = workloads.heavy7b(n=n)
+    ffn, w = _ffn(sffn, wl)
+    x = wl.x()
+    hot = wl.hot().numpy()
+    y0 = ffn.forward(x.cuda(), tau=wl.tau).clone()
+    ffn.set_hot(hot)
+    y, sets, _ = check_forward(ffn, w, x, "dense", "threshold", tau=wl.tau)
+    assert ffn.last_kernel_names() == ["decode_fused"]
+    assert torch.equal(y, y0)                  # the set moves reads, not results
+    assert_y(to_np(y), oracle.forward_hybrid(x, w, "dense", wl.tau, hot).y, YTOL, "vs the hybrid oracle")
+    assert all(np.isin(hot, s).mean() >= 0.99 for s in sets)
+    ffn.set_hot([])
+    assert torch.equal(ffn.forward(x.cuda(), tau=wl.tau), y0)
+    ffn.close()
+
+
+@pytest.mark.parametrize("gate,dtype", [("dense", "bf16"), ("lopa", "bf16"), ("dense", "f32")])
+def test_hot_set_leaves_results_bitwise_unchanged(sffn, gate, dtype):
+    d, d_ff, r = 256, 2000, 64                 # d_ff not a multiple of 32: a ragged last bit word
+    w = workloads.ffn_weights(d, d_ff, dtype, seed=41, gate="both", r=r)
+    ffn = sffn.SparseFFN(d, d_ff, r, 8, dtype)
+    ffn.set_weights(**w)
+    hot = np.union1d(workloads.hot_channels(d_ff, 0.1, seed=7).numpy(), [0, 1, d_ff - 1])
+    tau = workloads.tau_for_sparsity(0.9)
+    plan = [(1, "threshold"), (2, "threshold"), (1, "topk")] + ([(8, "threshold")] if dtype == "bf16" else [])
+    for i, (n, select) in enumerate(plan):
+        x = workloads.tokens(n, d, dtype, seed=200 + i)
+        kw = dict(gate=gate, select=select, tau=tau, k=d_ff // 8)
+        ffn.set_hot([])
+        a = ffn.forward(x.cuda(), **kw).clone()
+        ffn.set_hot(hot)
+        b, _, _ = check_forward(ffn, w, x, gate, select, tau=tau, k=d_ff // 8)
+        assert torch.equal(a, b)
+        if select == "threshold":
+            assert_y(to_np(b), oracle.forward_hybrid(x, w, gate, tau, hot).y, YTOL, "vs the hybrid oracle")
+    ffn.close()
+
+
+def test_hot_set_errors(sffn):
+    ffn = sffn.SparseFFN(64, 100, 0, 1, "bf16")
+    for bad in ([100], [-1], [5, 3, 1000]):
+        with pytest.raises(sffn.SFFNError) as e:
+            ffn.set_hot(bad)
+        assert e.value.code == sffn.SFFN_ERR_INVALID_ARG
+    ffn.set_hot([0, 99, 99])                   # duplicates are fine
+    ffn.set_hot([])
+    ffn.close()

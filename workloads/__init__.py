@@ -84,6 +84,21 @@ def tokens(n: int, d: int, dtype: str = "bf16", seed: int = 0, tag: str = "") ->
     return normal((n, d), 1.0, dtype, seed, tag + f"x{n}")
 
 
+def hot_channels(d_ff: int, frac: float, seed: int = 0) -> torch.Tensor:
+    """A seeded random set of round(frac * d_ff) channels, ascending (int64)."""
+    m = int(round(frac * d_ff))
+    if m <= 0:
+        return torch.zeros(0, dtype=torch.int64)
+    g = torch.Generator().manual_seed(_seed_for(seed, "hot"))
+    return torch.sort(torch.randperm(d_ff, generator=g)[:m]).values
+
+
+def outlier_feature(d: int, seed: int = 0) -> int:
+    """The input feature that carries the heavy hitters' common large value."""
+    g = torch.Generator().manual_seed(_seed_for(seed, "outlier"))
+    return int(torch.randint(d, (1,), generator=g).item())
+
+
 @dataclass
 class Workload:
     """One of the pages' workload shapes, as a synthetic stand-in."""
@@ -101,24 +116,41 @@ class Workload:
     p: float = 0.0            # top-p budget
     seed: int = 0
     extra: dict = field(default_factory=dict)
+    hot_frac: float = 0.0     # heavy hitters: fraction of channels active for every token
+    outlier: float = 0.0      # ... driven by this value in one feature of every token
 
     def __post_init__(self):
         if self.select == "threshold" and self.tau is None:
             self.tau = tau_for_sparsity(self.sparsity)
 
     def weights(self, gate: Optional[str] = None) -> Dict[str, torch.Tensor]:
-        return ffn_weights(self.d, self.d_ff, self.dtype, self.seed, gate or self.gate, self.r)
+        w = ffn_weights(self.d, self.d_ff, self.dtype, self.seed, gate or self.gate, self.r)
+        if self.hot_frac > 0.0:
+            # the outlier feature's gate weight of a hot channel sets its mean
+            # pre-activation to tau + 3 (active with probability Phi(3))
+            if "w_gate" not in w:
+                raise ValueError("heavy hitters are defined for a dense gate")
+            w["w_gate"][outlier_feature(self.d, self.seed), self.hot()] = (self.tau + 3.0) / self.outlier
+        return w
 
     def x(self, n: Optional[int] = None, tag: str = "") -> torch.Tensor:
-        return tokens(self.n if n is None else n, self.d, self.dtype, self.seed, tag)
+        x = tokens(self.n if n is None else n, self.d, self.dtype, self.seed, tag)
+        if self.outlier:
+            x[:, outlier_feature(self.d, self.seed)] = self.outlier
+        return x
+
+    def hot(self) -> torch.Tensor:
+        """The heavy-hitter channels (ascending), empty without them."""
+        return hot_channels(self.d_ff, self.hot_frac, self.seed)
 
     def describe(self) -> str:
         sel = (f"tau={self.tau:.5f}" if self.select == "threshold" else
                f"top-p p={self.p:g}" if self.select == "topp" else f"top-k k={self.k}")
         sp = f" sparsity={self.sparsity:g}" if self.sparsity is not None else ""
         rr = f" r={self.r}" if self.gate == "lopa" else ""
+        hh = (f" heavy-hitters={len(self.hot())} outlier={self.outlier:g}" if self.hot_frac > 0.0 else "")
         return (f"{self.name}: d={self.d} d_ff={self.d_ff} n={self.n} {self.dtype} "
-                f"{self.gate}-gate{rr} {sel}{sp}")
+                f"{self.gate}-gate{rr} {sel}{sp}{hh}")
 
 
 def tiny() -> Workload:
@@ -141,6 +173,17 @@ def lopa7b(sparsity: float = 0.9, n: int = 1) -> Workload:
 def moc_topk(n: int = 16) -> Workload:
     """Mixture-of-Channels top-K: d=2048, d_ff=5632, 16 tokens, K = d_ff / 8."""
     return Workload("moc-topk", 2048, 5632, n, "bf16", "dense", "topk", k=5632 // 8)
+
+
+def heavy7b(n: int = 1, hot_frac: float = 0.02) -> Workload:
+    """Llama-7B-shaped decode whose activations have heavy hitters: every
+    token carries the value 16 in one input feature, and a fraction hot_frac
+    of the channels respond to it strongly enough to be active for every
+    token (the heavy-hitter abstract in the "FFN modules" paper listing: a
+    few neurons have a large output for any input); the rest stay about 90 %
+    sparse."""
+    return Workload("heavy7b-ffn-decode", 4096, 11008, n, "bf16", "dense", "threshold",
+                    sparsity=0.9, hot_frac=hot_frac, outlier=16.0)
 
 
 def llama70b(n: int = 1, gate: str = "dense", sparsity: float = 0.9) -> Workload:
