@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     __shared__ int sh[40];
     __shared__ uint32_t s_prefix;
     __shared__ int s_remaining;
+    __shared__ unsigned s_binw;                           // weight of the final pass's chosen bin
     __shared__ unsigned s_red[33];
     const int lane = threadIdx.x & 31;
     const size_t row = (size_t)blockIdx.x * p.d_ff;
@@ -65,7 +66,21 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     griddep_launch_dependents();
     auto make_key = [&](int k) -> uint32_t { return order_key(topp ? z[k] : silu_f(z[k])); };
     if (SMEM) {
-        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) skeys[k] = make_key(k);
+        // eight loads of z in flight per thread before the keys are made
+        constexpr int U = 8;
+        for (int k0 = threadIdx.x; k0 < p.d_ff; k0 += U * kTopkThreads) {
+            float zv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = k0 + u * kTopkThreads;
+                zv[u] = k < p.d_ff ? __ldcg(z + k) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = k0 + u * kTopkThreads;
+                if (k < p.d_ff) skeys[k] = order_key(topp ? zv[u] : silu_f(zv[u]));
+            }
+        }
         __syncthreads();
     }
     auto key_at = [&](int k) -> uint32_t { return SMEM ? skeys[k] : make_key(k); };
@@ -140,6 +155,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
             if (threadIdx.x < 256 && c > 0 && before < remaining && before + c >= remaining) {
                 s_prefix = prefix | ((uint32_t)(255 - threadIdx.x) << shift);
                 s_remaining = remaining - before;
+                s_binw = (unsigned)c;
             }
             __syncthreads();
             prefix = s_prefix;
@@ -158,22 +174,36 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     }
     // Channels tied at the boundary key: when all of them are kept (the usual
     // case) the choice needs no ranks and the writes stream in channel order.
+    // The last pass's chosen bin holds exactly the keys equal to the boundary,
+    // so its weight gives their number (top-p: every tie weighs m_tie).
     int nties = 0;
     if (partial) {
-        int c = 0;
-        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) c += key_at(k) == prefix;
-        int tot0 = 0;
-        block_exclusive_scan(c, &tot0, sh);
-        nties = tot0;
+        const unsigned m_tie = topp ? mass_of(prefix) : 1u;
+        if (m_tie) {
+            nties = (int)(s_binw / m_tie);
+        } else {
+            int c = 0;
+            for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) c += key_at(k) == prefix;
+            int tot0 = 0;
+            block_exclusive_scan(c, &tot0, sh);
+            nties = tot0;
+        }
     }
     if (!partial || nties <= take) {
-        for (int k = threadIdx.x; k < p.d_ff; k += kTopkThreads) {
-            const uint32_t key = key_at(k);
-            const float gv = topp ? silu_f(key_value(key)) : (SMEM ? key_value(key) : silu_f(z[k]));
-            const bool s = partial ? key >= prefix : (!topp && target > 0);
-            p.sel[row + k] = s ? 1 : 0;
-            p.gbuf[row + k] = s ? gv : 0.f;
-            if (s && p.ubits) atomicOr(&p.ubits[k >> 5], 1u << (k & 31));
+        // a warp covers 32 consecutive channels, one word of the union bitmap
+        const int warp = threadIdx.x >> 5;
+        for (int base = warp * 32; base < p.d_ff; base += kTopkThreads) {
+            const int k = base + lane;
+            bool s = false;
+            if (k < p.d_ff) {
+                const uint32_t key = key_at(k);
+                const float gv = topp ? silu_f(key_value(key)) : (SMEM ? key_value(key) : silu_f(z[k]));
+                s = partial ? key >= prefix : (!topp && target > 0);
+                p.sel[row + k] = s ? 1 : 0;
+                p.gbuf[row + k] = s ? gv : 0.f;
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, s);
+            if (lane == 0 && m && p.ubits) atomicOr(&p.ubits[base >> 5], m);
         }
         return;
     }
