@@ -103,7 +103,7 @@ struct sffn_ctx {
 
     void* h2 = nullptr;          // [2 npad][tc_ldh] bf16: h as hi/lo rows
     void* u2 = nullptr;          // [2 npad][r] bf16: LoPA x A as hi/lo rows
-    float* tc_part = nullptr;    // [sms][2][128][256]
+    float* tc_part = nullptr;    // [sms][2][128][256] floats: room for one parked part per CTA at any N
     unsigned* tc_tickets = nullptr;
     bool maps_ok = false;        // weight tensor maps encoded
     CUtensorMap map_wg{}, map_at{}, map_bcm{}, map_wup{}, map_wdn{};

@@ -307,8 +307,8 @@ struct alignas(64) TcParams {
     float tau;
     int topk;
     uint32_t* ubits;        // gate: union bitmap out (threshold), zeroed (top-K); up, down: read
-    float* part;            // [CTAs][2][128][nb] stream-K partial tiles
-    unsigned* tickets;      // two counters per tile (parts arrived, quarters summed), zero between launches
+    float* part;            // [CTAs][128][nb] each CTA's parked stream-K part (room for [CTAs][2][128][256])
+    unsigned* tickets;      // two counters per tile (parts arrived, owner warps done), zero between launches
     int* status;
     int stages;             // set by the launcher
     uint32_t tmem_cols;     // set by the launcher
