@@ -2,12 +2,13 @@
 //
 // Host-side orchestration only: argument checks, the device workspace plan,
 // weight repacking, and the kernel sequence of one forward:
-//   threshold, n <= 4:  [LoPA x A] -> one fused decode kernel
-//   n > 4, bf16 (tensor cores):
-//               gate GEMM (z, union bitmap) [-> top-K] -> up GEMM -> down GEMM
-//               (LoPA: x A GEMM, then the z GEMM)
-//   otherwise:  [LoPA x A] -> gate+select+up -> down, or for top-K
-//               [LoPA x A] -> gate (z) -> top-K -> preselected up -> down
+//   bf16, 3..128 tokens (or 2 where the decode kernel does not fit):
+//               gate GEMM (z, union bitmap) [-> top-K / top-p] -> up GEMM ->
+//               down GEMM on the tensor cores (LoPA: x A GEMM, then the z GEMM)
+//   threshold, 1..2 tokens (fp32: up to 4): one fused decode kernel (LoPA's
+//               x A inside it)
+//   otherwise:  [LoPA x A] -> gate+select+up -> down, or for top-K / top-p
+//               [LoPA x A] -> gate (z) -> select -> preselected up -> down
 // Every kernel is launched with programmatic dependent launch so its launch
 // latency overlaps the previous kernel's tail; each kernel waits on its
 // predecessor before touching shared buffers.

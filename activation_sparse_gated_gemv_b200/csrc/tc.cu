@@ -23,16 +23,16 @@
 // token), so the batched passes read what a per-channel gather would, in whole
 // tiles the TMA engine moves with one instruction.
 //
-// Kernel structure (one CTA per SM, 192 threads):
+// Kernel structure (one CTA per SM, 224 threads):
 //   warp 0     one thread: TMA 2-D tile copies (cp.async.bulk.tensor, 128-byte
-//              swizzle, no multicast) of the A and B tiles of each 64-wide
-//              k-block into a ring of stages on mbarriers;
+//              swizzle, no multicast) of the A and B tiles of the even 64-wide
+//              k-blocks into a ring of stages on mbarriers;
 //   warp 1     allocates tensor memory; one thread issues tcgen05.mma (M = 128,
 //              N = token columns, K = 16 per instruction, bf16 in, fp32
 //              accumulate in tensor memory) and tcgen05.commit;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
 //              lanes), the mode's epilogue, stores;
-//   warp 6     one thread: the second TMA producer (alternate k-blocks).
+//   warp 6     one thread: the second TMA producer (the odd k-blocks).
 // Work is split stream-K: the (tile, k-block) iterations are cut into one
 // contiguous range per CTA, so every SM streams the same number of weight
 // bytes.  A tile cut between CTAs is finished by the CTA holding its first
