@@ -115,7 +115,7 @@ struct sffn_ctx {
     int last_n = -1;
     cudaStream_t last_stream = nullptr;
     int last_launches = 0;
-    const char* last_names[8] = {};
+    const char* last_names[64] = {};
     std::vector<cudaEvent_t> events;
     uint32_t* hot = nullptr;     // heavy-hitter channel bits [ceil(d_ff / 32)] (kept once allocated)
     bool hot_on = false;         // a non-empty hot set is in force
@@ -154,6 +154,11 @@ StreamGeom stream_geom(const sffn_ctx* h, int n, int gate_kind) {
 
 // Stage events are recorded as external event nodes under stream capture so
 // that a replayed graph still timestamps them.
+// Name of launch i of the forward (for profiles and timing reports).
+void set_name(sffn_ctx* h, int i, const char* name) {
+    if (i < 64) h->last_names[i] = name;
+}
+
 void record(sffn_ctx* h, int i, cudaStream_t s) {
     if (i >= (int)h->events.size()) return;
     cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
@@ -208,7 +213,7 @@ int check_forward(const sffn_ctx* h, const void* x, int n, int gate_mode, const 
 // Returns SFFN_ERR_UNSUPPORTED (nothing launched) when a tensor map cannot be
 // made for this call; the caller then takes the CUDA-core path.
 int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel, void* out, cudaStream_t s,
-           bool dense, int& launches) {
+           bool dense, int& launches, int t0) {
     const sffn_config& c = h->cfg;
     const bool topk = sel->kind != SFFN_SELECT_THRESHOLD;   // a top-K or top-p mask decides
     const int npad = (int)round_up(n, 16);
@@ -232,7 +237,10 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
 
     TcParams g = base;
     g.mode = kTcGateZ;
-    g.z = h->zbuf;
+    float* zrows = h->zbuf + (size_t)t0 * c.d_ff;      // this pass's tokens' rows of the workspace
+    float* grows = h->gbuf + (size_t)t0 * c.d_ff;
+    uint8_t* srows = h->sel + (size_t)t0 * c.d_ff;
+    g.z = zrows;
     g.ldz = c.d_ff;
     g.ubits = h->ubits;
     g.m_total = c.d_ff;
@@ -243,7 +251,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
         u.m_total = c.lopa_rank; u.k_total = c.d; u.nb = npad;
         u.out = h->u2; u.ldo = c.lopa_rank;
         SFFN_CUDA(launch_tc(u, h->sms, s, true), "tensor-core x A launch");
-        h->last_names[launches] = "tc_lopa_u";
+        set_name(h, launches, "tc_lopa_u");
         record(h, ++launches, s);
         g.ta = h->map_bcm; g.tb = map_u2;
         g.k_total = c.lopa_rank; g.nb = 2 * npad; g.paired = 1;
@@ -252,17 +260,17 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
         g.k_total = c.d; g.nb = npad;
     }
     SFFN_CUDA(launch_tc(g, h->sms, s, true), "tensor-core gate launch");
-    h->last_names[launches] = "tc_gate";
+    set_name(h, launches, "tc_gate");
     record(h, ++launches, s);
 
     if (topk) {
         TopkParams tp{};
-        tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
+        tp.zbuf = zrows; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = grows; tp.sel = srows;
         tp.ubits = h->ubits;
         tp.mode = sel->kind == SFFN_SELECT_TOPP ? 1 : 0;
         tp.p = sel->p;
         SFFN_CUDA(launch_topk(tp, s, true), "top-K / top-p launch");
-        h->last_names[launches] = tp.mode ? "topp" : "topk";
+        set_name(h, launches, tp.mode ? "topp" : "topk");
         record(h, ++launches, s);
     }
 
@@ -272,9 +280,9 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     w.ubits = h->ubits; w.d_ff = c.d_ff; w.force_all = dense ? 1 : 0;
     w.m_total = c.d_ff; w.k_total = c.d; w.nb = npad;
     w.out = h->h2; w.ldo = h->tc_ldh; w.h_pairs = 1;
-    w.zsel = h->zbuf; w.gsel = h->gbuf; w.ldsel = c.d_ff;
+    w.zsel = zrows; w.gsel = grows; w.ldsel = c.d_ff;
     SFFN_CUDA(launch_tc(w, h->sms, s, true), "tensor-core up launch");
-    h->last_names[launches] = "tc_up";
+    set_name(h, launches, "tc_up");
     record(h, ++launches, s);
 
     TcParams dn = base;                         // y = sum over the active blocks of h W_down[ch]
@@ -284,7 +292,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     dn.m_total = c.d; dn.nb = 2 * npad; dn.paired = 1;
     dn.out = out; dn.ldo = c.d;
     SFFN_CUDA(launch_tc(dn, h->sms, s, true), "tensor-core down launch");
-    h->last_names[launches] = "tc_down";
+    set_name(h, launches, "tc_down");
     record(h, ++launches, s);
 
     h->last_n = n;
@@ -321,16 +329,28 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     // decode kernel from n = 3 on every shape but one); one or two: the fused
     // decode kernel, or the tensor-core path for two tokens where the decode
     // kernel's shared memory does not fit.
-    if (h->tc && n <= kTcMaxTokens && (n > kFusedMaxTokens || (n > 1 && !fused))) {
-        const int rc = run_tc(h, x, n, lopa, sel, out, s, dense, launches);
-        if (rc != SFFN_ERR_UNSUPPORTED) return rc;
+    if (h->tc && (n > kFusedMaxTokens || (n > 1 && !fused))) {
+        // More than kTcMaxTokens tokens: one tensor-core pass per block of
+        // kTcMaxTokens tokens (each pass streams the weights again, which still
+        // beats the CUDA-core path's fp32 arithmetic at such batches).
+        int rc = SFFN_OK;
+        for (int t0 = 0; t0 < n && rc == SFFN_OK; t0 += kTcMaxTokens) {
+            const int nc = n - t0 < kTcMaxTokens ? n - t0 : kTcMaxTokens;
+            rc = run_tc(h, static_cast<const char*>(x) + (size_t)t0 * c.d * h->esz, nc, lopa, sel,
+                        static_cast<char*>(out) + (size_t)t0 * c.d * h->esz, s, dense, launches, t0);
+            if (rc == SFFN_ERR_UNSUPPORTED && t0 > 0) rc = fail(SFFN_ERR_CUDA, "tensor-core pass failed mid-batch");
+        }
+        if (rc != SFFN_ERR_UNSUPPORTED) {
+            h->last_n = n;
+            return rc;
+        }
     }
 
     if (lopa && !fused) {
         LopaUParams lp{};
         lp.x = x; lp.at = h->a; lp.n = n; lp.d = c.d; lp.r = c.lopa_rank; lp.u = h->u;
         SFFN_CUDA(launch_lopa_u(c.wdtype, lp, pick_nt(n), s, pdl), "LoPA x*A launch");
-        h->last_names[launches] = "lopa_u";
+        set_name(h, launches, "lopa_u");
         record(h, ++launches, s);
     }
 
@@ -343,7 +363,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.part = h->fpart;
         dp.tickets = h->dbar; dp.y = out; dp.hot = h->hot_on ? h->hot : nullptr;
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
-        h->last_names[launches] = "decode_fused";
+        set_name(h, launches, "decode_fused");
         record(h, ++launches, s);
         h->last_n = n;
         h->last_stream = s;
@@ -368,26 +388,26 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     if (sel->kind == SFFN_SELECT_THRESHOLD) {
         gp.out = kOutSelectUp;
         SFFN_CUDA(launch_gate_stream(c.wdtype, gp, sg.nt, gk, P.g1, sg.smem, s, pdl), "gate/select/up launch");
-        h->last_names[launches] = "gate_select_up";
+        set_name(h, launches, "gate_select_up");
         record(h, ++launches, s);
     } else {
         gp.out = kOutWriteZ;
         SFFN_CUDA(launch_gate_stream(c.wdtype, gp, sg.nt, gk, P.g1, sg.smem, s, pdl), "gate launch");
-        h->last_names[launches] = "gate_z";
+        set_name(h, launches, "gate_z");
         record(h, ++launches, s);
         TopkParams tp{};
         tp.zbuf = h->zbuf; tp.n = n; tp.d_ff = c.d_ff; tp.k = sel->k; tp.gbuf = h->gbuf; tp.sel = h->sel;
         tp.mode = sel->kind == SFFN_SELECT_TOPP ? 1 : 0;
         tp.p = sel->p;
         SFFN_CUDA(launch_topk(tp, s, pdl), "top-K / top-p launch");
-        h->last_names[launches] = tp.mode ? "topp" : "topk";
+        set_name(h, launches, tp.mode ? "topp" : "topk");
         record(h, ++launches, s);
         gp.out = kOutSelectUp;
         const int nt = presel_nt(h, n);
         SFFN_CUDA(launch_gate(c.wdtype, gp, nt, 1, kGatePreselected, P.g1,
                               gate_smem_bytes(c.wdtype, nt, c.d, 0, kGatePreselected, P.cpb, P.mw), s, pdl),
                   "selected up launch");
-        h->last_names[launches] = "preselected_up";
+        set_name(h, launches, "preselected_up");
         record(h, ++launches, s);
     }
 
@@ -402,7 +422,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     const int nseg = (P.g1 + P.down_chunks - 1) / P.down_chunks;
     SFFN_CUDA(launch_down(c.wdtype, dp, dnt, P.down_slices, down_smem_bytes(c.wdtype, dnt, nseg, P.cpb), s, pdl),
               "down launch");
-    h->last_names[launches] = "down";
+    set_name(h, launches, "down");
     record(h, ++launches, s);
 
     h->last_n = n;
@@ -764,7 +784,7 @@ int sffn_last_launches(sffn_handle h, int32_t* launches) {
 }
 
 const char* sffn_last_kernel_name(sffn_handle h, int i) {
-    if (!h || i < 0 || i >= h->last_launches || i >= 8 || !h->last_names[i]) return "";
+    if (!h || i < 0 || i >= h->last_launches || i >= 64 || !h->last_names[i]) return "";
     return h->last_names[i];
 }
 

@@ -430,9 +430,15 @@ def main():
             per_kernel[i] += evs[i].elapsed_time(evs[i + 1])
     per_kernel /= K2
     kernel_names = ffns[0].last_kernel_names()
-    dominant = int(np.argmax(per_kernel))
+    # launches of the same kernel (a batch above 128 tokens takes one
+    # tensor-core pass per 128 tokens) are counted together
+    names = [kernel_names[i] if i < len(kernel_names) else f"k{i}" for i in range(launches)]
+    per_name = {}
+    for i, nm in enumerate(names):
+        per_name[nm] = per_name.get(nm, 0.0) + per_kernel[i]
+    launch_count = {nm: names.count(nm) for nm in per_name}
+    dom_name = max(per_name, key=per_name.get)
     peaks, peak_kind = measured_peaks()
-    dom_name = kernel_names[dominant] if dominant < len(kernel_names) else f"k{dominant}"
     w = bytes_per_elem(wl.dtype)
     if dom_name == "decode_fused":
         # everything (LoPA's stage 1 runs inside the same launch)
@@ -463,8 +469,9 @@ def main():
     # without its overlap with its neighbours.  The steady-state launch time
     # is the timed region's time per step apportioned by those shares; for a
     # one-kernel step it is exactly the timed region divided by the steps.
-    share = per_kernel / per_kernel.sum()
-    avg_launch_ms = ms_per_step * share[dominant]
+    total = sum(per_name.values())
+    share = {nm: v / total for nm, v in per_name.items()}
+    avg_launch_ms = ms_per_step * share[dom_name]
     achieved = dom_bytes / (avg_launch_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom_name, "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
@@ -474,10 +481,11 @@ def main():
                 "avg_launch_us": round(avg_launch_ms * 1e3, 3),
                 "kernel_timing": (f"timed region per step x the kernel's share of the step; shares from "
                                   f"CUDA events around each kernel over {K2} steps replayed from a graph"),
-                "share": {kernel_names[i] if i < len(kernel_names) else f"k{i}":
-                          round(float(share[i]), 4) for i in range(launches)},
-                "isolated_launch_us": {kernel_names[i] if i < len(kernel_names) else f"k{i}":
-                                       round(per_kernel[i] * 1e3, 3) for i in range(launches)}}
+                "share": {nm: round(float(v), 4) for nm, v in share.items()},
+                "isolated_launch_us": {nm: round(v * 1e3, 3) for nm, v in per_name.items()}}
+    if any(c > 1 for c in launch_count.values()):
+        roofline["launches_per_step"] = launch_count
+        roofline["kernel_timing"] += "; a kernel launched several times per step counts all its launches"
     step_gbs = fwd_bytes / (ms_per_step * 1e-3) / 1e9
 
     # -- dense FFN on the same weights (the library's dense path)

@@ -376,3 +376,34 @@ def test_hot_set_errors(sffn):
     ffn.set_hot([0, 99, 99])                   # duplicates are fine
     ffn.set_hot([])
     ffn.close()
+
+
+# --------------------------------------------------------------------------
+# batches above 128 tokens: one tensor-core pass per 128 tokens
+
+@pytest.mark.parametrize("gate,select", [("dense", "threshold"), ("lopa", "threshold"), ("dense", "topk"),
+                                         ("lopa", "topp")])
+def test_batch_above_128_tokens_in_passes(sffn, gate, select):
+    d, d_ff, r, n = 256, 2000, 64, 300         # passes of 128, 128 and 44 tokens
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=51, gate="both", r=r)
+    ffn = sffn.SparseFFN(d, d_ff, r, n, "bf16")
+    ffn.set_weights(**w)
+    x = workloads.tokens(n, d, "bf16", seed=52)
+    tau, k = workloads.tau_for_sparsity(0.9), d_ff // 8
+    edges = [0, 1, 127, 128, 129, 255, 256, 257, 299]
+    check_forward(ffn, w, x, gate, select, tau=tau, k=k, p=0.7, tokens=edges)
+    assert ffn.last_kernel_names().count("tc_gate") == 3
+    ffn.close()
+
+
+def test_dense_ffn_above_128_tokens(sffn):
+    d, d_ff, n = 256, 1024, 200
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=53)
+    ffn = sffn.SparseFFN(d, d_ff, 0, n, "bf16")
+    ffn.set_weights(**w)
+    x = workloads.tokens(n, d, "bf16", seed=54)
+    tau = workloads.tau_for_sparsity(0.9)
+    yd, _, _ = check_forward(ffn, w, x, "dense", "threshold", tau=tau, dense=True, tokens=[0, 127, 128, 199])
+    ys = ffn.forward(x.cuda(), tau=tau)
+    assert_y(to_np(ys), to_np(yd), YTOL, "sparse vs dense")
+    ffn.close()
