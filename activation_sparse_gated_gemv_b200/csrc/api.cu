@@ -2,9 +2,10 @@
 //
 // Host-side orchestration only: argument checks, the device workspace plan,
 // weight repacking, and the kernel sequence of one forward:
-//   bf16, 3..128 tokens (or 2 where the decode kernel does not fit):
+//   bf16, 3 tokens and more (or 2 where the decode kernel does not fit):
 //               gate GEMM (z, union bitmap) [-> top-K / top-p] -> up GEMM ->
-//               down GEMM on the tensor cores (LoPA: x A GEMM, then the z GEMM)
+//               down GEMM on the tensor cores (LoPA: x A GEMM, then the z GEMM),
+//               one pass per 128 tokens
 //   threshold, 1..2 tokens (fp32: up to 4): one fused decode kernel (LoPA's
 //               x A inside it)
 //   otherwise:  [LoPA x A] -> gate+select+up -> down, or for top-K / top-p
