@@ -71,3 +71,22 @@ def test_reference_arm_prints_only_on_rank_zero(tmp_path):
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_traffic_is_reported_only_for_the_current_kernel_sources(tmp_path, monkeypatch):
+    """A committed ncu traffic figure is used only while the kernel sources
+    still hash to the value it was captured on; otherwise the bench reports null."""
+    sys.path.insert(0, ROOT)
+    import bench
+    (tmp_path / "profiles").mkdir()
+    ent = {"dram_bytes_per_launch": 123, "kernel_hash": bench.kernel_hash()}
+    data = {"llama7b-decode": {"decode_fused": ent},
+            "llama70b:n16": {"tc_up": dict(ent, dram_bytes_per_launch=456)}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(data))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("decode_fused", "llama7b-decode", 1) == 123
+    assert bench.traffic_for("tc_up", "llama70b", 16) == 456
+    assert bench.traffic_for("tc_up", "llama70b", 64) is None
+    data["llama7b-decode"]["decode_fused"]["kernel_hash"] = "0" * 16
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(data))
+    assert bench.traffic_for("decode_fused", "llama7b-decode", 1) is None
