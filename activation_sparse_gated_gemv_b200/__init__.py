@@ -41,6 +41,7 @@ SFFN_ERR_DEVICE_CHECK = 7
 SFFN_BF16, SFFN_F32 = 0, 1
 SFFN_GATE_DENSE, SFFN_GATE_LOPA = 0, 1
 SFFN_SELECT_THRESHOLD, SFFN_SELECT_TOPK, SFFN_SELECT_TOPP = 0, 1, 2
+SFFN_INJECT_WAIT_TIMEOUT, SFFN_INJECT_BAD_LIST_ENTRY = 1, 2
 
 
 class sffn_config(ctypes.Structure):
@@ -52,10 +53,11 @@ class sffn_select(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("tau", ctypes.c_float), ("k", ctypes.c_int32), ("p", ctypes.c_float)]
 
 
-if not os.path.exists(LIB_PATH):
-    # a fresh checkout: compile the library in-tree first (nvcc, sm_100a); if
-    # that fails the import fails with it
-    from . import build as _build
+from . import build as _build  # noqa: E402
+
+if not _build.up_to_date():
+    # a fresh checkout, or sources newer than the library: compile it in-tree
+    # first (nvcc, sm_100a); if that fails the import fails with it
     _build.build()
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -76,6 +78,9 @@ _sigs = {
     "sffn_forward_noalloc": ([_P, _P, _P, _I, _I, _I, _P, _I, ctypes.c_float, _P, _P], _I),
     "sffn_last_kernel_name": ([_P, _I], ctypes.c_char_p),
     "sffn_set_hot": ([_P, _P, _I], _I),
+    "sffn_get_union": ([_P, _P, _I], _I),
+    "sffn_debug_inject": ([_P, _I, ctypes.c_longlong], _I),
+    "sffn_noalloc_check_status": ([], _I),
 }
 for _name, (_args, _res) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -98,6 +103,9 @@ sffn_last_error = _lib.sffn_last_error
 sffn_forward_noalloc = _lib.sffn_forward_noalloc
 sffn_last_kernel_name = _lib.sffn_last_kernel_name
 sffn_set_hot = _lib.sffn_set_hot
+sffn_get_union = _lib.sffn_get_union
+sffn_debug_inject = _lib.sffn_debug_inject
+sffn_noalloc_check_status = _lib.sffn_noalloc_check_status
 
 EXPORTED = tuple(_sigs)
 
@@ -209,6 +217,18 @@ class SparseFFN:
         check(sffn_get_active(self._h, idx.ctypes.data_as(ctypes.c_void_p),
                               cnt.ctypes.data_as(ctypes.c_void_p), ctypes.byref(uni)), "sffn_get_active")
         return [idx[t, :cnt[t]].copy() for t in range(n)], int(uni.value)
+
+    def union_bits(self) -> np.ndarray:
+        """The union bitmap (uint32 words, bit k = channel k) the last
+        tensor-core forward's up and down kernels read their active blocks from."""
+        words = (self.d_ff + 31) // 32
+        bits = np.zeros(words, np.uint32)
+        check(sffn_get_union(self._h, bits.ctypes.data_as(ctypes.c_void_p), words), "sffn_get_union")
+        return bits
+
+    def debug_inject(self, what: int, arg: int = 0) -> None:
+        """Arm a one-shot host-side failure injection (SFFN_INJECT_*)."""
+        check(sffn_debug_inject(self._h, int(what), int(arg)), "sffn_debug_inject")
 
     def set_hot(self, channels) -> None:
         """Heavy-hitter channels (any int sequence; empty clears the set): the

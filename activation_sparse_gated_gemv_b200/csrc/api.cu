@@ -16,6 +16,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -62,6 +63,35 @@ struct DeviceGuard {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Host-side fault injection for the error paths of sffn_create and
+// sffn_set_weights.  The environment variable SFFN_FAULT = "alloc:N" or
+// "copy:N" makes the N-th device allocation (cudaMalloc, cudaHostAlloc) or
+// the N-th host-to-device copy of one such call report failure (out of
+// memory, or a CUDA error) without touching the device; unset, it costs one
+// getenv per call.
+struct HostFaults {
+    int alloc_at = 0, copy_at = 0, allocs = 0, copies = 0;
+    HostFaults() {
+        const char* f = std::getenv("SFFN_FAULT");
+        if (!f) return;
+        int n = 0;
+        if (std::sscanf(f, "alloc:%d", &n) == 1) alloc_at = n;
+        else if (std::sscanf(f, "copy:%d", &n) == 1) copy_at = n;
+    }
+    cudaError_t malloc_dev(void** p, size_t bytes) {
+        if (alloc_at > 0 && ++allocs == alloc_at) return cudaErrorMemoryAllocation;
+        return cudaMalloc(p, bytes);
+    }
+    cudaError_t malloc_host_mapped(void** p, size_t bytes) {
+        if (alloc_at > 0 && ++allocs == alloc_at) return cudaErrorMemoryAllocation;
+        return cudaHostAlloc(p, bytes, cudaHostAllocMapped);
+    }
+    cudaError_t copy(void* dst, const void* src, size_t bytes, cudaMemcpyKind kind, cudaStream_t s) {
+        if (copy_at > 0 && ++copies == copy_at) return cudaErrorInvalidValue;
+        return cudaMemcpyAsync(dst, src, bytes, kind, s);
+    }
+};
+
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Plan {
@@ -95,6 +125,8 @@ struct sffn_ctx {
     unsigned* tickets = nullptr;
     unsigned* dbar = nullptr;    // fused decode: grid-barrier arrival counters
     int* status = nullptr;
+    int* hstat = nullptr;        // host-mapped mirror of the status word (host address)
+    int* hstat_dev = nullptr;    // ... and its device address, given to the kernels
     void* xdev = nullptr;
     void* ydev = nullptr;
     // tensor-core batched path (bf16 handles with max_tokens > 1)
@@ -102,6 +134,8 @@ struct sffn_ctx {
     int tc_npad_max = 0;
     long long tc_ldh = 0;
     uint32_t* ubits = nullptr;
+    uint32_t* selbits = nullptr; // [max_tokens][ceil(d_ff / 32)] per-token selection bits of the tensor-core gate
+    int selw = 0;
 
     void* h2 = nullptr;          // [2 npad][tc_ldh] bf16: h as hi/lo rows
     void* u2 = nullptr;          // [2 npad][r] bf16: LoPA x A as hi/lo rows
@@ -120,6 +154,9 @@ struct sffn_ctx {
     std::vector<cudaEvent_t> events;
     uint32_t* hot = nullptr;     // heavy-hitter channel bits [ceil(d_ff / 32)] (kept once allocated)
     bool hot_on = false;         // a non-empty hot set is in force
+    // one-shot injections for the failure tests (sffn_debug_inject)
+    unsigned long long inj_wait_ns = 0;   // next fused decode: this wait limit, and a barrier no one completes
+    bool inj_bad_index = false;           // next unfused forward: a bad list entry before the down kernel
 };
 
 namespace {
@@ -169,6 +206,21 @@ void record(sffn_ctx* h, int i, cudaStream_t s) {
         cudaEventRecord(h->events[i], s);
 }
 
+// The status word's bits as a return code: a failed bounds check before a
+// timed-out wait.
+int status_code(int st) {
+    if (st & kStatusBounds) return fail(SFFN_ERR_DEVICE_CHECK, "a kernel's bounds check failed (status 0x%x)", st);
+    if (st & kStatusWaitTimeout) return fail(SFFN_ERR_TIMEOUT, "a bounded device wait timed out (status 0x%x)", st);
+    if (st) return fail(SFFN_ERR_DEVICE_CHECK, "device status word 0x%x", st);
+    return SFFN_OK;
+}
+
+// The host-mapped mirror of the status word, read without synchronising: set
+// once a kernel of an earlier forward that has finished raised a bit.
+int mirrored_status(const sffn_ctx* h) {
+    return h->hstat ? *reinterpret_cast<volatile const int*>(h->hstat) : 0;
+}
+
 int check_select(const sffn_ctx* h, const sffn_select* sel) {
     if (!sel) return fail(SFFN_ERR_INVALID_ARG, "sel is NULL");
     if (sel->kind == SFFN_SELECT_THRESHOLD) {
@@ -189,6 +241,7 @@ int check_select(const sffn_ctx* h, const sffn_select* sel) {
 int check_forward(const sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_select* sel,
                   const void* out, bool device_ptrs) {
     if (!h) return fail(SFFN_ERR_INVALID_ARG, "handle is NULL");
+    if (const int st = mirrored_status(h)) return status_code(st);
     if (n < 0 || n > h->cfg.max_tokens)
         return fail(SFFN_ERR_INVALID_ARG, "n_tokens=%d outside [0, max_tokens=%d]", n, h->cfg.max_tokens);
     if (gate_mode != SFFN_GATE_DENSE && gate_mode != SFFN_GATE_LOPA)
@@ -235,6 +288,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     base.part = h->tc_part;
     base.tickets = h->tc_tickets;
     base.status = h->status;
+    base.hstatus = h->hstat_dev;
 
     TcParams g = base;
     g.mode = kTcGateZ;
@@ -244,6 +298,8 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     g.z = zrows;
     g.ldz = c.d_ff;
     g.ubits = h->ubits;
+    g.selbits = topk ? nullptr : h->selbits + (size_t)t0 * h->selw;
+    g.selw = h->selw;
     g.m_total = c.d_ff;
     if (lopa) {
         TcParams u = base;                      // u = x A, as hi/lo bf16 rows
@@ -361,7 +417,10 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         dp.wg = h->wg; dp.bcm = h->bcm; dp.at = h->a; dp.u = h->u; dp.wup = h->wup; dp.wdn = h->wdn;
         dp.tau = sel->tau; dp.cpb = P.cpb; dp.mw = P.mw;
         dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
-        dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.part = h->fpart;
+        dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.hstatus = h->hstat_dev; dp.part = h->fpart;
+        dp.wait_ns = h->inj_wait_ns ? h->inj_wait_ns : kWaitLimitNs;
+        dp.bar_extra = h->inj_wait_ns ? 1 : 0;
+        h->inj_wait_ns = 0;
         dp.tickets = h->dbar; dp.y = out; dp.hot = h->hot_on ? h->hot : nullptr;
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
         set_name(h, launches, "decode_fused");
@@ -386,6 +445,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     gp.sb = sg.sb;
     gp.nb = sg.nb;
     gp.status = h->status;
+    gp.hstatus = h->hstat_dev;
     if (sel->kind == SFFN_SELECT_THRESHOLD) {
         gp.out = kOutSelectUp;
         SFFN_CUDA(launch_gate_stream(c.wdtype, gp, sg.nt, gk, P.g1, sg.smem, s, pdl), "gate/select/up launch");
@@ -419,6 +479,18 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     dp.tickets = h->tickets; dp.y = out;
     dp.chunks = P.down_chunks;
     dp.status = h->status;
+    dp.hstatus = h->hstat_dev;
+    if (h->inj_bad_index) {
+        // failure test: a list entry outside its segment and a count beyond its
+        // segment's slots, written by the host between the gate and the down
+        // kernel; the down kernel's checks must catch both
+        h->inj_bad_index = false;
+        const int bad_idx = c.d_ff + 7, bad_cnt = P.cpb + 5;
+        SFFN_CUDA(cudaMemcpyAsync(h->lst_idx, &bad_idx, sizeof bad_idx, cudaMemcpyHostToDevice, s), "inject");
+        if (P.g1 > 1)
+            SFFN_CUDA(cudaMemcpyAsync(h->seg_count + 1, &bad_cnt, sizeof bad_cnt, cudaMemcpyHostToDevice, s),
+                      "inject");
+    }
     const int dnt = pick_nt(n);
     const int nseg = (P.g1 + P.down_chunks - 1) / P.down_chunks;
     SFFN_CUDA(launch_down(c.wdtype, dp, dnt, P.down_slices, down_smem_bytes(c.wdtype, dnt, nseg, P.cpb), s, pdl),
@@ -486,6 +558,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     if (c.device < 0 || c.device >= ndev) return fail(SFFN_ERR_INVALID_ARG, "no CUDA device %d", c.device);
     DeviceGuard g(c.device);
     if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    HostFaults faults;
 
     sffn_ctx* h = new (std::nothrow) sffn_ctx();
     if (!h) return fail(SFFN_ERR_OOM, "host allocation failed");
@@ -523,11 +596,28 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t FDR = F > D ? (F > R ? F : R) : (D > R ? D : R);
     const size_t tiles = round_up(FDR, 128) / 128 + 1;
     const size_t o_ub = take(h->tc ? tiles * 4 * 4 : 0);
+    h->selw = (int)((F + 31) / 32);
+    const size_t o_sb = take(h->tc ? T * (size_t)h->selw * 4 : 0);
     const size_t o_h2 = take(2 * NP * (size_t)h->tc_ldh * 2), o_u2 = take(2 * NP * R * 2);
     // stream-K partial tiles: two slots per CTA of up to 256 accumulator columns x 128 rows
     const size_t o_tp = take(h->tc ? (size_t)h->sms * 2 * 256 * 128 * 4 : 0), o_tt = take(h->tc ? tiles * 8 : 0);
-    e = cudaMalloc(&h->ws, off);
+    e = faults.malloc_dev(&h->ws, off);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "workspace allocation"); }
+    void* hs = nullptr;
+    e = faults.malloc_host_mapped(&hs, 64);
+    if (e == cudaSuccess) {
+        h->hstat = static_cast<int*>(hs);
+        *h->hstat = 0;
+        void* hd = nullptr;
+        e = cudaHostGetDevicePointer(&hd, hs, 0);
+        h->hstat_dev = static_cast<int*>(hd);
+    }
+    if (e != cudaSuccess) {
+        if (h->hstat) cudaFreeHost(h->hstat);
+        cudaFree(h->ws);
+        delete h;
+        return cuda_fail(e, "status mirror allocation");
+    }
     char* b = static_cast<char*>(h->ws);
     h->zbuf = reinterpret_cast<float*>(b + o_z);
     h->gbuf = reinterpret_cast<float*>(b + o_g);
@@ -546,6 +636,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->ydev = b + o_y;
     if (h->tc) {
         h->ubits = reinterpret_cast<uint32_t*>(b + o_ub);
+        h->selbits = reinterpret_cast<uint32_t*>(b + o_sb);
         h->h2 = b + o_h2;
         h->u2 = b + o_u2;
         h->tc_part = reinterpret_cast<float*>(b + o_tp);
@@ -553,7 +644,12 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     }
     e = cudaMemset(h->ws, 0, off);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(e, "workspace init"); }
+    if (e != cudaSuccess) {
+        cudaFreeHost(h->hstat);
+        cudaFree(h->ws);
+        delete h;
+        return cuda_fail(e, "workspace init");
+    }
     *out = h;
     return SFFN_OK;
 }
@@ -574,6 +670,7 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     SFFN_CUDA(cudaStreamSynchronize(s), "stream synchronize");
     free_weights(h);
+    HostFaults faults;
 
     const size_t big = (size_t)c.d * c.d_ff * h->esz;
     const size_t r_d = (size_t)c.lopa_rank * c.d * h->esz, r_ff = (size_t)c.lopa_rank * c.d_ff * h->esz;
@@ -581,26 +678,31 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
     int rc = SFFN_OK;
     auto stage = [&](const void* src, size_t bytes) -> const void* {
         if (src_is_device) return src;
-        if (cudaMemcpyAsync(staging, src, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return nullptr;
+        if (faults.copy(staging, src, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return nullptr;
         return staging;
     };
-    auto alloc = [&](void** p, size_t bytes) { return cudaMalloc(p, bytes); };
+    auto alloc = [&](void** p, size_t bytes) { return faults.malloc_dev(p, bytes); };
     cudaError_t e = cudaSuccess;
+    // a failed staging copy: the runtime's error, or the injected one
+    auto copy_error = [&]() {
+        const cudaError_t le = cudaGetLastError();
+        return le != cudaSuccess ? le : cudaErrorInvalidValue;
+    };
     do {
         if (!src_is_device && (e = alloc(&staging, big > r_ff ? big : r_ff)) != cudaSuccess) break;
         if ((e = alloc(&h->wup, big)) != cudaSuccess) break;
         if ((e = alloc(&h->wdn, big)) != cudaSuccess) break;
         const void* src = stage(w_up, big);
-        if (!src) { e = cudaGetLastError(); break; }
+        if (!src) { e = copy_error(); break; }
         if ((e = launch_transpose(c.wdtype, src, h->wup, c.d, c.d_ff, s)) != cudaSuccess) break;
         if ((e = cudaStreamSynchronize(s)) != cudaSuccess) break;
-        if ((e = cudaMemcpyAsync(h->wdn, w_down, big, src_is_device ? cudaMemcpyDeviceToDevice
-                                                                     : cudaMemcpyHostToDevice, s)) != cudaSuccess)
+        if ((e = faults.copy(h->wdn, w_down, big, src_is_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice,
+                             s)) != cudaSuccess)
             break;
         if (w_gate) {
             if ((e = alloc(&h->wg, big)) != cudaSuccess) break;
             src = stage(w_gate, big);
-            if (!src) { e = cudaGetLastError(); break; }
+            if (!src) { e = copy_error(); break; }
             if ((e = launch_transpose(c.wdtype, src, h->wg, c.d, c.d_ff, s)) != cudaSuccess) break;
             if ((e = cudaStreamSynchronize(s)) != cudaSuccess) break;
         }
@@ -608,11 +710,11 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
             if ((e = alloc(&h->a, r_d)) != cudaSuccess) break;
             if ((e = alloc(&h->bcm, r_ff)) != cudaSuccess) break;
             src = stage(A, r_d);
-            if (!src) { e = cudaGetLastError(); break; }
+            if (!src) { e = copy_error(); break; }
             if ((e = launch_transpose(c.wdtype, src, h->a, c.d, c.lopa_rank, s)) != cudaSuccess) break;
             if ((e = cudaStreamSynchronize(s)) != cudaSuccess) break;
             src = stage(B, r_ff);
-            if (!src) { e = cudaGetLastError(); break; }
+            if (!src) { e = copy_error(); break; }
             if ((e = launch_transpose(c.wdtype, src, h->bcm, c.lopa_rank, c.d_ff, s)) != cudaSuccess) break;
         }
         e = cudaStreamSynchronize(s);
@@ -675,8 +777,7 @@ int sffn_check_status(sffn_handle h) {
     SFFN_CUDA(cudaDeviceSynchronize(), "device synchronize");
     int st = 0;
     SFFN_CUDA(cudaMemcpy(&st, h->status, sizeof st, cudaMemcpyDeviceToHost), "status read");
-    if (st) return fail(SFFN_ERR_DEVICE_CHECK, "device status word 0x%x", st);
-    return SFFN_OK;
+    return status_code(st);
 }
 
 int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union_size) {
@@ -706,14 +807,21 @@ int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union
                         any[k] = 1;
                     }
         } else {
-            std::vector<float> z((size_t)n * F);
-            SFFN_CUDA(cudaMemcpy(z.data(), h->zbuf, z.size() * 4, cudaMemcpyDeviceToHost), "gate copy");
+            // the gate kernel's own per-token selection bits
+            const int W = h->selw;
+            std::vector<uint32_t> bits((size_t)n * W);
+            SFFN_CUDA(cudaMemcpy(bits.data(), h->selbits, bits.size() * 4, cudaMemcpyDeviceToHost), "selection copy");
             for (int t = 0; t < n; ++t)
                 for (int k = 0; k < F; ++k)
-                    if (z[(size_t)t * F + k] > h->last_tau) {
+                    if ((bits[(size_t)t * W + (k >> 5)] >> (k & 31)) & 1u) {
                         idx[(size_t)t * F + counts[t]++] = k;
                         any[k] = 1;
                     }
+            // bits past d_ff in the last word must be clear
+            if (F & 31)
+                for (int t = 0; t < n; ++t)
+                    if (bits[(size_t)t * W + W - 1] >> (F & 31))
+                        return fail(SFFN_ERR_DEVICE_CHECK, "selection bit past d_ff for token %d", t);
         }
         int uni = 0;
         for (int k = 0; k < F; ++k) uni += any[k];
@@ -742,6 +850,38 @@ int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union
     }
     if (union_size) *union_size = uni;
     return SFFN_OK;
+}
+
+int sffn_get_union(sffn_handle h, uint32_t* bits, int nwords) {
+    if (!h || !bits) return fail(SFFN_ERR_INVALID_ARG, "handle or bits is NULL");
+    const int W = (h->cfg.d_ff + 31) / 32;
+    if (nwords < W) return fail(SFFN_ERR_INVALID_ARG, "nwords=%d < ceil(d_ff / 32)=%d", nwords, W);
+    if (h->last_n < 0) return fail(SFFN_ERR_NOT_READY, "no forward has run");
+    if (!h->last_tc) return fail(SFFN_ERR_UNSUPPORTED, "the last forward did not take the tensor-core path");
+    DeviceGuard g(h->cfg.device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    SFFN_CUDA(cudaStreamSynchronize(h->last_stream), "stream synchronize");
+    const int rc = sffn_check_status(h);
+    if (rc) return rc;
+    SFFN_CUDA(cudaMemcpy(bits, h->ubits, (size_t)W * 4, cudaMemcpyDeviceToHost), "union copy");
+    for (int w = W; w < nwords; ++w) bits[w] = 0u;
+    return SFFN_OK;
+}
+
+int sffn_debug_inject(sffn_handle h, int what, long long arg) {
+    if (!h) return fail(SFFN_ERR_INVALID_ARG, "handle is NULL");
+    switch (what) {
+        case SFFN_INJECT_WAIT_TIMEOUT:
+            if (arg < 1000 || arg > 2000000000LL)
+                return fail(SFFN_ERR_INVALID_ARG, "wait limit %lld ns outside [1 us, 2 s]", arg);
+            h->inj_wait_ns = (unsigned long long)arg;
+            return SFFN_OK;
+        case SFFN_INJECT_BAD_LIST_ENTRY:
+            h->inj_bad_index = true;
+            return SFFN_OK;
+        default:
+            return fail(SFFN_ERR_INVALID_ARG, "unknown injection %d", what);
+    }
 }
 
 int sffn_set_hot(sffn_handle h, const int32_t* channels, int count) {
@@ -796,6 +936,7 @@ int sffn_destroy(sffn_handle h) {
         free_weights(h);
         if (h->ws) cudaFree(h->ws);
         if (h->hot) cudaFree(h->hot);
+        if (h->hstat) cudaFreeHost(h->hstat);
     }
     delete h;
     return SFFN_OK;

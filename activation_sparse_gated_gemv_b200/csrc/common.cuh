@@ -222,6 +222,7 @@ struct GateParams {
     int sb;                 // streamed piece bytes (multiple of 16)
     int nb;                 // pieces in flight per warp
     int* status;            // sticky device status word
+    int* hstatus;           // its host-mapped mirror, or NULL
 };
 
 struct LopaUParams {
@@ -253,6 +254,7 @@ struct DownParams {
     void* y;                // [n][d] T
     int chunks;             // chunk CTAs per column slice (grid.y), each a run of gate segments
     int* status;            // sticky device status word (bit set on a failed check)
+    int* hstatus;           // its host-mapped mirror, or NULL
 };
 
 struct DecodeParams {
@@ -272,6 +274,9 @@ struct DecodeParams {
     int* seg_count;         // [CTAs]
     int sb, nb;             // streamed piece bytes, pieces in flight per streaming warp
     int* status;
+    int* hstatus;           // host-mapped mirror of the status word, or NULL
+    unsigned long long wait_ns;   // limit of the grid-barrier waits
+    int bar_extra;          // arrivals the final grid barrier expects beyond the grid (0; 1 makes it time out)
     float* part;            // [CTAs][n][d] per-CTA partials of y
     unsigned* tickets;      // two 64-bit grid-barrier arrival counters (8-byte aligned), zero at creation
     void* y;                // [n][d] T
@@ -307,16 +312,31 @@ struct alignas(64) TcParams {
     float tau;
     int topk;
     uint32_t* ubits;        // gate: union bitmap out (threshold), zeroed (top-K); up, down: read
+    uint32_t* selbits;      // gate, threshold: per-token selection bits [n][selw] (bit k: z[t,k] > tau), or NULL
+    int selw;               // words per token row of selbits (ceil(d_ff / 32))
     float* part;            // [CTAs][128][nb] each CTA's parked stream-K part (room for [CTAs][2][128][256])
     unsigned* tickets;      // two counters per tile (parts arrived, owner warps done), zero between launches
     int* status;
+    int* hstatus;           // host-mapped mirror of the status word, or NULL
     int stages;             // set by the launcher
     uint32_t tmem_cols;     // set by the launcher
 };
 
 
-// Bits of the device status word.
-enum StatusBits { kStatusWaitTimeout = 2 };
+// Bits of the device status word: a bounded wait gave up, or a kernel's own
+// bounds check rejected an index or a count written by an earlier kernel (the
+// access was skipped).
+enum StatusBits { kStatusWaitTimeout = 2, kStatusBounds = 4 };
+
+// Set `bits` in the sticky device status word `st`, and copy the word into the
+// handle's host-mapped mirror `hst` (NULL: none) with a plain system-scope
+// store, so the host sees the failure on its next call without synchronising.
+// Racing raisers may leave the mirror short of a bit; it is never zero after a
+// raise, and the device word keeps every bit.
+__device__ __forceinline__ void raise_status(int* st, int* hst, int bits) {
+    const int old = st ? atomicOr(st, bits) : 0;
+    if (hst) asm volatile("st.relaxed.sys.global.b32 [%0], %1;" ::"l"(hst), "r"(old | bits) : "memory");
+}
 
 // Raise a kernel's dynamic shared-memory limit once per device (so a forward
 // inside stream capture issues launches only).  `cache` is per kernel.
@@ -335,20 +355,31 @@ inline cudaError_t ensure_smem(K kernel, size_t smem, SmemAttrCache& cache) {
     return e;
 }
 
-// Launch with programmatic dependent launch (PDL) when `pdl` is set.
+// Launch with programmatic dependent launch (PDL) when `pdl` is set.  A
+// `cooperative` launch is one whose CTAs meet at grid-wide barriers: the
+// runtime then refuses a grid that cannot have all its CTAs resident at once.
 template <class K, class P>
 inline cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
-                             const P& params) {
+                             const P& params, bool cooperative = false) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = pdl ? attr : nullptr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (cooperative) {
+        attr[na].id = cudaLaunchAttributeCooperative;
+        attr[na].val.cooperative = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kernel, params);
 }
 

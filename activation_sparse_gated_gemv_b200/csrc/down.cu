@@ -61,8 +61,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_down(const DownParams p) {
     griddep_wait();
     griddep_launch_dependents();
 
-    // Counts and the segments' whole slot ranges, in one round trip.
-    for (int i = threadIdx.x; i < nseg; i += kThreads) cnt[i] = p.seg_count[seg0 + i];
+    // Counts and the segments' whole slot ranges, in one round trip.  Counts
+    // and channel ids come from the gate kernel: a count beyond its segment's
+    // slots, or a channel outside its segment's range, raises kStatusBounds
+    // and is dropped (clamped, or its row skipped) instead of being followed.
+    for (int i = threadIdx.x; i < nseg; i += kThreads) {
+        const int c = p.seg_count[seg0 + i];
+        const int room = max(0, min(p.cpb, p.d_ff - (seg0 + i) * p.cpb));
+        if (c < 0 || c > room) raise_status(p.status, p.hstatus, kStatusBounds);
+        cnt[i] = min(max(c, 0), room);
+    }
     for (int i = threadIdx.x; i < nseg * p.cpb; i += kThreads) {
         const int slot = seg0 * p.cpb + i;
         idx[i] = slot < p.d_ff ? p.lst_idx[slot] : 0;
@@ -88,7 +96,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_down(const DownParams p) {
     const int rows = pre[nseg];
     for (int i = threadIdx.x; i < nseg * p.cpb; i += kThreads) {
         const int j = i / p.cpb, o = i - j * p.cpb;
-        if (o < cnt[j]) rowk[pre[j] + o] = idx[i];
+        if (o < cnt[j]) {
+            const int k = idx[i], lo = (seg0 + j) * p.cpb;
+            const bool ok = k >= lo && k < lo + p.cpb && k < p.d_ff;
+            if (!ok) raise_status(p.status, p.hstatus, kStatusBounds);
+            rowk[pre[j] + o] = ok ? k : -1;
+        }
     }
     __syncthreads();
 
@@ -108,8 +121,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_down(const DownParams p) {
 #pragma unroll
             for (int u = 0; u < UB; ++u) {
                 const int i = i0 + u * RG;
-                const bool in = i < rows;
-                const int k = in ? rowk[i] : 0;
+                const int k = i < rows ? rowk[i] : -1;        // -1: no row, or one a check dropped
+                const bool in = k >= 0;
                 w[u] = (in && colok) ? ld_stream(wcol + (size_t)k * p.d) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) h[u][t] = (in && t < nt) ? p.lst_h[(size_t)k * p.n + t0 + t] : 0.f;

@@ -246,8 +246,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             unsigned backoff = 32;
             int ok = 1;
             while (ld_acquire_u64(bar + 1) < target) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                if (globaltimer_ns() - t0 > p.wait_ns) {
+                    raise_status(p.status, p.hstatus, kStatusWaitTimeout);
                     atomicExch(ctr + kAbort, 1);
                     ok = 0;
                     break;
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                 abort = true;
                 abort_at = j;
                 if (lane == 0) {
-                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                    raise_status(p.status, p.hstatus, kStatusWaitTimeout);
                     atomicExch(ctr + kAbort, 1);
                 }
             }
@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                 if ((vc[kGateDone] == kDecStreamWarps && vc[kQueueTail] <= i) || vc[kAbort]) break;
                 __nanosleep(64);
                 if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                    raise_status(p.status, p.hstatus, kStatusWaitTimeout);
                     atomicExch(ctr + kAbort, 1);
                     break;
                 }
@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     if (threadIdx.x == 0) {
         // release: the CTA's partial (ordered before this thread by the barrier) is visible first
         __threadfence();
-        if (col0 < p.d) target = grid_arrive(bar, G);
+        if (col0 < p.d) target = grid_arrive(bar, G) + (unsigned long long)p.bar_extra;
         else atomicAdd(bar, 1ull);                        // arrives only, waits for no one
     }
     // the CTA's list, for sffn_get_active only: off the path to the barrier
@@ -516,8 +516,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             const unsigned long long t0 = globaltimer_ns();
             unsigned backoff = 32;
             while (ld_acquire_u64(bar) < target) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    atomicOr(p.status, (int)kStatusWaitTimeout);
+                if (globaltimer_ns() - t0 > p.wait_ns) {
+                    raise_status(p.status, p.hstatus, kStatusWaitTimeout);
                     ok = 0;
                     break;
                 }
@@ -608,7 +608,8 @@ static cudaError_t launch_decode_t(const DecodeParams& p, int grid, size_t smem,
     static SmemAttrCache cache;
     cudaError_t e = ensure_smem(kern, smem, cache);
     if (e != cudaSuccess) return e;
-    return launch_ex(kern, dim3(grid), dim3(kDecThreads), smem, s, pdl, p);
+    // cooperative: the kernel's grid barriers need every CTA resident at once
+    return launch_ex(kern, dim3(grid), dim3(kDecThreads), smem, s, pdl, p, true);
 }
 
 template <class T, int NT>

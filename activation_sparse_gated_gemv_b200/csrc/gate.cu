@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_gate_stream(const GatePar
             if (!mbar_wait_warp(bars + cc.buf, (uint32_t)cc.parity)) {
                 abort = true;
                 abort_at = consumed;
-                if (lane == 0) atomicOr(p.status, (int)kStatusWaitTimeout);
+                if (lane == 0) raise_status(p.status, p.hstatus, kStatusWaitTimeout);
                 continue;
             }
             const unsigned char* buf = bufs + (size_t)cc.buf * p.sb;

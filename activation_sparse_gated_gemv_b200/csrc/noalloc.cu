@@ -126,8 +126,9 @@ extern "C" int sffn_forward_noalloc(const void* w_gate_cm, const void* w_up_cm, 
     while (!gate_stream_geometry(gnt, d, 0, kGateDense, cpb, 1, &sb, &nb, &gsmem) && gnt > 1) gnt /= 2;
     if (!sb) return na_fail(SFFN_ERR_UNSUPPORTED, "shape does not fit shared memory");
 
-    // The ticket counters and the status word must start at zero: clear them.
-    e = cudaMemsetAsync(b + kOffTickets, 0, kOffStatus + 256 - kOffTickets, s);
+    // The ticket counters must start at zero: clear them.  The status word is
+    // left alone: it keeps every failure until sffn_noalloc_check_status reads it.
+    e = cudaMemsetAsync(b + kOffTickets, 0, kOffStatus - kOffTickets, s);
     if (e != cudaSuccess) return na_fail(SFFN_ERR_CUDA, "clearing scratch: %s", cudaGetErrorString(e));
 
     GateParams gp{};
@@ -154,5 +155,29 @@ extern "C" int sffn_forward_noalloc(const void* w_gate_cm, const void* w_up_cm, 
     const int nseg = (g1 + chunks - 1) / chunks;
     e = launch_down(wdtype, dp, nt, slices, down_smem_bytes(wdtype, nt, nseg, cpb), s, true);
     if (e != cudaSuccess) return na_fail(SFFN_ERR_CUDA, "down launch: %s", cudaGetErrorString(e));
+    return SFFN_OK;
+}
+
+// Read, then clear, the status word in this device's scratch.
+extern "C" int sffn_noalloc_check_status(void) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) return na_fail(SFFN_ERR_CUDA, "cudaGetDevice failed");
+    void* base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_na_mutex);
+        base = g_na_ptr[dev];
+    }
+    if (!base) return SFFN_OK;                 // no call has run on this device
+    int* st = reinterpret_cast<int*>(static_cast<char*>(base) + kOffStatus);
+    int v = 0;
+    e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(&v, st, sizeof v, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && v) e = cudaMemset(st, 0, sizeof v);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return na_fail(SFFN_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (v & kStatusBounds) return na_fail(SFFN_ERR_DEVICE_CHECK, "a bounds check failed (status 0x%x)", v);
+    if (v & kStatusWaitTimeout) return na_fail(SFFN_ERR_TIMEOUT, "a bounded wait timed out (status 0x%x)", v);
+    if (v) return na_fail(SFFN_ERR_DEVICE_CHECK, "status word 0x%x", v);
     return SFFN_OK;
 }

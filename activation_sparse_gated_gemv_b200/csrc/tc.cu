@@ -186,9 +186,6 @@ __device__ __forceinline__ uint32_t mma_idesc(int n, int a_mn_major) {
            ((uint32_t)(kBM >> 4) << 24);
 }
 
-__device__ __forceinline__ void set_status(int* st, int bits) {
-    if (st) atomicOr(st, bits);
-}
 
 // The CTA c whose range [floor(c I/C), floor((c+1) I/C)) holds iteration i
 // (C <= I, so no range is empty).
@@ -287,7 +284,7 @@ __device__ void run_producer(const TcParams& p, const Problem& q, unsigned char*
             const int st = (int)(g % S);
             if (!mbar_wait_one(&sh->empty[st], (uint32_t)(((g / S) & 1) ^ 1))) {
                 sh->abort = 1;
-                set_status(p.status, kStatusWaitTimeout);
+                raise_status(p.status, p.hstatus, kStatusWaitTimeout);
                 return;
             }
             const uint32_t sA = smem_addr(stages + (size_t)st * stage_bytes);
@@ -350,7 +347,7 @@ __device__ void run_mma(const TcParams& p, const Problem& q, unsigned char* stag
     }
     if (!ok) {
         sh->abort = 1;
-        set_status(p.status, kStatusWaitTimeout);
+        raise_status(p.status, p.hstatus, kStatusWaitTimeout);
     }
     // all issued MMAs complete before the accumulators are released
     tc_commit(&sh->drain);
@@ -536,12 +533,12 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
         if (p.mode == kTcUp && owner) up_g_load(p, m, cols, g);   // in flight during the mainloop
         if (owner && !whole && !wait_parts(p, s.t, (unsigned)(c_last - c_first))) {
             sh->abort = 1;
-            set_status(p.status, kStatusWaitTimeout);
+            raise_status(p.status, p.hstatus, kStatusWaitTimeout);
             return;
         }
         if (!mbar_wait_warp(&sh->tfull[acc], use & 1u)) {
             sh->abort = 1;
-            set_status(p.status, kStatusWaitTimeout);
+            raise_status(p.status, p.hstatus, kStatusWaitTimeout);
             return;
         }
         tc_fence_after();
@@ -566,7 +563,7 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
                 }
                 if (!mbar_wait_warp(&sh->fix, 0)) {
                     sh->abort = 1;
-                    set_status(p.status, kStatusWaitTimeout);
+                    raise_status(p.status, p.hstatus, kStatusWaitTimeout);
                     return;
                 }
                 pbase = reinterpret_cast<const float*>(ring);
@@ -594,6 +591,17 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
                     }
                     add_parts16(p, pbase, slot_floats, np, row, c0, pglobal, v);
                     emit16(p, m, c0, v, act);
+                    if (p.mode == kTcGateZ && p.selbits && !p.topk) {
+                        // the selection itself, per token: one word per 32 channels of this warp
+                        const bool word_ok = m0 + quarter * 32 < p.m_total;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int tok = c0 + i;
+                            const unsigned b = __ballot_sync(0xffffffffu, tok < p.n && m < p.m_total && v[i] > p.tau);
+                            if (lane == 0 && word_ok && tok < p.n)
+                                p.selbits[(long long)tok * p.selw + ((m0 + quarter * 32) >> 5)] = b;
+                        }
+                    }
                 }
             }
             tc_fence_before();

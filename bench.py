@@ -6,11 +6,17 @@ of the workload's tokens.  Default workload: Llama-7B-shaped FFN decode
 (d=4096, d_ff=11008, one token, dense gate, tau for 90 % sparsity), the shape
 of the headline metric.  Prints one JSON line (rank 0).
 
-Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs on one
-stream, bracketed by a barrier and device synchronisation, timed with CUDA
-events; the max over ranks is taken.  Consecutive steps use different weight
-replicas whose total footprint exceeds 3x the L2, so no step finds its
-weights in L2.  Multi-GPU runs are independent replicas (weak scaling).
+Timing: W warm-up steps, then every captured graph is replayed once untimed
+(its first launch uploads it), then at least 50 ms of untimed replays run
+straight into the timed region, so the timed steps start in steady state.
+Exactly K steps are then replayed from CUDA graphs on one stream, bracketed by
+a barrier and device synchronisation, timed with CUDA events; the max over
+ranks is taken.  Consecutive steps use different weight replicas whose total
+footprint exceeds 3x the L2, so no step finds its weights in L2.  A second
+series times each replay of the graph on its own (median, p10, p90 per step),
+and a third times the same steps with one weight copy reused every step
+(weights warm in L2; labelled as such, not the headline).  Multi-GPU runs are
+independent replicas (weak scaling).
 
 Also reported: the same metric end to end through sffn_forward_host (host
 buffers, copies in the timed region), the library's dense FFN on the same
@@ -369,26 +375,40 @@ def main():
                 step(i, dense)
         return g
 
+    sampler = ClockSampler(local)
+    sampler.start()                            # sampling from the warm-up on: no idle gap before the timing
+
     G = max(1, min(a.graph_steps, a.steps))
     G = max(R, G - G % R) if G >= R else G
     graphs = [capture(0, G)]
     rem = a.steps % G
     rem_graph = capture(0, rem) if rem else None
 
-    # warm-up (untimed)
+    # warm-up (untimed), then one untimed replay of each graph (the first
+    # launch of a graph uploads it)
     with torch.cuda.stream(stream):
         for i in range(a.warmup):
             step(i)
+        graphs[0].replay()
+        if rem_graph is not None:
+            rem_graph.replay()
     torch.cuda.synchronize()
 
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
+    # pre-roll: untimed replays worth at least 50 ms of GPU time, queued
+    # straight ahead of the timed region, so it starts with the GPU busy
+    t_one = time.perf_counter()
+    with torch.cuda.stream(stream):
+        graphs[0].replay()
+    torch.cuda.synchronize()
+    t_one = time.perf_counter() - t_one
+    pre_replays = max(2, min(5000, int(0.05 / max(t_one, 1e-6)) + 1))
     sampler.mark("t0")
     with torch.cuda.stream(stream):
+        for _ in range(pre_replays):
+            graphs[0].replay()
         ev0.record(stream)
         for _ in range(a.steps // G):
             graphs[0].replay()
@@ -401,6 +421,42 @@ def main():
     ms_total = reduce_max(ev0.elapsed_time(ev1), world)
     ms_per_step = ms_total / a.steps
     us_per_token = ms_total * 1e3 / (a.steps * wl.n * world)
+
+    # -- spread: each replay of the G-step graph timed on its own, back to back
+    M = 50
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(M + 1)]
+    with torch.cuda.stream(stream):
+        graphs[0].replay()
+        evs[0].record(stream)
+        for j in range(M):
+            graphs[0].replay()
+            evs[j + 1].record(stream)
+    torch.cuda.synchronize()
+    per_rep = sorted(evs[j].elapsed_time(evs[j + 1]) * 1e3 / (G * wl.n) for j in range(M))
+    q = lambda f: per_rep[min(M - 1, int(round(f * (M - 1))))]
+    spread = {"median": round(statistics.median(per_rep), 4), "p10": round(q(0.1), 4), "p90": round(q(0.9), 4),
+              "unit": UNIT, "replays": M, "steps_per_replay": G,
+              "how": "CUDA events between back-to-back replays of the timed graph, per-step mean of each replay"}
+
+    # -- warm L2: the same steps with one weight copy reused every step
+    gw = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw, stream=stream, capture_error_mode="thread_local"):
+        for i in range(G):
+            ffns[0].forward(xs[i % P], gate=wl.gate, out=ys[i % P], stream=stream, **sel)
+    ew0, ew1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Mw = max(1, min(20, 2000 // G))
+    with torch.cuda.stream(stream):
+        gw.replay()
+        gw.replay()
+        ew0.record(stream)
+        for _ in range(Mw):
+            gw.replay()
+        ew1.record(stream)
+    torch.cuda.synchronize()
+    warm = {"value": round(ew0.elapsed_time(ew1) * 1e3 / (Mw * G * wl.n), 4), "unit": UNIT,
+            "note": f"L2-warm: one weight copy reused by every step ({algorithmic_bytes(wl, union) / 1e6:.0f} MB "
+                    f"touched per step, L2 {l2 / 2**20:.0f} MiB); not the headline"}
+    del gw
 
     # -- second pass: stage events around each kernel, same steps, replayed
     #    from a graph (events become external record nodes between kernels)
@@ -527,18 +583,31 @@ def main():
     # -- end to end through the C ABI with host buffers
     xs_host = [x.cpu().pin_memory() for x in xs]
     ys_host = [torch.empty((wl.n, wl.d), dtype=xs[0].dtype).pin_memory() for _ in range(P)]
-    Ke = min(a.e2e_steps, a.steps)
-    for i in range(min(20, Ke)):
-        ffns[i % R].forward_host(xs_host[i % P], gate=wl.gate, out=ys_host[i % P], stream=stream, **sel)
+    Ke = max(20, min(a.e2e_steps, a.steps))
+    # the C entry point itself, its arguments built once (what a caller with
+    # its own buffers does); each call copies x in, runs the forward, copies y
+    # out and synchronises
+    import ctypes
+    sel_c = sffn.make_select(**sel)
+    sel_ref = ctypes.byref(sel_c)
+    gcode = sffn.gate_code(wl.gate)
+    calls = [(ffns[i % R].handle, xs_host[i % P].data_ptr(), wl.n, gcode, sel_ref, ys_host[i % P].data_ptr(),
+              stream.cuda_stream) for i in range(math.lcm(R, P))]
+    fwd_host = sffn.sffn_forward_host
+    for i in range(20):
+        sffn.check(fwd_host(*calls[i % len(calls)]), "sffn_forward_host")
     torch.cuda.synchronize()
     barrier(world)
+    rcs = 0
     t0 = time.perf_counter()
     for i in range(Ke):
-        ffns[i % R].forward_host(xs_host[i % P], gate=wl.gate, out=ys_host[i % P], stream=stream, **sel)
+        rcs |= fwd_host(*calls[i % len(calls)])
     e2e_s = reduce_max(time.perf_counter() - t0, world)
+    sffn.check(rcs, "sffn_forward_host")
     xbytes = wl.n * wl.d * bytes_per_elem(wl.dtype)
     e2e = {"value": e2e_s * 1e6 / (Ke * wl.n * world), "unit": UNIT, "h2d_bytes_per_step": xbytes,
-           "d2h_bytes_per_step": xbytes, "steps": Ke, "timer": "host wall clock around synchronous calls"}
+           "d2h_bytes_per_step": xbytes, "steps": Ke,
+           "timer": "host wall clock around synchronous sffn_forward_host calls (pinned host x and y)"}
 
     clocks = sampler.stop()
     gpu_launches = a.steps * launches
@@ -560,7 +629,10 @@ def main():
                        "l2": f"{R} weight replicas rotated ({R * dense_bytes(wl) / 1e9:.2f} GB > L2 "
                              f"{l2 / 2**20:.0f} MiB), no step reuses L2-resident weights",
                        "mean_union": union, "timed_with": "CUDA graphs of "
-                       f"{G} steps, CUDA events on the launch stream"},
+                       f"{G} steps, CUDA events on the launch stream, after one untimed replay of each graph "
+                       f"and {pre_replays} untimed pre-roll replays (>= 50 ms) queued straight ahead of it"},
+            "spread": spread,
+            "warm_l2": warm,
             "tokens_per_s": round(wl.n * world / (ms_per_step * 1e-3), 1),
             "step_gbs": round(step_gbs, 1),
             "step_frac_of_hbm": round(step_gbs / peaks["hbm_gbs"], 4),

@@ -26,6 +26,17 @@
  *  - A handle is not thread-safe: one host thread at a time, and forwards on
  *    one handle must be ordered (same stream, or the caller orders them),
  *    because they share the handle's workspace.
+ *  - Device-side failures are recorded, not trapped.  Every wait inside a
+ *    kernel (on a bulk copy, a tensor-core commit, a grid barrier or another
+ *    CTA's part) is bounded in time; a wait that runs out sets the timeout bit
+ *    of the handle's sticky status word and the kernel returns early.  The down
+ *    kernel checks the channel ids and counts it reads from the gate kernel's
+ *    lists and skips any that lie outside their segment, setting the bounds
+ *    bit.  The word is mirrored into host-mapped memory, so sffn_forward,
+ *    sffn_forward_dense and sffn_forward_host return SFFN_ERR_TIMEOUT or
+ *    SFFN_ERR_DEVICE_CHECK, and launch nothing, once a forward that failed has
+ *    finished on the device.  The word stays set for the handle's lifetime:
+ *    destroy the handle and make a new one.
  */
 #ifndef SFFN_H
 #define SFFN_H
@@ -45,7 +56,7 @@ typedef enum {
     SFFN_ERR_UNSUPPORTED = 3,  /* e.g. LoPA forward on a handle without A and B */
     SFFN_ERR_CUDA = 4,         /* a CUDA runtime call or a launch failed */
     SFFN_ERR_OOM = 5,          /* device allocation failed */
-    SFFN_ERR_TIMEOUT = 6,      /* reserved for bounded device-side waits */
+    SFFN_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out (sticky) */
     SFFN_ERR_DEVICE_CHECK = 7  /* a kernel's own bounds check failed (sticky) */
 } sffn_status;
 
@@ -84,9 +95,14 @@ typedef struct {
     float p;             /* TOPP */
 } sffn_select;
 
-/* Allocate a handle and its device workspace, sized for cfg->max_tokens.
- * The library owns all device memory it allocates; sffn_destroy frees it.
- * Errors: INVALID_ARG (bad shape), CUDA (bad device), OOM. */
+/* Allocate a handle and its device workspace, sized for cfg->max_tokens,
+ * plus one small host-mapped pinned block (the status mirror).
+ * The library owns all memory it allocates; sffn_destroy frees it.
+ * Errors: INVALID_ARG (bad shape), CUDA (bad device), OOM; on any error
+ * nothing stays allocated and *out is NULL.
+ * Failure testing: with the environment variable SFFN_FAULT set to "alloc:N"
+ * (or "copy:N") the N-th allocation (or host-to-device copy) made by one call
+ * of sffn_create or sffn_set_weights reports failure without being made. */
 int sffn_create(sffn_handle* out, const sffn_config* cfg);
 
 /* Copy the weights in (host or device memory, src_is_device says which) and
@@ -97,7 +113,8 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg);
  * w_gate may be NULL when A and B are given and vice versa (not all three
  * NULL); A and B need lopa_rank > 0.  The caller keeps ownership of its
  * buffers.  Synchronises `stream` before returning.
- * Errors: INVALID_ARG, CUDA, OOM. */
+ * Errors: INVALID_ARG, CUDA, OOM; after an error the handle holds no weights
+ * (NOT_READY) and nothing it allocated for them stays allocated. */
 int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const void* B,
                      const void* w_up, const void* w_down, int src_is_device, void* stream);
 
@@ -105,7 +122,8 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
  * buffer, both in wdtype and caller-owned.  gate_mode: sffn_gate_mode.
  * Asynchronous on `stream`, no host synchronisation; n_tokens = 0 is a no-op.
  * The output is deterministic: the same inputs give bitwise the same y.
- * Errors: INVALID_ARG, NOT_READY, UNSUPPORTED, CUDA. */
+ * Errors: INVALID_ARG, NOT_READY, UNSUPPORTED, CUDA; TIMEOUT or DEVICE_CHECK
+ * when an earlier forward on the handle recorded a device-side failure. */
 int sffn_forward(sffn_handle h, const void* x, int n_tokens, int gate_mode,
                  const sffn_select* sel, void* out, void* stream);
 
@@ -125,9 +143,22 @@ int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_
 /* The last forward's active channels per token, for checking: idx (host,
  * n_tokens x d_ff int32) receives token t's ascending channel list at row t,
  * counts (host, n_tokens) its length, *union_size (host, may be NULL) the
- * number of distinct channels over all tokens.  Synchronises the last
- * forward's stream.  Errors: INVALID_ARG, NOT_READY (no forward yet), CUDA. */
+ * number of distinct channels over all tokens.  The lists are the kernels'
+ * own decisions: the fused decode kernel's compacted lists, the tensor-core
+ * gate's per-token selection bits (threshold), or the selection kernel's
+ * masks (top-K, top-p).  Synchronises the last forward's stream.
+ * Errors: INVALID_ARG, NOT_READY (no forward yet), CUDA, and the status
+ * word's TIMEOUT or DEVICE_CHECK. */
 int sffn_get_active(sffn_handle h, int32_t* idx, int32_t* counts, int32_t* union_size);
+
+/* The union bitmap the last tensor-core forward's up and down kernels took
+ * their active 128-channel blocks from (bit k of word k / 32: some token of
+ * the pass selected channel k; for more than 128 tokens, the last pass of
+ * 128).  bits: host, nwords >= ceil(d_ff / 32) words (words past that are
+ * zeroed).  Synchronises the last forward's stream.  Errors: INVALID_ARG,
+ * NOT_READY, UNSUPPORTED (the last forward did not take the tensor-core
+ * path), CUDA, and the status word's TIMEOUT or DEVICE_CHECK. */
+int sffn_get_union(sffn_handle h, uint32_t* bits, int nwords);
 
 /* Heavy-hitter channels (the heavy-hitter split, an abstract in the "FFN
  * modules" paper listing: a few FFN neurons carry a large output for every
@@ -160,11 +191,28 @@ int sffn_last_launches(sffn_handle h, int32_t* launches);
  * profiles and timing reports; "" when there is no such kernel. */
 const char* sffn_last_kernel_name(sffn_handle h, int i);
 
-/* Synchronise the device and read the handle's sticky device status word,
- * which kernels set when one of their own bounds checks fails (they then skip
- * the access instead of faulting).  Returns SFFN_OK or SFFN_ERR_DEVICE_CHECK
- * (the word stays set); also INVALID_ARG, CUDA. */
+/* Synchronise the device and read the handle's sticky device status word
+ * (see the conventions above).  Returns SFFN_OK, SFFN_ERR_DEVICE_CHECK (a
+ * bounds check failed), or SFFN_ERR_TIMEOUT (a bounded wait ran out); the
+ * word stays set.  Also INVALID_ARG, CUDA. */
 int sffn_check_status(sffn_handle h);
+
+/* Failure testing: arm a one-shot, host-side injection on the handle.
+ *  SFFN_INJECT_WAIT_TIMEOUT, arg = a wait limit in ns (1e3 .. 2e9): the next
+ *    fused decode forward (threshold selection, one or two tokens) waits at
+ *    its final grid barrier for one arrival more than the grid makes, gives up
+ *    after `arg` ns, records the timeout and leaves y unwritten; later calls
+ *    return SFFN_ERR_TIMEOUT.
+ *  SFFN_INJECT_BAD_LIST_ENTRY: the next forward that runs the separate down
+ *    kernel (fp32 top-K, for instance) has the host overwrite, between the
+ *    gate and the down kernel, the first entry of the first list segment with
+ *    a channel outside every segment and the second segment's count with one
+ *    beyond its slots; the down kernel's checks skip both and record them;
+ *    later calls return SFFN_ERR_DEVICE_CHECK.
+ * Nothing here makes a kernel fault: the failures are planted by the host and
+ * caught by the kernels' own bounded waits and checks.  Errors: INVALID_ARG. */
+enum { SFFN_INJECT_WAIT_TIMEOUT = 1, SFFN_INJECT_BAD_LIST_ENTRY = 2 };
+int sffn_debug_inject(sffn_handle h, int what, long long arg);
 
 /* Sparse forward that allocates no device memory, for callers that cannot
  * call cudaMalloc while they run: a host runtime that owns all device memory
@@ -192,10 +240,20 @@ int sffn_check_status(sffn_handle h);
  * two threads -- race and give wrong results: order them.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress, once per
  * device); make that first call before any stream capture.
+ * Device-side failures (a bounded wait that ran out, a list entry the down
+ * kernel's checks rejected) set a status word inside the scratch, which stays
+ * set until sffn_noalloc_check_status reads it.
  * Asynchronous on `stream` (cudaStream_t as void*, NULL = legacy default).
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 int sffn_forward_noalloc(const void* w_gate_cm, const void* w_up_cm, const void* w_down, int d, int d_ff,
                          int wdtype, const void* x, int n_tokens, float tau, void* out, void* stream);
+
+/* Synchronise the current device and read, then clear, the status word that
+ * sffn_forward_noalloc's kernels set on this device.  Returns SFFN_OK (also
+ * when no such call has run on the device), SFFN_ERR_TIMEOUT or
+ * SFFN_ERR_DEVICE_CHECK (some call since the last read failed: its output is
+ * not to be trusted), or SFFN_ERR_CUDA.  Allocates nothing. */
+int sffn_noalloc_check_status(void);
 
 /* Free the handle and everything it owns.  NULL is accepted. */
 int sffn_destroy(sffn_handle h);

@@ -336,14 +336,35 @@ def test_flop_ratio_closed_form_and_page_cap():
     assert ratio > cap
 
 
-def test_byte_counter_matches_layout_arithmetic():
-    # the dense gate, two bf16 rows of 8 KB per union channel, x in and y out
-    assert oracle.bytes_moved(1, 4096, 11008, 1101, 2, 2) == \
-        4096 * 11008 * 2 + 2 * 1101 * 8192 + 2 * 8192
-    assert oracle.bytes_moved(1, 4096, 11008, 1101, 2, 2, r=256) == \
-        256 * (4096 + 11008) * 2 + 2 * 1101 * 8192 + 2 * 8192
-    assert oracle.dense_bytes(1, 4096, 11008, 2, 2) == 3 * 4096 * 11008 * 2 + 2 * 8192
-    assert oracle.union_size([np.array([1, 5]), np.array([5, 7])]) == 3
+def test_byte_counter_counts_an_enumerated_row_list():
+    """The byte counters against the reads of one forward listed one by one on a
+    tiny case: every gate column (LoPA: every column of A and of B), each union
+    channel's W_up column and W_down row once for all tokens, each token's x
+    row read and y row written (dense FFN: every W_up column and W_down row)."""
+    d, d_ff, n, r = 16, 40, 3, 8
+    for dtype, wb in (("bf16", 2), ("f32", 4)):
+        w = workloads.ffn_weights(d, d_ff, dtype, seed=9, gate="both", r=r)
+        x = workloads.tokens(n, d, dtype, seed=9)
+        for gate in ("dense", "lopa"):
+            ref = oracle.forward(x, w, gate, "threshold", tau=0.3)
+            touched = sorted({int(k) for s in ref.sets for k in s})
+            assert 0 < len(touched) < d_ff
+            reads = []                                   # (what, index, elements)
+            if gate == "dense":
+                reads += [("W_gate column", k, d) for k in range(d_ff)]
+            else:
+                reads += [("A column", j, d) for j in range(r)] + [("B column", k, r) for k in range(d_ff)]
+            for k in touched:
+                reads += [("W_up column", k, d), ("W_down row", k, d)]
+            reads += [("x row", t, d) for t in range(n)] + [("y row", t, d) for t in range(n)]
+            assert len({(m, i) for m, i, _ in reads}) == len(reads)      # nothing listed twice
+            total = sum(e for _, _, e in reads) * wb
+            assert oracle.bytes_moved(n, d, d_ff, len(touched), wb, wb, r=r if gate == "lopa" else 0) == total
+            assert oracle.union_size(ref.sets) == len(touched)
+        dense = [("W_gate column", k, d) for k in range(d_ff)] + [("W_up column", k, d) for k in range(d_ff)]
+        dense += [("W_down row", k, d) for k in range(d_ff)] + [("x row", t, d) for t in range(n)]
+        dense += [("y row", t, d) for t in range(n)]
+        assert oracle.dense_bytes(n, d, d_ff, wb, wb) == sum(e for _, _, e in dense) * wb
 
 
 def test_thread_count_does_not_change_results():

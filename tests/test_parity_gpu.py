@@ -110,10 +110,101 @@ def test_llama70b_batches(llama70b_model, gate, n):
     assert union == len(set(np.concatenate(sets).tolist()))
 
 
+@pytest.mark.parametrize("gate", ["dense", "lopa"])
 @pytest.mark.parametrize("sparsity", workloads.SWEEP_70B_SPARSITIES)
-def test_llama70b_sparsity_sweep_lopa(llama70b_model, sparsity):
+def test_llama70b_sparsity_sweep_one_token(llama70b_model, gate, sparsity):
     wl, ffn, w = llama70b_model
-    check_forward(ffn, w, wl.x(n=1, tag="s"), "lopa", "threshold", tau=workloads.tau_for_sparsity(sparsity))
+    _, sets, _ = check_forward(ffn, w, wl.x(n=1, tag="s"), gate, "threshold",
+                               tau=workloads.tau_for_sparsity(sparsity))
+    assert ffn.last_kernel_names() == ["decode_fused"]
+    assert abs(len(sets[0]) / wl.d_ff - (1 - sparsity)) < 0.05
+
+
+# Every batch of the 70B-shaped sweep at sparsities other than 90 %, both
+# gates, on the tensor-core path (oracle on sampled tokens; the union is
+# checked against the oracle's at block granularity).
+@pytest.mark.parametrize("gate", ["dense", "lopa"])
+@pytest.mark.parametrize("n,sparsity", [(4, 0.7), (16, 0.5), (16, 0.99), (64, 0.8), (64, 0.95), (4, 0.99)])
+def test_llama70b_batches_other_sparsities(llama70b_model, gate, n, sparsity):
+    wl, ffn, w = llama70b_model
+    tau = workloads.tau_for_sparsity(sparsity)
+    x = wl.x(n=n, tag=f"b{sparsity}")
+    tokens = range(n) if n <= 4 else [0, n // 3, n - 1]
+    _, sets, union = check_forward(ffn, w, x, gate, "threshold", tau=tau, tokens=tokens)
+    assert "tc_gate" in ffn.last_kernel_names()
+    _check_union(ffn, sets, union)
+
+
+def _check_union(ffn, sets, union):
+    """The tensor-core kernels' union bitmap is exactly the OR of the per-token
+    selections the kernels made (which the parity checks compared with the
+    oracle up to the exempt band), and so are its active 128-channel blocks."""
+    bits = ffn.union_bits()
+    mask = np.zeros(ffn.d_ff, bool)
+    for s in sets:
+        mask[s] = True
+    got = ((bits[np.arange(ffn.d_ff) >> 5] >> (np.arange(ffn.d_ff) & 31).astype(np.uint32)) & 1).astype(bool)
+    assert np.array_equal(got, mask)
+    assert union == int(mask.sum())
+    nblk = (ffn.d_ff + 127) // 128
+    blk_got = np.zeros(nblk, bool)
+    blk_got[np.nonzero(got)[0] >> 7] = True
+    blk_want = np.zeros(nblk, bool)
+    blk_want[np.nonzero(mask)[0] >> 7] = True
+    assert np.array_equal(blk_got, blk_want)
+
+
+def _check_union_vs_oracle(ffn, w, x, gate, select, tau=0.0, k=0, p=0.0):
+    """Union bitmap against the oracle's union over all tokens: equal except
+    for channels inside the exempt band of the token that flips them; at block
+    granularity, equal except blocks whose only differences are such channels."""
+    from parity import silu, topp_exempt
+    ref = oracle.forward(x, w, gate, select, tau=tau, k=k, p=p)
+    bits = ffn.union_bits()
+    ch = np.arange(ffn.d_ff)
+    got = ((bits[ch >> 5] >> (ch & 31).astype(np.uint32)) & 1).astype(bool)
+    want = np.zeros(ffn.d_ff, bool)
+    exempt = np.zeros(ffn.d_ff, bool)
+    for t, s in enumerate(ref.sets):
+        want[s] = True
+        z = ref.z[t]
+        if select == "threshold":
+            exempt |= np.abs(z - tau) <= EXEMPT
+        elif select == "topk":
+            sv = silu(z)
+            gk = np.sort(sv)[::-1][k - 1] if k > 0 else np.inf
+            exempt |= np.abs(sv - gk) <= EXEMPT
+        else:
+            exempt[list(topp_exempt(z, p))] = True
+    diff = got ^ want
+    assert not np.any(diff & ~exempt), np.nonzero(diff & ~exempt)[0][:8]
+    nblk = (ffn.d_ff + 127) // 128
+    bg, bw = np.zeros(nblk, bool), np.zeros(nblk, bool)
+    bg[np.nonzero(got)[0] >> 7] = True
+    bw[np.nonzero(want)[0] >> 7] = True
+    for b in np.nonzero(bg ^ bw)[0]:
+        assert np.all(exempt[b * 128:(b + 1) * 128][diff[b * 128:(b + 1) * 128]]), f"block {b}"
+
+
+@pytest.mark.parametrize("select", ["threshold", "topk", "topp"])
+@pytest.mark.parametrize("n,sparsity", [(5, 0.999), (16, 0.995), (64, 0.9)])
+def test_union_bitmap_matches_oracle(sffn, select, n, sparsity):
+    # sparse enough that some 128-channel blocks stay inactive at small n
+    d, d_ff = 256, 4000
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=61, gate="dense")
+    x = workloads.tokens(n, d, "bf16", seed=62)
+    ffn = sffn.SparseFFN(d, d_ff, 0, n, "bf16")
+    ffn.set_weights(**w)
+    tau = workloads.tau_for_sparsity(sparsity)
+    k = max(1, int(round(d_ff * (1 - sparsity))))
+    _, sets, union = check_forward(ffn, w, x, "dense", select, tau=tau, k=k, p=0.3)
+    assert "tc_gate" in ffn.last_kernel_names()
+    _check_union(ffn, sets, union)
+    _check_union_vs_oracle(ffn, w, x, "dense", select, tau=tau, k=k, p=0.3)
+    if select == "threshold" and n == 5:
+        nact = len({c >> 7 for s in sets for c in s})
+        assert nact < (d_ff + 127) // 128              # the case does skip blocks
+    ffn.close()
 
 
 # --------------------------------------------------------------------------

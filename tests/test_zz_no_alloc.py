@@ -4,14 +4,18 @@ pool, or latency-critical code where an allocation may stall the device).
 It takes the caller's channel-major weights and keeps its scratch in a
 file-scope device array, so it needs no handle.
 
-Checked against the handle-based sffn_forward on the same weights and tokens,
-on two calls in a row (the second finds the first call's leftovers in the
-shared scratch), with the tolerance of the parity tests.  This file is named
-to run last so that a run stopping at the first failure has run the rest.
+Checked against the CPU oracle directly and against the handle-based
+sffn_forward on the same weights and tokens, on two calls in a row (the second
+finds the first call's leftovers in the shared scratch), with the tolerance of
+the parity tests; one case sits at the documented limits (d = 8192, 8 tokens,
+the 70B-shaped d_ff).  After the calls the no-alloc status word must be clean.
+This file is named to run last so that a run stopping at the first failure has
+run the rest.
 """
 import pytest
 import torch
 
+import oracle
 import workloads
 from parity import YTOL, assert_y, to_np
 
@@ -27,17 +31,19 @@ def sffn(cuda_device):
 
 
 CASES = [
-    # d, d_ff, n, dtype, tau
-    (4096, 11008, 1, "bf16", workloads.tau_for_sparsity(0.9)),
-    (512, 3000, 5, "bf16", workloads.tau_for_sparsity(0.8)),
-    (256, 1024, 4, "f32", 1.2816),
+    # d, d_ff, n, dtype, tau, oracle tokens
+    (4096, 11008, 1, "bf16", workloads.tau_for_sparsity(0.9), [0]),
+    (512, 3000, 5, "bf16", workloads.tau_for_sparsity(0.8), None),
+    (256, 1024, 4, "f32", 1.2816, None),
+    (8192, 28672, 8, "bf16", workloads.tau_for_sparsity(0.9), [0, 7]),   # at the limits
 ]
 
 
-@pytest.mark.parametrize("d,d_ff,n,dtype,tau", CASES)
-def test_noalloc_matches_handle_forward_twice(sffn, d, d_ff, n, dtype, tau):
+@pytest.mark.parametrize("d,d_ff,n,dtype,tau,tokens", CASES)
+def test_noalloc_matches_oracle_and_handle_forward_twice(sffn, d, d_ff, n, dtype, tau, tokens):
     w = workloads.ffn_weights(d, d_ff, dtype, seed=d_ff + 1)
-    x = workloads.tokens(n, d, dtype, seed=d_ff + 2).cuda()
+    x_cpu = workloads.tokens(n, d, dtype, seed=d_ff + 2)
+    x = x_cpu.cuda()
     ffn = sffn.SparseFFN(d, d_ff, 0, n, dtype)
     ffn.set_weights(**w)
     y_ref = ffn.forward(x, gate="dense", select="threshold", tau=tau)
@@ -56,8 +62,13 @@ def test_noalloc_matches_handle_forward_twice(sffn, d, d_ff, n, dtype, tau):
                                        x.data_ptr(), n, tau, out.data_ptr(), stream)
         assert rc == sffn.SFFN_OK
         torch.cuda.synchronize()
+    assert sffn.sffn_noalloc_check_status() == sffn.SFFN_OK
+    tok = list(range(n)) if tokens is None else tokens
+    ref = oracle.forward(x_cpu[tok], w, "dense", "threshold", tau=tau)
     for i, out in enumerate(outs):
-        assert_y(to_np(out), to_np(y_ref), YTOL, f"call {i + 1}")
+        assert_y(to_np(out), to_np(y_ref), YTOL, f"call {i + 1} vs the handle forward")
+        assert_y(to_np(out)[tok], ref.y, YTOL, f"call {i + 1} vs the oracle")
+    del wg_cm, wu_cm, wd
 
 
 def test_noalloc_rejects_sizes_beyond_its_limits(sffn):
@@ -66,3 +77,4 @@ def test_noalloc_rejects_sizes_beyond_its_limits(sffn):
     for d, d_ff, n in ((8200, 1024, 1), (4096, 32769, 1), (4096, 1024, 9), (12, 1024, 1)):
         rc = sffn.sffn_forward_noalloc(p, p, p, d, d_ff, sffn.SFFN_BF16, p, n, 1.0, p, None)
         assert rc == sffn.SFFN_ERR_INVALID_ARG, (d, d_ff, n)
+    assert sffn.sffn_noalloc_check_status() == sffn.SFFN_OK
