@@ -121,7 +121,7 @@ struct sffn_ctx {
     int* seg_count = nullptr;
     float* u = nullptr;
     float* dpart = nullptr;
-    float* fpart = nullptr;      // fused decode: [g1][min(max_tokens, 4)][d] partials of y
+    uint32_t* umask = nullptr;   // fused decode: [g1][ceil(cpb / 32)] union mask of each CTA's slots
     unsigned* tickets = nullptr;
     unsigned* dbar = nullptr;    // fused decode: grid-barrier arrival counters
     int* status = nullptr;
@@ -143,6 +143,10 @@ struct sffn_ctx {
     unsigned* tc_tickets = nullptr;
     bool maps_ok = false;        // weight tensor maps encoded
     CUtensorMap map_wg{}, map_at{}, map_bcm{}, map_wup{}, map_wdn{};
+    bool maps_g_ok = false;      // one-row-box maps of W_up and W_down for the gathered passes
+    CUtensorMap map_wup_g{}, map_wdn_g{};
+    int* ulist = nullptr;        // [round_up(d_ff, 128)] the union's channels, ascending (gathered passes)
+    int* ucount = nullptr;
     bool last_tc = false;        // the last forward took the tensor-core path
     bool last_topk = false;
     float last_tau = 0.f;
@@ -331,9 +335,20 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
         record(h, ++launches, s);
     }
 
+    // Small batches: the up and down passes gather exactly the union's rows
+    // (a list built from the union bitmap); larger ones, whose union covers
+    // nearly every channel, read whole 128-channel blocks.
+    const bool gather = !dense && n <= kTcGatherMaxTokens && h->maps_g_ok;
+    if (gather) {
+        SFFN_CUDA(launch_union_list(h->ubits, c.d_ff, h->ulist, h->ucount, s, true), "union list launch");
+        set_name(h, launches, "union_list");
+        record(h, ++launches, s);
+    }
+
     TcParams w = base;                          // h = g * <x, W_up[ch]> over the active channel blocks
     w.mode = kTcUp;
-    w.ta = h->map_wup; w.tb = map_x;
+    w.ta = gather ? h->map_wup_g : h->map_wup; w.tb = map_x;
+    w.gather = gather ? 1 : 0; w.ulist = h->ulist; w.ucount = h->ucount;
     w.ubits = h->ubits; w.d_ff = c.d_ff; w.force_all = dense ? 1 : 0;
     w.m_total = c.d_ff; w.k_total = c.d; w.nb = npad;
     w.out = h->h2; w.ldo = h->tc_ldh; w.h_pairs = 1;
@@ -344,7 +359,8 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
 
     TcParams dn = base;                         // y = sum over the active blocks of h W_down[ch]
     dn.mode = kTcDown;
-    dn.ta = h->map_wdn; dn.tb = map_h2;
+    dn.ta = gather ? h->map_wdn_g : h->map_wdn; dn.tb = map_h2;
+    dn.gather = gather ? 1 : 0; dn.ulist = h->ulist; dn.ucount = h->ucount;
     dn.ubits = h->ubits; dn.d_ff = c.d_ff; dn.force_all = dense ? 1 : 0;
     dn.m_total = c.d; dn.nb = 2 * npad; dn.paired = 1;
     dn.out = out; dn.ldo = c.d;
@@ -372,11 +388,12 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     record(h, 0, s);
     for (auto& nm : h->last_names) nm = nullptr;
 
-    // Fused decode path: threshold selection, a few tokens, sparse forward.
+    // Fused decode path: threshold selection, a few tokens; the sparse forward,
+    // or the dense FFN with a dense gate.
     int dec_sb = 0, dec_nb = 0;
     size_t dec_smem = 0;
     const int dec_nt = pick_nt(n);
-    const bool fused = sel->kind == SFFN_SELECT_THRESHOLD && !dense && n <= kDecodeMaxTokens &&
+    const bool fused = sel->kind == SFFN_SELECT_THRESHOLD && !(dense && lopa) && n <= kDecodeMaxTokens &&
                        decode_geometry(dec_nt, c.d, lopa ? c.lopa_rank : 0, gk, P.cpb, P.mw,
                                        c.wdtype == SFFN_BF16 ? 8 : 4, P.g1, &dec_sb, &dec_nb,
                                        &dec_smem);
@@ -417,13 +434,14 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         dp.wg = h->wg; dp.bcm = h->bcm; dp.at = h->a; dp.u = h->u; dp.wup = h->wup; dp.wdn = h->wdn;
         dp.tau = sel->tau; dp.cpb = P.cpb; dp.mw = P.mw;
         dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
-        dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.hstatus = h->hstat_dev; dp.part = h->fpart;
+        dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.hstatus = h->hstat_dev; dp.umask = h->umask;
         dp.wait_ns = h->inj_wait_ns ? h->inj_wait_ns : kWaitLimitNs;
         dp.bar_extra = h->inj_wait_ns ? 1 : 0;
         h->inj_wait_ns = 0;
-        dp.tickets = h->dbar; dp.y = out; dp.hot = h->hot_on ? h->hot : nullptr;
+        dp.tickets = h->dbar; dp.y = out; dp.hot = h->hot_on && !dense ? h->hot : nullptr;
+        dp.dense = dense ? 1 : 0;
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
-        set_name(h, launches, "decode_fused");
+        set_name(h, launches, dense ? "decode_dense" : "decode_fused");
         record(h, ++launches, s);
         h->last_n = n;
         h->last_stream = s;
@@ -584,7 +602,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_seg = take((size_t)P.g1 * 4);
     const size_t o_u = take(T * R * 4);
     const size_t o_dp = take((size_t)P.down_chunks * T * D * 4);
-    const size_t o_fp = take((size_t)P.g1 * (T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * D * 4);
+    const size_t o_um = take((size_t)P.g1 * ((P.cpb + 31) / 32) * 4);
     const size_t o_tk = take((size_t)(P.down_slices > 2 ? P.down_slices : 2) * 4), o_st = take(4);
     const size_t o_db = take(16);   // the decode kernel's two grid-barrier counters (64-bit, never reset)
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
@@ -599,6 +617,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->selw = (int)((F + 31) / 32);
     const size_t o_sb = take(h->tc ? T * (size_t)h->selw * 4 : 0);
     const size_t o_h2 = take(2 * NP * (size_t)h->tc_ldh * 2), o_u2 = take(2 * NP * R * 2);
+    const size_t o_ul = take(h->tc ? (size_t)h->tc_ldh * 4 : 0), o_uc = take(h->tc ? 16 : 0);
     // stream-K partial tiles: two slots per CTA of up to 256 accumulator columns x 128 rows
     const size_t o_tp = take(h->tc ? (size_t)h->sms * 2 * 256 * 128 * 4 : 0), o_tt = take(h->tc ? tiles * 8 : 0);
     e = faults.malloc_dev(&h->ws, off);
@@ -628,7 +647,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->seg_count = reinterpret_cast<int*>(b + o_seg);
     h->u = reinterpret_cast<float*>(b + o_u);
     h->dpart = reinterpret_cast<float*>(b + o_dp);
-    h->fpart = reinterpret_cast<float*>(b + o_fp);
+    h->umask = reinterpret_cast<uint32_t*>(b + o_um);
     h->tickets = reinterpret_cast<unsigned*>(b + o_tk);
     h->dbar = reinterpret_cast<unsigned*>(b + o_db);
     h->status = reinterpret_cast<int*>(b + o_st);
@@ -637,6 +656,8 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     if (h->tc) {
         h->ubits = reinterpret_cast<uint32_t*>(b + o_ub);
         h->selbits = reinterpret_cast<uint32_t*>(b + o_sb);
+        h->ulist = reinterpret_cast<int*>(b + o_ul);
+        h->ucount = reinterpret_cast<int*>(b + o_uc);
         h->h2 = b + o_h2;
         h->u2 = b + o_u2;
         h->tc_part = reinterpret_cast<float*>(b + o_tp);
@@ -729,7 +750,7 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
     h->has_lopa = A != nullptr;
     h->ready = true;
     // tensor maps of the weights for the batched tensor-core path (host-side encoding only)
-    h->maps_ok = false;
+    h->maps_ok = h->maps_g_ok = false;
     if (h->tc && c.d >= 64) {
         const uint64_t F = c.d_ff, D = c.d, R = c.lopa_rank;
         bool ok = encode_tile_map(&h->map_wup, h->wup, D, F, D * 2, 64, 128) == cudaSuccess &&
@@ -739,6 +760,8 @@ int sffn_set_weights(sffn_handle h, const void* w_gate, const void* A, const voi
             ok = encode_tile_map(&h->map_at, h->a, D, R, D * 2, 64, 128) == cudaSuccess &&
                  encode_tile_map(&h->map_bcm, h->bcm, R, F, R * 2, 64, 128) == cudaSuccess;
         h->maps_ok = ok;
+        h->maps_g_ok = ok && encode_tile_map(&h->map_wup_g, h->wup, D, F, D * 2, 64, 1) == cudaSuccess &&
+                       encode_tile_map(&h->map_wdn_g, h->wdn, D, F, D * 2, 64, 1) == cudaSuccess;
     }
     return SFFN_OK;
 }
@@ -762,10 +785,25 @@ int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_
     if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = (size_t)n_tokens * h->cfg.d * h->esz;
+    // A page-locked output that the device can address (any cudaHostAlloc'd or
+    // registered buffer under unified addressing) is written by the fused
+    // decode kernel itself, one slice store per CTA: no device-to-host copy.
+    // Other outputs, and batches that take the multi-kernel paths, go through
+    // the workspace and a copy.
+    // (The check runs on every call: a buffer can be freed and its address reused.)
+    void* ydst = h->ydev;
+    if (n_tokens <= kFusedMaxTokens) {
+        cudaPointerAttributes pa{};
+        if (cudaPointerGetAttributes(&pa, out_host) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
+            pa.devicePointer && aligned16(pa.devicePointer))
+            ydst = pa.devicePointer;
+        cudaGetLastError();
+    }
     SFFN_CUDA(cudaMemcpyAsync(h->xdev, x_host, bytes, cudaMemcpyHostToDevice, s), "x host-to-device copy");
-    rc = run_forward(h, h->xdev, n_tokens, gate_mode, sel, h->ydev, s, false);
+    rc = run_forward(h, h->xdev, n_tokens, gate_mode, sel, ydst, s, false);
     if (rc) return rc;
-    SFFN_CUDA(cudaMemcpyAsync(out_host, h->ydev, bytes, cudaMemcpyDeviceToHost, s), "y device-to-host copy");
+    if (ydst == h->ydev)
+        SFFN_CUDA(cudaMemcpyAsync(out_host, h->ydev, bytes, cudaMemcpyDeviceToHost, s), "y device-to-host copy");
     SFFN_CUDA(cudaStreamSynchronize(s), "stream synchronize");
     return SFFN_OK;
 }

@@ -268,19 +268,20 @@ struct DecodeParams {
     const void* wdn;        // [d_ff][d]
     float tau;
     int cpb, mw;
-    int* lst_idx;           // [CTAs][cpb] each CTA's active channels, ascending
-    float* lst_h;           // unused by the fused kernel
-    uint32_t* lst_mask;     // [d_ff][mw]
-    int* seg_count;         // [CTAs]
+    int* lst_idx;           // [CTAs][cpb] each CTA's active channels, ascending (for sffn_get_active)
+    float* lst_h;           // [d_ff][n] h of the union's channels (0 for a token that did not select one)
+    uint32_t* lst_mask;     // [d_ff][mw] (for sffn_get_active)
+    int* seg_count;         // [CTAs] (for sffn_get_active)
+    uint32_t* umask;        // [CTAs][ceil(cpb / 32)] union mask of each CTA's channel slots
     int sb, nb;             // streamed piece bytes, pieces in flight per streaming warp
     int* status;
     int* hstatus;           // host-mapped mirror of the status word, or NULL
     unsigned long long wait_ns;   // limit of the grid-barrier waits
     int bar_extra;          // arrivals the final grid barrier expects beyond the grid (0; 1 makes it time out)
-    float* part;            // [CTAs][n][d] per-CTA partials of y
     unsigned* tickets;      // two 64-bit grid-barrier arrival counters (8-byte aligned), zero at creation
     void* y;                // [n][d] T
     const uint32_t* hot;    // [ceil(d_ff / 32)] heavy-hitter channel bits, or NULL
+    int dense;              // dense FFN (dense gate): every channel, W_up rows streamed with the gate's
 };
 
 // Batched tensor-core GEMM (tcgen05): modes and parameters.
@@ -314,6 +315,9 @@ struct alignas(64) TcParams {
     uint32_t* ubits;        // gate: union bitmap out (threshold), zeroed (top-K); up, down: read
     uint32_t* selbits;      // gate, threshold: per-token selection bits [n][selw] (bit k: z[t,k] > tau), or NULL
     int selw;               // words per token row of selbits (ceil(d_ff / 32))
+    int gather;             // up, down: gather the union's channel rows (ta is a one-row-box map) in list order
+    const int* ulist;       // gather: the union's channels, ascending, padded with channel 0 to a multiple of 128
+    const int* ucount;      // gather: the union's size
     float* part;            // [CTAs][128][nb] each CTA's parked stream-K part (room for [CTAs][2][128][256])
     unsigned* tickets;      // two counters per tile (parts arrived, owner warps done), zero between launches
     int* status;
@@ -415,6 +419,10 @@ size_t tc_smem_bytes(int nb, int* stages);
 cudaError_t encode_tile_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                             uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
 cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s, bool pdl);
+// The union bitmap (bit k of word k / 32) as an ascending channel list,
+// padded with channel 0 to a multiple of 128, and its size.
+cudaError_t launch_union_list(const uint32_t* ubits, int d_ff, int* list, int* count, cudaStream_t s, bool pdl);
+constexpr int kTcGatherMaxTokens = 3;  // batches up to this size gather the union's rows
 constexpr int kTcMaxTokens = 128;     // token columns of one tensor-core pass (hi/lo pairs fill N = 256)
 
 }  // namespace sffn

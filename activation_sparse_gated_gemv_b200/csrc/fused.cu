@@ -49,9 +49,26 @@ __host__ __device__ inline int decode_slice_chunks(int d, int vec, int grid) {
     while (cps * vec * grid < d) cps <<= 1;
     return cps;
 }
-// Bytes the cross-CTA sum keeps in the (then idle) streaming ring.
-__host__ __device__ inline size_t decode_tail_bytes(int, int, int, int) {
-    return (size_t)kDecThreads * 16;                     // one float4 per thread for the partial sums
+// Words of a CTA's union mask (one bit per channel slot).
+__host__ __device__ inline int decode_mask_words(int cpb) { return (cpb + 31) / 32; }
+
+// The column-slice pass after the grid barrier keeps, in the (then idle)
+// streaming ring: every CTA's union mask, the union's ascending channel list
+// (at most cpb x grid entries), the per-group partial sums of the slice
+// (threads x V x NT floats: kDecThreads / cps groups of NT x cps V) and the
+// sub-sums of the fixed-order reduction.
+struct DecodeTail {
+    size_t masks, list, red, red2, total;
+};
+__host__ __device__ inline DecodeTail decode_tail_layout(int nt, int cpb, int vec, int grid) {
+    DecodeTail T;
+    size_t o = 0;
+    T.masks = o; o += ((size_t)grid * decode_mask_words(cpb) * 4 + 15) & ~(size_t)15;
+    T.list = o;  o += ((size_t)grid * cpb * 4 + 15) & ~(size_t)15;
+    T.red = o;   o += (size_t)kDecThreads * vec * nt * sizeof(float);
+    T.red2 = o;  o += (size_t)kDecThreads * sizeof(float);
+    T.total = o;
+    return T;
 }
 __host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, int gate_kind, int cpb, int mw,
                                                          int sb, int nb, int vec, int grid) {
@@ -62,7 +79,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, i
     size_t o = 0;
     L.xs = o;    o += (size_t)nt * d * sizeof(float);
     L.us = o;    o += gate_kind == kGateLopa ? (size_t)nt * r * sizeof(float) : 0;
-    L.zpart = o; o += (size_t)cpb * ppr * nt * sizeof(float);
+    L.zpart = o; o += (size_t)cpb * 2 * ppr * nt * sizeof(float);   // x2: dense mode's up parts
     L.zfin = o;  o += (size_t)cpb * nt * sizeof(float);
     L.hs = o;    o += (size_t)cpb * nt * sizeof(float);
     L.hu = o;    o += (size_t)cpb * nt * sizeof(float);
@@ -73,12 +90,12 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int nt, int d, int r, i
     L.mask = o;  o += (size_t)cpb * mw * sizeof(uint32_t);
     L.flag = o;  o += ((size_t)cpb + 15) & ~(size_t)15;
     L.hrdy = o;  o += ((size_t)cpb + 15) & ~(size_t)15;
-    L.scan = o;  o += 48 * sizeof(int);
+    L.scan = o;  o += 96 * sizeof(int);
     o = (o + 15) & ~(size_t)15;
     L.bars = o;  o += (size_t)kDecStreamWarps * nb * sizeof(uint64_t);
     o = (o + 127) & ~(size_t)127;
     L.bufs = o;
-    const size_t ring = (size_t)kDecStreamWarps * nb * sb, tail = decode_tail_bytes(nt, d, vec, grid);
+    const size_t ring = (size_t)kDecStreamWarps * nb * sb, tail = decode_tail_layout(nt, cpb, vec, grid).total;
     o += ring > tail ? ring : tail;
     L.total = o;
     return L;
@@ -134,8 +151,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     const T* wdn = static_cast<const T*>(p.wdn);
     const char* gbase = reinterpret_cast<const char*>(static_cast<const T*>(GATE == kGateLopa ? p.bcm : p.wg) +
                                                       (size_t)c0 * glen);
+    // Dense FFN mode (dense gate only): every channel is kept, and its W_up row
+    // is streamed through the ring right after its gate row, as parts
+    // ppr .. 2 ppr - 1 of the channel, so z and the up dot finish together.
+    const bool dense = GATE == kGateDense && p.dense;
+    const bool rows_mode = !dense && rb <= p.sb;          // pieces of whole rows, else parts of a row
+    const char* ubase = reinterpret_cast<const char*>(wup + (size_t)c0 * glen);
     int rpp, ppr, pb;
-    if (rb <= p.sb) {
+    if (rows_mode) {
         const int per_warp = (nslots + kDecStreamWarps - 1) / kDecStreamWarps;
         rpp = max(1, min(p.sb / rb, per_warp));
         ppr = 1;
@@ -146,32 +169,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         pb = ((rb + ppr - 1) / ppr + 15) & ~15;
         ppr = (rb + pb - 1) / pb;
     }
-    const int npieces = rb <= p.sb ? (nslots + rpp - 1) / rpp : nslots * ppr;
+    const int pps = dense ? 2 * ppr : ppr;               // parts per channel slot
+    const int npieces = rows_mode ? (nslots + rpp - 1) / rpp : nslots * pps;
     const int w0 = streamer ? (int)((long long)npieces * warp / kDecStreamWarps) : 0;
     const int wcount = streamer ? (int)((long long)npieces * (warp + 1) / kDecStreamWarps) - w0 : 0;
     const uint64_t pol = l2_evict_first();
 
     // Cursor over this warp's pieces (w0 + j): row group g, part, ring slot, parity.
-    int ig = rb <= p.sb ? w0 : w0 / ppr, ipart = rb <= p.sb ? 0 : w0 - (w0 / ppr) * ppr, ibuf = 0;
+    int ig = rows_mode ? w0 : w0 / pps, ipart = rows_mode ? 0 : w0 - (w0 / pps) * pps, ibuf = 0;
     int issued = 0;
     auto issue_next = [&]() {
         uint32_t bytes;
         const char* src;
-        if (rb <= p.sb) {
+        if (rows_mode) {
             const int r0 = ig * rpp;
             bytes = (uint32_t)(min(rpp, nslots - r0) * rb);
             src = gbase + (size_t)r0 * rb;
         } else {
-            const int off = ipart * pb;
+            const int q = ipart < ppr ? ipart : ipart - ppr;
+            const int off = q * pb;
             bytes = (uint32_t)min(pb, rb - off);
-            src = gbase + (size_t)ig * rb + off;
+            src = (ipart < ppr ? gbase : ubase) + (size_t)ig * rb + off;
         }
         if (lane == 0) {
             mbar_expect_tx(bars + ibuf, bytes);
             bulk_load(bufs + (size_t)ibuf * p.sb, src, bytes, bars + ibuf, pol);
         }
         if (++ibuf == p.nb) ibuf = 0;
-        if (++ipart >= ppr) {
+        if (++ipart >= pps) {
             ipart = 0;
             ++ig;
         }
@@ -263,18 +288,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         __syncthreads();
     }
 
-    // Row s is complete: z from its parts in order, select, queue it.
+    // Row s is complete: z from its parts in order, select, queue it.  Dense
+    // mode: the up dot is complete too (parts ppr ..), so h is formed here
+    // and every channel is kept (with h = 0 for a token whose z <= tau).
     auto finalize = [&](int s) {                         // lane 0 only
         __threadfence_block();
         uint32_t tokmask = 0u;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             float z = 0.f;
-            for (int q = 0; q < ppr; ++q) z += zpart[(s * ppr + q) * NT + t];
+            for (int q = 0; q < ppr; ++q) z += zpart[(s * pps + q) * NT + t];
             zfin[s * NT + t] = z;
             if (t < n && z > p.tau) tokmask |= 1u << t;
+            if (dense) {
+                float u = 0.f;
+                for (int q = ppr; q < pps; ++q) u += zpart[(s * pps + q) * NT + t];
+                hs[s * NT + t] = (t < n && z > p.tau) ? (z - p.tau) * u : 0.f;
+            }
         }
-        if (tokmask) {
+        if (dense) {
+            flag[s] = 1;
+            smask[s * p.mw] = (1u << n) - 1u;
+            bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+        } else if (tokmask) {
             flag[s] = 1;
             smask[s * p.mw] = tokmask;                   // n <= 4: tokens sit in mask word 0
             bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
@@ -287,7 +323,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     // ---- streaming warps
     if (streamer) {
         int cbuf = 0, cpar = 0;
-        int g = rb <= p.sb ? w0 : w0 / ppr, part = rb <= p.sb ? 0 : w0 - (w0 / ppr) * ppr;
+        int g = rows_mode ? w0 : w0 / pps, part = rows_mode ? 0 : w0 - (w0 / pps) * pps;
         bool abort = false;
         int abort_at = 0;
         for (int j = 0; j < wcount; ++j) {
@@ -301,7 +337,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             }
             if (!abort) {
                 const unsigned char* buf = bufs + (size_t)cbuf * p.sb;
-                if (rb <= p.sb) {
+                if (rows_mode) {
                     const int r0 = g * rpp, cnt = min(rpp, nslots - r0);
                     for (int q = 0; q < cnt; ++q) {
                         float2 v2[NT];
@@ -317,7 +353,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                         if (lane == 0) finalize(r0 + q);
                     }
                 } else {
-                    const int off = part * pb;
+                    const int off = (part < ppr ? part : part - ppr) * pb;
                     float2 v2[NT];
 #pragma unroll
                     for (int t = 0; t < NT; ++t) v2[t] = make_float2(0.f, 0.f);
@@ -325,12 +361,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
                         const float v = warp_sum(v2[t].x + v2[t].y);
-                        if (lane == t) zpart[(g * ppr + part) * NT + t] = v;
+                        if (lane == t) zpart[(g * pps + part) * NT + t] = v;
                     }
                     __syncwarp();
                     if (lane == 0) {
                         __threadfence_block();
-                        if (atomicAdd(done + g, 1) == ppr - 1) finalize(g);
+                        if (atomicAdd(done + g, 1) == pps - 1) finalize(g);
                     }
                 }
                 __syncwarp();
@@ -343,7 +379,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                 cbuf = 0;
                 cpar ^= 1;
             }
-            if (++part >= ppr) {
+            if (++part >= pps) {
                 part = 0;
                 ++g;
             }
@@ -428,89 +464,54 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     }
     __syncthreads();
 
-    // ---- the CTA's list (ascending, one warp, ballots), then its share of the down projection
-    if (warp == 0) {
-        int cnt = 0;
-        for (int base = 0; base < nslots; base += 32) {
-            const int sl = base + lane;
-            const bool f = sl < nslots && flag[sl];
-            const unsigned m = __ballot_sync(0xffffffffu, f);
-            if (f) wl[cnt + __popc(m & ((1u << lane) - 1u))] = sl;
-            cnt += __popc(m);
+    // ---- publish this CTA's part of the union: one mask bit per slot that
+    // some token selected, and h for those slots (every token; 0 for a token
+    // that did not select the channel)
+    const int mwc = decode_mask_words(p.cpb);
+    for (int w = threadIdx.x; w < mwc; w += kDecThreads) {
+        uint32_t m = 0u;
+        for (int i = 0; i < 32; ++i) {
+            const int sl = 32 * w + i;
+            if (sl < nslots && flag[sl]) m |= 1u << i;
         }
-        if (lane == 0) scan_sh[0] = cnt;
+        p.umask[(size_t)blockIdx.x * mwc + w] = m;
     }
-    __syncthreads();
-    const int tot = scan_sh[0];
-
-    // ---- the CTA's share of the down projection: h_k W_down[k, :] over its
-    // active channels in list order (whole rows, mostly in L2 by now), as an
-    // fp32 partial of y.
-    constexpr int UB = 8;
-    const int cpd = p.d / V;                              // 16-byte chunks per output row
-    for (int cch = threadIdx.x; cch < cpd; cch += kDecThreads) {
-        float2 acc[NT][V / 2];
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-            for (int e = 0; e < V / 2; ++e) acc[t][e] = make_float2(0.f, 0.f);
-        for (int i0 = 0; i0 < tot; i0 += UB) {
-            uint4 w[UB];
-#pragma unroll
-            for (int u2 = 0; u2 < UB; ++u2) {
-                const int i = i0 + u2;
-                w[u2] = i < tot ? ld_stream(wdn + (size_t)(c0 + wl[i]) * p.d + (size_t)cch * V)
-                                : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int u2 = 0; u2 < UB; ++u2) {
-                const int i = i0 + u2;
-                if (i < tot) {
-                    float wf[V];
-                    unpack<T>(w[u2], wf);
-#pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        const float h = hs[wl[i] * NT + t];
-                        const float2 hh = make_float2(h, h);
-#pragma unroll
-                        for (int e = 0; e < V / 2; ++e)
-                            acc[t][e] = __ffma2_rn(make_float2(wf[2 * e], wf[2 * e + 1]), hh, acc[t][e]);
-                    }
-                }
-            }
-        }
-        for (int t = 0; t < n; ++t) {
-            float* dst = p.part + ((size_t)blockIdx.x * n + t) * p.d + (size_t)cch * V;
-#pragma unroll
-            for (int e = 0; e < V / 2; e += 2)
-                *reinterpret_cast<float4*>(dst + 2 * e) =
-                    make_float4(acc[t][e].x, acc[t][e].y, acc[t][e + 1].x, acc[t][e + 1].y);
-        }
+    for (int i = threadIdx.x; i < nslots * n; i += kDecThreads) {
+        const int sl = i / n, t = i - sl * n;
+        if (flag[sl]) p.lst_h[(size_t)(c0 + sl) * n + t] = hs[sl * NT + t];
     }
 
-    // ---- grid barrier: every CTA's partial is out.  All CTAs are resident
-    // (one per SM, grid <= SMs, and a dependent launch waits until every CTA of
-    // this grid has started), so the wait ends; it is bounded all the same.
-    // A CTA without a column slice only arrives.
+    // ---- grid barrier: every CTA's mask and h are out.  All CTAs are
+    // resident (a cooperative launch of one CTA per SM), so the wait ends; it
+    // is bounded all the same.  A CTA without a column slice of y only arrives.
     const int G = gridDim.x;
     const int cps = decode_slice_chunks(p.d, V, G);       // 16-byte chunks per column slice
     const int col0 = blockIdx.x * cps * V;
     __syncthreads();
     unsigned long long target = 0ull;
     if (threadIdx.x == 0) {
-        // release: the CTA's partial (ordered before this thread by the barrier) is visible first
-        __threadfence();
+        __threadfence();                                  // release: the CTA's mask and h first
         if (col0 < p.d) target = grid_arrive(bar, G) + (unsigned long long)p.bar_extra;
-        else atomicAdd(bar, 1ull);                        // arrives only, waits for no one
+        else atomicAdd(bar, 1ull);
     }
-    // the CTA's list, for sffn_get_active only: off the path to the barrier
-    for (int i = threadIdx.x; i < tot; i += kDecThreads) {
-        const int sl = wl[i];
-        p.lst_idx[c0 + i] = c0 + sl;
-        for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + sl) * p.mw + w] = smask[sl * p.mw + w];
+    // the CTA's ascending list and token masks, for sffn_get_active only: off
+    // the path to the barrier (one warp, ballots)
+    if (warp == 0) {
+        int cnt = 0;
+        for (int base = 0; base < nslots; base += 32) {
+            const int sl = base + lane;
+            const bool f = sl < nslots && flag[sl];
+            const unsigned m = __ballot_sync(0xffffffffu, f);
+            if (f) {
+                const int i = cnt + __popc(m & ((1u << lane) - 1u));
+                p.lst_idx[c0 + i] = c0 + sl;
+                for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + sl) * p.mw + w] = smask[sl * p.mw + w];
+            }
+            cnt += __popc(m);
+        }
+        if (lane == 0) p.seg_count[blockIdx.x] = cnt;
     }
     if (threadIdx.x == 0) {
-        p.seg_count[blockIdx.x] = tot;
         int ok = 1;
         if (col0 < p.d) {
             const unsigned long long t0 = globaltimer_ns();
@@ -528,49 +529,101 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         scan_sh[2] = ok;
     }
     __syncthreads();
-    if (scan_sh[2] && col0 < p.d) {
-        __threadfence();
-        // y[:, col0 : col0 + cps V] = sum over the G partials.  Thread (g, item)
-        // adds partials g, g + GR, ... in order; then the GR sums in order.
-        const int q4 = min(cps * V, p.d - col0) / 4;     // float4 per token
-        const int items = n * q4;
-        const int GR = max(1, kDecThreads / items);
-        float4* red = reinterpret_cast<float4*>(smem + L.bufs);          // the idle ring
-        const int g = (int)threadIdx.x / items, item = (int)threadIdx.x - g * items;
-        if (g < GR) {
-            const int t = item / q4, c = col0 + (item - t * q4) * 4;
-            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-            constexpr int UB = 16;
-            for (int b0 = g; b0 < G; b0 += UB * GR) {
-                float4 v[UB];
-#pragma unroll
-                for (int u2 = 0; u2 < UB; ++u2) {
-                    const int b = b0 + u2 * GR;
-                    v[u2] = b < G ? __ldcg(reinterpret_cast<const float4*>(p.part + ((size_t)b * n + t) * p.d + c))
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int u2 = 0; u2 < UB; ++u2)
-                    if (b0 + u2 * GR < G) {
-                        sum.x += v[u2].x; sum.y += v[u2].y; sum.z += v[u2].z; sum.w += v[u2].w;
-                    }
-            }
-            red[g * items + item] = sum;
+    if (!scan_sh[2] || col0 >= p.d) return;
+    __threadfence();
+
+    // ---- y[:, col0 : col0 + cps V] = sum over the union, in ascending channel
+    // order, of h[k] W_down[k, slice].  The W_down rows were pulled into L2
+    // when their channels were selected, so the slices come from L2.
+    const DecodeTail TL = decode_tail_layout(NT, p.cpb, V, G);
+    uint32_t* gm = reinterpret_cast<uint32_t*>(smem + L.bufs + TL.masks);     // [G][mwc]
+    int* list = reinterpret_cast<int*>(smem + L.bufs + TL.list);              // [<= d_ff]
+    float* red = reinterpret_cast<float*>(smem + L.bufs + TL.red);            // [groups][NT][slice]
+    float* red2 = reinterpret_cast<float*>(smem + L.bufs + TL.red2);          // [kDecThreads]
+    const int nw = G * mwc;
+    for (int i = threadIdx.x; i < nw; i += kDecThreads) gm[i] = __ldcg(p.umask + i);
+    __syncthreads();
+    // the union's channels in ascending order: word i is CTA i / mwc's slots
+    // 32 (i % mwc) .. + 31, so word order is channel order
+    const int per = (nw + kDecThreads - 1) / kDecThreads;
+    const int wa = min(nw, (int)threadIdx.x * per), wb = min(nw, wa + per);
+    int cw = 0;
+    for (int i = wa; i < wb; ++i) cw += __popc(gm[i]);
+    int U = 0;
+    int pos = block_exclusive_scan(cw, &U, scan_sh + 48);
+    for (int i = wa; i < wb; ++i) {
+        uint32_t m = gm[i];
+        const int b = i / mwc, base = b * p.cpb + 32 * (i - b * mwc);
+        while (m) {
+            list[pos++] = base + __ffs(m) - 1;
+            m &= m - 1u;
         }
-        __syncthreads();
-        if ((int)threadIdx.x < items) {
-            float4 sum = red[threadIdx.x];
-            for (int q = 1; q < GR; ++q) {
-                const float4 v = red[q * items + threadIdx.x];
-                sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-            }
-            const int t = (int)threadIdx.x / q4, c = col0 + ((int)threadIdx.x - t * q4) * 4;
-            T* dst = static_cast<T*>(p.y) + (size_t)t * p.d + c;
-            dst[0] = from_f32<T>(sum.x);
-            dst[1] = from_f32<T>(sum.y);
-            dst[2] = from_f32<T>(sum.z);
-            dst[3] = from_f32<T>(sum.w);
+    }
+    __syncthreads();
+
+    // thread (group g, chunk cc): rows g, g + NG, ... of the list, 16 bytes each
+    const int NG = kDecThreads / cps;
+    const int g = (int)threadIdx.x / cps, cc = (int)threadIdx.x - g * cps;
+    const int col = col0 + cc * V;
+    const bool colok = col < p.d;
+    float2 acc[NT][V / 2];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < V / 2; ++e) acc[t][e] = make_float2(0.f, 0.f);
+    constexpr int UB = 8;
+    for (int i0 = g; i0 < U; i0 += UB * NG) {
+        uint4 w[UB];
+        float hv[UB][NT];
+#pragma unroll
+        for (int u2 = 0; u2 < UB; ++u2) {
+            const int i = i0 + u2 * NG;
+            const int k = i < U ? list[i] : -1;
+            w[u2] = (k >= 0 && colok) ? ld_stream(wdn + (size_t)k * p.d + col) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) hv[u2][t] = (k >= 0 && t < n) ? __ldcg(p.lst_h + (size_t)k * n + t) : 0.f;
         }
+#pragma unroll
+        for (int u2 = 0; u2 < UB; ++u2) {
+            float wf[V];
+            unpack<T>(w[u2], wf);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const float2 hh = make_float2(hv[u2][t], hv[u2][t]);
+#pragma unroll
+                for (int e = 0; e < V / 2; ++e)
+                    acc[t][e] = __ffma2_rn(make_float2(wf[2 * e], wf[2 * e + 1]), hh, acc[t][e]);
+            }
+        }
+    }
+    // fixed-order sum over the NG groups: Q sub-sums of consecutive groups,
+    // then the Q sub-sums in order
+    const int SC = cps * V;
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < V / 2; ++e)
+            *reinterpret_cast<float2*>(red + ((size_t)g * NT + t) * SC + cc * V + 2 * e) = acc[t][e];
+    __syncthreads();
+    const int items = n * SC;
+    const int Q = kDecThreads / items;                    // >= 1 (the geometry checks n SC <= threads)
+    const int GPQ = (NG + Q - 1) / Q;
+    {
+        const int q = (int)threadIdx.x / items, it = (int)threadIdx.x - q * items;
+        if (q < Q) {
+            const int t = it / SC, j = it - t * SC;
+            float sum = 0.f;
+            const int ga = q * GPQ, gb = min(NG, ga + GPQ);
+            for (int gg = ga; gg < gb; ++gg) sum += red[((size_t)gg * NT + t) * SC + j];
+            red2[q * items + it] = sum;
+        }
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < items) {
+        const int it = threadIdx.x, t = it / SC, j = it - t * SC;
+        float sum = 0.f;
+        for (int q = 0; q < Q; ++q) sum += red2[q * items + it];
+        if (col0 + j < p.d) static_cast<T*>(p.y)[(size_t)t * p.d + col0 + j] = from_f32<T>(sum);
     }
 }
 
@@ -582,8 +635,10 @@ size_t decode_smem_bytes(int nt, int d, int r, int gate_kind, int cpb, int mw, i
 
 bool decode_geometry(int nt, int d, int r, int gate_kind, int cpb, int mw, int vec, int grid, int* sb, int* nb,
                      size_t* smem) {
-    // the cross-CTA sum gives one thread to each (token, 4 columns) of a slice
-    if (grid < 1 || (long)nt * decode_slice_chunks(d, vec, grid) * vec / 4 > kDecThreads) return false;
+    // the column-slice pass gives one thread to each (token, column) of a slice
+    // in its last step, and at least one thread to each 16-byte chunk
+    const int cps = grid < 1 ? 0 : decode_slice_chunks(d, vec, grid);
+    if (grid < 1 || (long)nt * cps * vec > kDecThreads || cps > kDecThreads) return false;
     int best_sb = 0, best_nb = 0;
     for (int cand_sb : {8192, 4096, 2048})
         for (int cand_nb = 2; cand_nb <= 4; ++cand_nb) {

@@ -66,6 +66,8 @@ constexpr int kMaxStages = 12;
 constexpr int kMaxBlocks = 1024;    // 128-channel blocks (d_ff <= 131072)
 constexpr int kMinIters = 8;        // iterations per CTA at least
 constexpr int kMaxParts = 8;        // CTAs sharing one tile at most
+constexpr int kIdxPerProducer = 4;  // gather: channel-index blocks each producer keeps in flight
+constexpr int kIdxSlots = kProducers * kIdxPerProducer;
 
 struct TcShared {
     uint64_t full[kMaxStages];
@@ -78,7 +80,10 @@ struct TcShared {
     int abort;
     int reducer;
     int wcount[kTcThreads / 32];
+    int ucount;             // gather: the union's size
     int blk[kMaxBlocks];    // up/down: the active 128-channel blocks
+    uint64_t ibar[kIdxSlots];
+    alignas(16) int idx[kIdxSlots][kBM];   // gather: channel indices of one k-block's rows
 };
 
 // ---- tcgen05 / TMA primitives ------------------------------------------------
@@ -148,6 +153,19 @@ __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, i
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
 }
+// Four rows of a one-row-box tensor map (rows r0..r3, columns x .. x + box)
+// into four consecutive 128-byte rows of this CTA's shared memory at dst (the
+// 128-byte swizzle follows the destination address, as for a tile), completing
+// on `bar`.  x is a multiple of 64 elements (128 bytes).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int4 r, uint64_t* bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r.x), "r"(r.y), "r"(r.z), "r"(r.w),
+          "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
 // Ask the TMA engine to bring the box at (x, y) of the tensor map into L2.
 __device__ __forceinline__ void tma_prefetch_tile(const CUtensorMap* map, int x, int y) {
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
@@ -203,15 +221,16 @@ struct Problem {
     long long I, it0, it1;
 };
 
+// nblk: the active 128-channel blocks, or with gather the union's size.
 __device__ __forceinline__ Problem make_problem(const TcParams& p, int nblk) {
     Problem q;
     q.nblk = nblk;
     if (p.mode == kTcUp) {
-        q.T = q.nblk;
+        q.T = p.gather ? (nblk + kBM - 1) / kBM : q.nblk;
         q.KB = (p.k_total + kBK - 1) / kBK;
     } else if (p.mode == kTcDown) {
         q.T = (p.m_total + kBM - 1) / kBM;
-        q.KB = 2 * q.nblk;
+        q.KB = p.gather ? (nblk + kBK - 1) / kBK : 2 * q.nblk;
     } else {
         q.T = (p.m_total + kBM - 1) / kBM;
         q.KB = (p.k_total + kBK - 1) / kBK;
@@ -270,8 +289,82 @@ __device__ void prefetch_first_tiles(const TcParams& p, int count) {
 // ring stays one sequence for the MMA issuer.  (A producer waits for stage
 // g - S to be consumed; with kProducers <= S the parity wait cannot be a phase
 // behind.)
+// Gather: k-block g of the CTA's range is iteration it0 + g, i.e. tile
+// (it0 + g) / KB and k-block (it0 + g) % KB, so a producer knows every future
+// k-block's rows.  Their channel indices (up: the tile's 128 list entries;
+// down: the k-block's 64) are bulk-copied into a small ring of index blocks,
+// kIdxPerProducer k-blocks ahead of their use.
+__device__ __forceinline__ void gather_index_copy(const TcParams& p, const Problem& q, TcShared* sh, int pr,
+                                                  long long g) {
+    const long long j = g / kProducers;
+    const int slot = pr * kIdxPerProducer + (int)(j % kIdxPerProducer);
+    const long long it = q.it0 + g;
+    const int t = (int)(it / q.KB), kb = (int)(it % q.KB);
+    const int* src = p.mode == kTcUp ? p.ulist + (size_t)t * kBM : p.ulist + (size_t)kb * kBK;
+    const uint32_t bytes = p.mode == kTcUp ? kBM * 4u : kBK * 4u;
+    mbar_expect_tx(&sh->ibar[slot], bytes);
+    bulk_load(sh->idx[slot], src, bytes, &sh->ibar[slot], l2_evict_last());
+}
+
+__device__ void run_producer_gather(const TcParams& p, const Problem& q, unsigned char* stages, uint32_t stage_bytes,
+                                    TcShared* sh, int pr) {
+    const uint64_t pol_w = l2_evict_first(), pol_b = l2_evict_last();
+    const int S = p.stages;
+    const uint32_t tx = kTileA + (uint32_t)p.nb * 128u;
+    const long long n_it = q.it1 - q.it0;
+    for (int j = 0; j < kIdxPerProducer; ++j) {
+        const long long g = pr + (long long)kProducers * j;
+        if (g < n_it) gather_index_copy(p, q, sh, pr, g);
+    }
+    for (long long g = pr; g < n_it; g += kProducers) {
+        const long long j = g / kProducers;
+        const int slot = pr * kIdxPerProducer + (int)(j % kIdxPerProducer);
+        const long long it = q.it0 + g;
+        const int t = (int)(it / q.KB), kb = (int)(it % q.KB);
+        const int st = (int)(g % S);
+        if (!mbar_wait_one(&sh->ibar[slot], (uint32_t)((j / kIdxPerProducer) & 1)) ||
+            !mbar_wait_one(&sh->empty[st], (uint32_t)(((g / S) & 1) ^ 1))) {
+            sh->abort = 1;
+            raise_status(p.status, p.hstatus, kStatusWaitTimeout);
+            return;
+        }
+        const uint32_t sA = smem_addr(stages + (size_t)st * stage_bytes);
+        const uint32_t sB = sA + kTileA;
+        const int4* rows = reinterpret_cast<const int4*>(sh->idx[slot]);
+        if (p.mode == kTcDown) {
+            // MN-major A: the k-block's 64 channels (rows of W_down) x 128 output columns, two 64-column
+            // halves; a half wholly past the last output column is not loaded (its accumulator rows are
+            // never stored, and each row of the product depends on its own A row only)
+            const int m0 = t * kBM;
+            const bool hi = m0 + 64 < p.m_total;
+            mbar_expect_tx(&sh->full[st], hi ? tx : tx - 8192u);
+#pragma unroll 4
+            for (int i = 0; i < kBK / 4; ++i) {
+                const int4 r = rows[i];
+                tma_gather4(sA + i * 512, &p.ta, m0, r, &sh->full[st], pol_w);
+                if (hi) tma_gather4(sA + 8192 + i * 512, &p.ta, m0 + 64, r, &sh->full[st], pol_w);
+            }
+            tma_tile(sB, &p.tb, kb * kBK, 0, &sh->full[st], pol_b);   // h, compacted by list position
+        } else {
+            // K-major A: the tile's 128 channels (rows of W_up) x 64 k
+            mbar_expect_tx(&sh->full[st], tx);
+#pragma unroll 4
+            for (int i = 0; i < kBM / 4; ++i) tma_gather4(sA + i * 512, &p.ta, kb * kBK, rows[i], &sh->full[st], pol_w);
+            tma_tile(sB, &p.tb, kb * kBK, 0, &sh->full[st], pol_b);
+        }
+        // this thread's reads of the index block come before the async copy that refills it
+        fence_proxy_async();
+        const long long gn = g + (long long)kProducers * kIdxPerProducer;
+        if (gn < n_it) gather_index_copy(p, q, sh, pr, gn);
+    }
+}
+
 __device__ void run_producer(const TcParams& p, const Problem& q, unsigned char* stages, uint32_t stage_bytes,
                              TcShared* sh, int pr) {
+    if (p.gather) {
+        run_producer_gather(p, q, stages, stage_bytes, sh, pr);
+        return;
+    }
     const uint64_t pol_w = l2_evict_first(), pol_b = l2_evict_last();
     const int S = p.stages;
     const uint32_t tx = kTileA + (uint32_t)p.nb * 128u;
@@ -404,11 +497,11 @@ struct UpG {
     float raw[kUpChunks * 16];
 };
 
-// Issue the loads of the gate source (z or the selected g) of channel m for the
-// first `cols` token columns.
+// Issue the loads of the gate source (z or the selected g) of channel m (m < 0:
+// none, a padding row of a gathered tile) for the first `cols` token columns.
 __device__ __forceinline__ void up_g_load(const TcParams& p, int m, int cols, UpG& g) {
     const float* src = p.topk ? p.gsel : p.zsel;
-    const bool row_ok = m < p.m_total;
+    const bool row_ok = m >= 0 && m < p.m_total;
 #pragma unroll
     for (int j = 0; j < kUpChunks; ++j) {
         if (16 * j < cols) {
@@ -421,19 +514,21 @@ __device__ __forceinline__ void up_g_load(const TcParams& p, int m, int cols, Up
     }
 }
 
-// Columns 16j..16j+15 of channel m: h = g * v, written as bf16 hi (and lo) rows.
-__device__ __forceinline__ void up_emit16(const TcParams& p, int m, int j, const float* v, const UpG& g) {
+// Columns 16j..16j+15 of channel m (m < 0: a padding row, h = 0): h = g * v,
+// written as bf16 hi (and lo) rows at output column mo (the channel, or with
+// gather its list position).
+__device__ __forceinline__ void up_emit16(const TcParams& p, int m, int mo, int j, const float* v, const UpG& g) {
     bf16* o = static_cast<bf16*>(p.out);
-    const bool row_ok = m < p.m_total;
+    const bool row_ok = m >= 0 && m < p.m_total;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int tok = 16 * j + i;
         const float raw = g.raw[16 * j + i];
         const float gv = (row_ok && tok < p.n) ? (p.topk ? raw : fmaxf(raw - p.tau, 0.f)) : 0.f;
-        const float h = gv * v[i];
+        const float h = row_ok ? gv * v[i] : 0.f;
         const bf16 hi = __float2bfloat16_rn(h);
-        o[(long long)tok * p.ldo + m] = hi;
-        if (p.h_pairs) o[(long long)(p.npad + tok) * p.ldo + m] = __float2bfloat16_rn(h - __bfloat162float(hi));
+        o[(long long)tok * p.ldo + mo] = hi;
+        if (p.h_pairs) o[(long long)(p.npad + tok) * p.ldo + mo] = __float2bfloat16_rn(h - __bfloat162float(hi));
     }
 }
 
@@ -527,8 +622,12 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
         const int c_first = whole ? (int)blockIdx.x : cta_of((long long)s.t * q.KB, q.I, C);
         const int c_last = whole ? (int)blockIdx.x : cta_of((long long)(s.t + 1) * q.KB - 1, q.I, C);
         const bool owner = c_first == (int)blockIdx.x;
-        const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
-        const int m = m0 + row;
+        // up: output row `row` of the tile is channel m, written at column mo
+        // (gather: list position mo = the tile's first position + row, whose
+        // channel is the list entry, none past the union's size)
+        const int m0 = p.mode == kTcUp ? (p.gather ? s.t * kBM : sh->blk[s.t] * kBM) : s.t * kBM;
+        const int mo = m0 + row;
+        const int m = (p.mode == kTcUp && p.gather) ? (mo < sh->ucount ? __ldcg(p.ulist + mo) : -1) : mo;
         UpG g;
         if (p.mode == kTcUp && owner) up_g_load(p, m, cols, g);   // in flight during the mainloop
         if (owner && !whole && !wait_parts(p, s.t, (unsigned)(c_last - c_first))) {
@@ -577,7 +676,7 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
                     float v[16];
                     tmem_ld16(taddr + 16 * j, v);
                     add_parts16(p, pbase, slot_floats, np, row, 16 * j, pglobal, v);
-                    up_emit16(p, m, j, v, g);
+                    up_emit16(p, m, mo, j, v, g);
                 }
             } else {
                 for (int c0 = 0; c0 < cols; c0 += 16) {
@@ -661,6 +760,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
         }
         mbar_init(&sh->drain, 1);
         mbar_init(&sh->fix, 1);
+        for (int i = 0; i < kIdxSlots; ++i) mbar_init(&sh->ibar[i], 1);
         sh->abort = 0;
         sh->reducer = 0;
         fence_mbar_init();
@@ -671,11 +771,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
 
-    if (warp == kProdWarp && (threadIdx.x & 31) == 0) prefetch_first_tiles(p, p.stages);
+    if (warp == kProdWarp && (threadIdx.x & 31) == 0 && !p.gather) prefetch_first_tiles(p, p.stages);
     griddep_launch_dependents();
     griddep_wait();
     int nblk = 0;
-    if (p.mode == kTcUp || p.mode == kTcDown) {
+    if (p.gather) {
+        // the union's size (its list was built by the previous kernel)
+        nblk = __ldcg(p.ucount);
+        if (threadIdx.x == 0) sh->ucount = nblk;
+        __syncthreads();
+    } else if (p.mode == kTcUp || p.mode == kTcDown) {
         // the 128-channel blocks holding a channel some token selected, from the union bitmap
         const int nbk = (p.d_ff + 127) / 128, nwords = (p.d_ff + 31) >> 5;
         const int lane = threadIdx.x & 31;
@@ -728,6 +833,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     if (warp == kMmaWarp) tmem_dealloc(tmem, p.tmem_cols);
 }
 
+// The union bitmap as an ascending channel list (one CTA): each thread takes a
+// run of words, a block scan places them, and the list is padded with channel
+// 0 (a real row, whose h is zero) to a multiple of 128 for the gathered tiles.
+constexpr int kListThreads = 1024;
+__global__ void __launch_bounds__(kListThreads) k_union_list(const uint32_t* ubits, int d_ff, int* list, int* count) {
+    __shared__ int sh[40];
+    griddep_wait();
+    griddep_launch_dependents();
+    const int W = (d_ff + 31) >> 5;
+    const int per = (W + kListThreads - 1) / kListThreads;
+    const int w0 = min(W, (int)threadIdx.x * per), w1 = min(W, w0 + per);
+    auto word = [&](int w) {
+        uint32_t b = __ldcg(ubits + w);
+        if (w == W - 1 && (d_ff & 31)) b &= (1u << (d_ff & 31)) - 1u;
+        return b;
+    };
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(word(w));
+    int U = 0;
+    int pos = block_exclusive_scan(c, &U, sh);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t b = word(w);
+        while (b) {
+            list[pos++] = 32 * w + __ffs(b) - 1;
+            b &= b - 1u;
+        }
+    }
+    const int padded = (U + kBM - 1) / kBM * kBM;
+    for (int i = U + (int)threadIdx.x; i < padded; i += kListThreads) list[i] = 0;
+    if (threadIdx.x == 0) *count = U;
+}
+
 SmemAttrCache g_tc_smem;
 std::once_flag g_enc_once;
 PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
@@ -743,11 +880,27 @@ size_t tc_smem_bytes(int nb, int* stages) {
     return 1024 + (size_t)s * stage + sizeof(TcShared);
 }
 
+cudaError_t launch_union_list(const uint32_t* ubits, int d_ff, int* list, int* count, cudaStream_t s, bool pdl) {
+    if (!ubits || !list || !count || d_ff < 1) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kListThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_union_list, ubits, d_ff, list, count);
+}
+
 cudaError_t launch_tc(const TcParams& p_in, int grid, cudaStream_t s, bool pdl) {
     TcParams p = p_in;
     if (p.nb < 16 || p.nb > 256 || p.nb % 16 || (p.paired && 2 * p.npad != p.nb)) return cudaErrorInvalidValue;
-    if ((p.mode == kTcUp || p.mode == kTcDown) && ((p.d_ff + 127) / 128 > kMaxBlocks || (!p.ubits && !p.force_all)))
+    if ((p.mode == kTcUp || p.mode == kTcDown) && !p.gather &&
+        ((p.d_ff + 127) / 128 > kMaxBlocks || (!p.ubits && !p.force_all)))
         return cudaErrorInvalidValue;
+    if (p.gather && (!p.ulist || !p.ucount || (p.mode != kTcUp && p.mode != kTcDown))) return cudaErrorInvalidValue;
     int st = 0;
     const size_t smem = tc_smem_bytes(p.nb, &st);
     if (!smem) return cudaErrorInvalidValue;

@@ -134,9 +134,12 @@ int sffn_forward_dense(sffn_handle h, const void* x, int n_tokens, int gate_mode
                        const sffn_select* sel, void* out, void* stream);
 
 /* sffn_forward with HOST buffers: copies x_host to the device, runs the
- * forward and copies the result into out_host, all on `stream`, then
- * synchronises it.  Pinned host memory gives asynchronous copies.
- * Errors: as sffn_forward. */
+ * forward and delivers the result into out_host, all on `stream`, then
+ * synchronises it.  Pinned host memory gives asynchronous copies; with one or
+ * two tokens and a page-locked out_host that the device can address (memory
+ * from cudaHostAlloc / cudaMallocHost or cudaHostRegister under unified
+ * addressing), the decode kernel stores y there directly instead of copying
+ * it back.  Errors: as sffn_forward. */
 int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_mode,
                       const sffn_select* sel, void* out_host, void* stream);
 

@@ -379,6 +379,28 @@ def test_forward_host_matches_device_forward(sffn):
     ffn.close()
 
 
+@pytest.mark.parametrize("n,pinned_out", [(1, True), (1, False), (2, True), (5, True)])
+def test_forward_host_output_kinds(sffn, n, pinned_out):
+    """One or two tokens into a page-locked output: the decode kernel stores y
+    in host memory itself; a pageable output, or a batch, goes through a copy.
+    Either way y is bitwise the device forward's."""
+    d, d_ff = 512, 3000
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=91)
+    ffn = sffn.SparseFFN(d, d_ff, 0, 8, "bf16")
+    ffn.set_weights(**w)
+    x = workloads.tokens(n, d, "bf16", seed=92)
+    tau = workloads.tau_for_sparsity(0.9)
+    yd = ffn.forward(x.cuda(), tau=tau).cpu()
+    out = torch.full((n, d), float("nan"), dtype=torch.bfloat16)
+    if pinned_out:
+        out = out.pin_memory()
+    for _ in range(2):
+        yh = ffn.forward_host(x.pin_memory(), tau=tau, out=out)
+        assert torch.equal(yd, yh)
+        out.fill_(float("nan"))
+    ffn.close()
+
+
 def test_device_source_weights(sffn):
     wl = workloads.tiny()
     ffn, w = _ffn(sffn, wl, device_src=True)
