@@ -122,6 +122,7 @@ struct sffn_ctx {
     float* u = nullptr;
     float* dpart = nullptr;
     uint32_t* umask = nullptr;   // fused decode: [g1][ceil(cpb / 32)] union mask of each CTA's slots
+    float* fpart = nullptr;      // fused decode, dense FFN: [g1][min(max_tokens, 4)][d] partials of y
     unsigned* tickets = nullptr;
     unsigned* dbar = nullptr;    // fused decode: grid-barrier arrival counters
     int* status = nullptr;
@@ -347,7 +348,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
 
     TcParams w = base;                          // h = g * <x, W_up[ch]> over the active channel blocks
     w.mode = kTcUp;
-    w.ta = gather ? h->map_wup_g : h->map_wup; w.tb = map_x;
+    w.ta = h->map_wup; w.tg = h->map_wup_g; w.tb = map_x;
     w.gather = gather ? 1 : 0; w.ulist = h->ulist; w.ucount = h->ucount;
     w.ubits = h->ubits; w.d_ff = c.d_ff; w.force_all = dense ? 1 : 0;
     w.m_total = c.d_ff; w.k_total = c.d; w.nb = npad;
@@ -359,7 +360,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
 
     TcParams dn = base;                         // y = sum over the active blocks of h W_down[ch]
     dn.mode = kTcDown;
-    dn.ta = gather ? h->map_wdn_g : h->map_wdn; dn.tb = map_h2;
+    dn.ta = h->map_wdn; dn.tg = h->map_wdn_g; dn.tb = map_h2;
     dn.gather = gather ? 1 : 0; dn.ulist = h->ulist; dn.ucount = h->ucount;
     dn.ubits = h->ubits; dn.d_ff = c.d_ff; dn.force_all = dense ? 1 : 0;
     dn.m_total = c.d; dn.nb = 2 * npad; dn.paired = 1;
@@ -434,7 +435,7 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         dp.wg = h->wg; dp.bcm = h->bcm; dp.at = h->a; dp.u = h->u; dp.wup = h->wup; dp.wdn = h->wdn;
         dp.tau = sel->tau; dp.cpb = P.cpb; dp.mw = P.mw;
         dp.lst_idx = h->lst_idx; dp.lst_h = h->lst_h; dp.lst_mask = h->lst_mask; dp.seg_count = h->seg_count;
-        dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.hstatus = h->hstat_dev; dp.umask = h->umask;
+        dp.sb = dec_sb; dp.nb = dec_nb; dp.status = h->status; dp.hstatus = h->hstat_dev; dp.umask = h->umask; dp.part = h->fpart;
         dp.wait_ns = h->inj_wait_ns ? h->inj_wait_ns : kWaitLimitNs;
         dp.bar_extra = h->inj_wait_ns ? 1 : 0;
         h->inj_wait_ns = 0;
@@ -603,8 +604,9 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_u = take(T * R * 4);
     const size_t o_dp = take((size_t)P.down_chunks * T * D * 4);
     const size_t o_um = take((size_t)P.g1 * ((P.cpb + 31) / 32) * 4);
+    const size_t o_fp = take((size_t)P.g1 * (T < kDecodeMaxTokens ? T : kDecodeMaxTokens) * D * 4);
     const size_t o_tk = take((size_t)(P.down_slices > 2 ? P.down_slices : 2) * 4), o_st = take(4);
-    const size_t o_db = take(16);   // the decode kernel's two grid-barrier counters (64-bit, never reset)
+    const size_t o_db = take(32);   // the decode kernel's grid-barrier counters (64-bit, never reset)
     const size_t o_x = take(T * D * h->esz), o_y = take(T * D * h->esz);
     // tensor-core path buffers
     h->tc = c.wdtype == SFFN_BF16 && c.max_tokens > 1;
@@ -648,6 +650,7 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     h->u = reinterpret_cast<float*>(b + o_u);
     h->dpart = reinterpret_cast<float*>(b + o_dp);
     h->umask = reinterpret_cast<uint32_t*>(b + o_um);
+    h->fpart = reinterpret_cast<float*>(b + o_fp);
     h->tickets = reinterpret_cast<unsigned*>(b + o_tk);
     h->dbar = reinterpret_cast<unsigned*>(b + o_db);
     h->status = reinterpret_cast<int*>(b + o_st);

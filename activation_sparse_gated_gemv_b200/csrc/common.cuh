@@ -273,12 +273,13 @@ struct DecodeParams {
     uint32_t* lst_mask;     // [d_ff][mw] (for sffn_get_active)
     int* seg_count;         // [CTAs] (for sffn_get_active)
     uint32_t* umask;        // [CTAs][ceil(cpb / 32)] union mask of each CTA's channel slots
+    float* part;            // dense mode: [CTAs][n][d] per-CTA partials of y
     int sb, nb;             // streamed piece bytes, pieces in flight per streaming warp
     int* status;
     int* hstatus;           // host-mapped mirror of the status word, or NULL
     unsigned long long wait_ns;   // limit of the grid-barrier waits
     int bar_extra;          // arrivals the final grid barrier expects beyond the grid (0; 1 makes it time out)
-    unsigned* tickets;      // two 64-bit grid-barrier arrival counters (8-byte aligned), zero at creation
+    unsigned* tickets;      // 64-bit grid-barrier arrival counters (h, LoPA's u, the union masks), zero at creation
     void* y;                // [n][d] T
     const uint32_t* hot;    // [ceil(d_ff / 32)] heavy-hitter channel bits, or NULL
     int dense;              // dense FFN (dense gate): every channel, W_up rows streamed with the gate's
@@ -295,6 +296,7 @@ enum TcMode {
 struct alignas(64) TcParams {
     CUtensorMap ta;         // A operand: weight rows, tile box 64 x 128 (down: W_down, box 64 x 64)
     CUtensorMap tb;         // B operand: token rows, tile box 64 x nb
+    CUtensorMap tg;         // gather: the A weights again with a one-row box (W_up, or W_down)
     int mode;
     int m_total;            // output rows: gate rows, d_ff (up), d (down)
     int k_total;            // contraction length of gate and up
@@ -315,7 +317,8 @@ struct alignas(64) TcParams {
     uint32_t* ubits;        // gate: union bitmap out (threshold), zeroed (top-K); up, down: read
     uint32_t* selbits;      // gate, threshold: per-token selection bits [n][selw] (bit k: z[t,k] > tau), or NULL
     int selw;               // words per token row of selbits (ceil(d_ff / 32))
-    int gather;             // up, down: gather the union's channel rows (ta is a one-row-box map) in list order
+    int gather;             // up, down: gather the union's channel rows (tg) in list order when the union is
+                            // under half the channels, else read whole 128-channel blocks (ta)
     const int* ulist;       // gather: the union's channels, ascending, padded with channel 0 to a multiple of 128
     const int* ucount;      // gather: the union's size
     float* part;            // [CTAs][128][nb] each CTA's parked stream-K part (room for [CTAs][2][128][256])
@@ -422,7 +425,7 @@ cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s, bool pdl);
 // The union bitmap (bit k of word k / 32) as an ascending channel list,
 // padded with channel 0 to a multiple of 128, and its size.
 cudaError_t launch_union_list(const uint32_t* ubits, int d_ff, int* list, int* count, cudaStream_t s, bool pdl);
-constexpr int kTcGatherMaxTokens = 3;  // batches up to this size gather the union's rows
+constexpr int kTcGatherMaxTokens = 16; // batches up to this size may gather the union's rows
 constexpr int kTcMaxTokens = 128;     // token columns of one tensor-core pass (hi/lo pairs fill N = 256)
 
 }  // namespace sffn

@@ -114,6 +114,82 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
     return v;
 }
 
+// One warp, once the CTA's selection is final: publish the CTA's union mask
+// (one bit per slot some token selected), arrive at the mask barrier, wait for
+// every CTA's mask (bounded), and write the union's channels in ascending
+// order to `list` (word order of the masks is channel order); scan_sh[6]
+// receives the union's size, or -1 if the wait gave up.
+__device__ __forceinline__ void build_union_list(uint32_t* umask, int cpb, unsigned long long wait_ns, int* status,
+                                                 int* hstatus, unsigned long long* bar, const uint8_t* flag,
+                                                 int nslots, int* list, uint32_t* gm, int* scan_sh) {
+    const int lane = threadIdx.x & 31;
+    const int G = gridDim.x, mwc = decode_mask_words(cpb);
+    for (int w = lane; w < mwc; w += 32) {
+        uint32_t m = 0u;
+        for (int i = 0; i < 32; ++i) {
+            const int sl = 32 * w + i;
+            if (sl < nslots && flag[sl]) m |= 1u << i;
+        }
+        umask[(size_t)blockIdx.x * mwc + w] = m;
+    }
+    __syncwarp();
+    int ok = 1;
+    if (lane == 0) {
+        __threadfence();                                  // release: the mask first
+        const unsigned long long target = grid_arrive(bar + 2, G);
+        const unsigned long long t0 = globaltimer_ns();
+        unsigned backoff = 32;
+        while (ld_acquire_u64(bar + 2) < target) {
+            if (globaltimer_ns() - t0 > wait_ns) {
+                raise_status(status, hstatus, kStatusWaitTimeout);
+                ok = 0;
+                break;
+            }
+            __nanosleep(backoff);
+            if (backoff < 256) backoff <<= 1;
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+        if (lane == 0) scan_sh[6] = -1;
+        return;
+    }
+    __threadfence();
+    const int nw = G * mwc;
+    // every CTA's mask words: 16 loads in flight per lane before any store
+    for (int i0 = lane; i0 < nw; i0 += 32 * 16) {
+        uint32_t v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] = i0 + 32 * u < nw ? __ldcg(umask + i0 + 32 * u) : 0u;
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+            if (i0 + 32 * u < nw) gm[i0 + 32 * u] = v[u];
+    }
+    __syncwarp();
+    const int per = (nw + 31) / 32;
+    const int wa = min(nw, lane * per), wb = min(nw, wa + per);
+    int c = 0;
+    for (int i = wa; i < wb; ++i) c += __popc(gm[i]);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    int pos = incl - c;
+    for (int i = wa; i < wb; ++i) {
+        uint32_t m = gm[i];
+        const int b = i / mwc, base = b * cpb + 32 * (i - b * mwc);
+        while (m) {
+            list[pos++] = base + __ffs(m) - 1;
+            m &= m - 1u;
+        }
+    }
+    const int U = __shfl_sync(0xffffffffu, incl, 31);
+    __syncwarp();
+    if (lane == 0) scan_sh[6] = U;
+}
+
 template <class T, int NT, int GATE>
 __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p) {
     constexpr int V = Elem<T>::kVec;
@@ -123,6 +199,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     const int nslots = max(0, min(p.cpb, p.d_ff - c0));
     const int n = p.n;                                  // n <= NT
     const DecodeSmem L = decode_smem_layout(NT, p.d, p.r, GATE, p.cpb, p.mw, p.sb, p.nb, V, gridDim.x);
+    const DecodeTail TLd = decode_tail_layout(NT, p.cpb, V, gridDim.x);
     float* xs = reinterpret_cast<float*>(smem + L.xs);
     float* us = reinterpret_cast<float*>(smem + L.us);
     float* zpart = reinterpret_cast<float*>(smem + L.zpart);
@@ -137,7 +214,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     float* hu = reinterpret_cast<float*>(smem + L.hu);           // hot channels' up dots
     uint8_t* hrdy = reinterpret_cast<uint8_t*>(smem + L.hrdy);   // ... and whether each is in
     int* scan_sh = reinterpret_cast<int*>(smem + L.scan);
-    // grid-barrier arrival counters: [0] the partials of y, [1] LoPA's stage 1
+    // grid-barrier arrival counters: [0] h published, [1] LoPA's stage 1, [2] union masks published
     unsigned long long* bar = reinterpret_cast<unsigned long long*>(p.tickets);
     const bool streamer = warp < kDecStreamWarps;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + (streamer ? warp : 0) * p.nb;
@@ -209,9 +286,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             fence_mbar_init();
         }
         __syncwarp();
-        // Weights never depend on an earlier kernel: fill the ring before the
-        // PDL wait, so the pieces land while the previous kernel finishes.
-        while (issued < min(p.nb, wcount)) issue_next();
+        // Weights never depend on an earlier kernel: the first piece goes out
+        // before the PDL wait, so it lands while the previous kernel finishes;
+        // the rest of the ring follows x, which then does not queue behind a
+        // full ring of weight traffic.
+        while (issued < min(1, wcount)) issue_next();
         __syncwarp();
     }
     // LoPA: this CTA's rows of A^T (stage 1) into L2 as well
@@ -309,10 +388,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         if (dense) {
             flag[s] = 1;
             smask[s * p.mw] = (1u << n) - 1u;
-            bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
         } else if (tokmask) {
             flag[s] = 1;
             smask[s * p.mw] = tokmask;                   // n <= 4: tokens sit in mask word 0
+            // both rows of the channel start towards L2 now: the up dot of a
+            // channel queued behind others then reads its W_up row from L2
+            const bool hot = p.hot && ((__ldg(p.hot + ((c0 + s) >> 5)) >> ((c0 + s) & 31)) & 1u);
+            if (!hot) bulk_prefetch_l2(wup + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
             bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
             const int slot = atomicAdd(ctr + kQueueTail, 1);
             __threadfence_block();
@@ -389,9 +471,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                 mbar_wait_warp(bars + (q % p.nb), (uint32_t)((q / p.nb) & 1));
         }
         __syncwarp();
+        int last = 0;
         if (lane == 0) {
             __threadfence_block();
-            atomicAdd(ctr + kGateDone, 1);
+            last = atomicAdd(ctr + kGateDone, 1) == kDecStreamWarps - 1;
+        }
+        if (!dense && __shfl_sync(0xffffffffu, last, 0)) {
+            // The CTA's selection is final: publish its union mask, arrive at
+            // the mask barrier, and build the union's ascending channel list
+            // while the other warps finish the up dots.
+            __threadfence_block();
+            build_union_list(p.umask, p.cpb, p.wait_ns, p.status, p.hstatus, bar, flag, nslots,
+                             reinterpret_cast<int*>(smem + L.bufs + TLd.list),
+                             reinterpret_cast<uint32_t*>(smem + L.bufs + TLd.masks), scan_sh);
         }
     }
 
@@ -464,26 +556,141 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     }
     __syncthreads();
 
-    // ---- publish this CTA's part of the union: one mask bit per slot that
-    // some token selected, and h for those slots (every token; 0 for a token
-    // that did not select the channel)
-    const int mwc = decode_mask_words(p.cpb);
-    for (int w = threadIdx.x; w < mwc; w += kDecThreads) {
-        uint32_t m = 0u;
-        for (int i = 0; i < 32; ++i) {
-            const int sl = 32 * w + i;
-            if (sl < nslots && flag[sl]) m |= 1u << i;
+    if (dense) {
+        // ---- dense FFN: every slot, in ascending order.  Each thread adds, for
+        // its 16-byte column chunks, h_k W_down[k, :] over the CTA's rows (read
+        // straight from HBM with 8 rows in flight), stores the CTA's fp32
+        // partial of y, and after a grid barrier every CTA sums one column
+        // slice of y over the partials in CTA order.
+        constexpr int UBD = 8;
+        const int cpd = p.d / V;                          // 16-byte chunks per output row
+        for (int cch = threadIdx.x; cch < cpd; cch += kDecThreads) {
+            float2 acc[NT][V / 2];
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < V / 2; ++e) acc[t][e] = make_float2(0.f, 0.f);
+            for (int s0 = 0; s0 < nslots; s0 += UBD) {
+                uint4 w[UBD];
+#pragma unroll
+                for (int u2 = 0; u2 < UBD; ++u2)
+                    w[u2] = s0 + u2 < nslots ? ld_stream(wdn + (size_t)(c0 + s0 + u2) * p.d + (size_t)cch * V)
+                                             : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int u2 = 0; u2 < UBD; ++u2) {
+                    if (s0 + u2 < nslots) {
+                        float wf[V];
+                        unpack<T>(w[u2], wf);
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) {
+                            const float h = hs[(s0 + u2) * NT + t];
+                            const float2 hh = make_float2(h, h);
+#pragma unroll
+                            for (int e = 0; e < V / 2; ++e)
+                                acc[t][e] = __ffma2_rn(make_float2(wf[2 * e], wf[2 * e + 1]), hh, acc[t][e]);
+                        }
+                    }
+                }
+            }
+            for (int t = 0; t < n; ++t) {
+                float* dst = p.part + ((size_t)blockIdx.x * n + t) * p.d + (size_t)cch * V;
+#pragma unroll
+                for (int e = 0; e < V / 2; e += 2)
+                    *reinterpret_cast<float4*>(dst + 2 * e) =
+                        make_float4(acc[t][e].x, acc[t][e].y, acc[t][e + 1].x, acc[t][e + 1].y);
+            }
         }
-        p.umask[(size_t)blockIdx.x * mwc + w] = m;
+        const int G = gridDim.x;
+        const int cps = decode_slice_chunks(p.d, V, G);
+        const int col0 = blockIdx.x * cps * V;
+        __syncthreads();
+        unsigned long long target = 0ull;
+        if (threadIdx.x == 0) {
+            __threadfence();                              // release: the CTA's partial first
+            if (col0 < p.d) target = grid_arrive(bar, G) + (unsigned long long)p.bar_extra;
+            else atomicAdd(bar, 1ull);
+        }
+        // every slot is listed, for sffn_get_active only
+        for (int i = threadIdx.x; i < nslots; i += kDecThreads) {
+            p.lst_idx[c0 + i] = c0 + i;
+            for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + i) * p.mw + w] = smask[i * p.mw + w];
+        }
+        if (threadIdx.x == 0) {
+            p.seg_count[blockIdx.x] = nslots;
+            int ok = 1;
+            if (col0 < p.d) {
+                const unsigned long long t0 = globaltimer_ns();
+                unsigned backoff = 32;
+                while (ld_acquire_u64(bar) < target) {
+                    if (globaltimer_ns() - t0 > p.wait_ns) {
+                        raise_status(p.status, p.hstatus, kStatusWaitTimeout);
+                        ok = 0;
+                        break;
+                    }
+                    __nanosleep(backoff);
+                    if (backoff < 256) backoff <<= 1;
+                }
+            }
+            scan_sh[2] = ok;
+        }
+        __syncthreads();
+        if (!scan_sh[2] || col0 >= p.d) return;
+        __threadfence();
+        // y[:, col0 : col0 + cps V] = sum over the G partials: thread (g, item)
+        // adds partials g, g + GR, ... in order, then the GR sums in order
+        const int q4 = min(cps * V, p.d - col0) / 4;      // float4 per token
+        const int items = n * q4;
+        const int GR = max(1, kDecThreads / items);
+        float4* red4 = reinterpret_cast<float4*>(smem + L.bufs);          // the idle ring
+        const int g = (int)threadIdx.x / items, item = (int)threadIdx.x - g * items;
+        if (g < GR) {
+            const int t = item / q4, c = col0 + (item - t * q4) * 4;
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            constexpr int UBS = 16;
+            for (int b0 = g; b0 < G; b0 += UBS * GR) {
+                float4 v[UBS];
+#pragma unroll
+                for (int u2 = 0; u2 < UBS; ++u2) {
+                    const int b = b0 + u2 * GR;
+                    v[u2] = b < G ? __ldcg(reinterpret_cast<const float4*>(p.part + ((size_t)b * n + t) * p.d + c))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u2 = 0; u2 < UBS; ++u2)
+                    if (b0 + u2 * GR < G) {
+                        sum.x += v[u2].x; sum.y += v[u2].y; sum.z += v[u2].z; sum.w += v[u2].w;
+                    }
+            }
+            red4[g * items + item] = sum;
+        }
+        __syncthreads();
+        if ((int)threadIdx.x < items) {
+            float4 sum = red4[threadIdx.x];
+            for (int q = 1; q < GR; ++q) {
+                const float4 v = red4[q * items + threadIdx.x];
+                sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+            }
+            const int t = (int)threadIdx.x / q4, c = col0 + ((int)threadIdx.x - t * q4) * 4;
+            T* dst = static_cast<T*>(p.y) + (size_t)t * p.d + c;
+            dst[0] = from_f32<T>(sum.x);
+            dst[1] = from_f32<T>(sum.y);
+            dst[2] = from_f32<T>(sum.z);
+            dst[3] = from_f32<T>(sum.w);
+        }
+        return;
     }
+
+    // ---- publish h for this CTA's union slots (every token; 0 for a token
+    // that did not select the channel); the union mask went out, and the
+    // union's list was built, when the CTA's selection became final
     for (int i = threadIdx.x; i < nslots * n; i += kDecThreads) {
         const int sl = i / n, t = i - sl * n;
         if (flag[sl]) p.lst_h[(size_t)(c0 + sl) * n + t] = hs[sl * NT + t];
     }
 
-    // ---- grid barrier: every CTA's mask and h are out.  All CTAs are
-    // resident (a cooperative launch of one CTA per SM), so the wait ends; it
-    // is bounded all the same.  A CTA without a column slice of y only arrives.
+    // ---- grid barrier: every CTA's h is out.  All CTAs are resident (a
+    // cooperative launch of one CTA per SM), so the wait ends; it is bounded
+    // all the same.  A CTA without a column slice of y only arrives.
     const int G = gridDim.x;
     const int cps = decode_slice_chunks(p.d, V, G);       // 16-byte chunks per column slice
     const int col0 = blockIdx.x * cps * V;
@@ -526,7 +733,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                 if (backoff < 256) backoff <<= 1;
             }
         }
-        scan_sh[2] = ok;
+        scan_sh[2] = ok && scan_sh[6] >= 0;
     }
     __syncthreads();
     if (!scan_sh[2] || col0 >= p.d) return;
@@ -535,31 +742,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     // ---- y[:, col0 : col0 + cps V] = sum over the union, in ascending channel
     // order, of h[k] W_down[k, slice].  The W_down rows were pulled into L2
     // when their channels were selected, so the slices come from L2.
-    const DecodeTail TL = decode_tail_layout(NT, p.cpb, V, G);
-    uint32_t* gm = reinterpret_cast<uint32_t*>(smem + L.bufs + TL.masks);     // [G][mwc]
-    int* list = reinterpret_cast<int*>(smem + L.bufs + TL.list);              // [<= d_ff]
-    float* red = reinterpret_cast<float*>(smem + L.bufs + TL.red);            // [groups][NT][slice]
-    float* red2 = reinterpret_cast<float*>(smem + L.bufs + TL.red2);          // [kDecThreads]
-    const int nw = G * mwc;
-    for (int i = threadIdx.x; i < nw; i += kDecThreads) gm[i] = __ldcg(p.umask + i);
-    __syncthreads();
-    // the union's channels in ascending order: word i is CTA i / mwc's slots
-    // 32 (i % mwc) .. + 31, so word order is channel order
-    const int per = (nw + kDecThreads - 1) / kDecThreads;
-    const int wa = min(nw, (int)threadIdx.x * per), wb = min(nw, wa + per);
-    int cw = 0;
-    for (int i = wa; i < wb; ++i) cw += __popc(gm[i]);
-    int U = 0;
-    int pos = block_exclusive_scan(cw, &U, scan_sh + 48);
-    for (int i = wa; i < wb; ++i) {
-        uint32_t m = gm[i];
-        const int b = i / mwc, base = b * p.cpb + 32 * (i - b * mwc);
-        while (m) {
-            list[pos++] = base + __ffs(m) - 1;
-            m &= m - 1u;
-        }
-    }
-    __syncthreads();
+    const int* list = reinterpret_cast<const int*>(smem + L.bufs + TLd.list);   // [U], ascending
+    float* red = reinterpret_cast<float*>(smem + L.bufs + TLd.red);            // [groups][NT][slice]
+    float* red2 = reinterpret_cast<float*>(smem + L.bufs + TLd.red2);          // [kDecThreads]
+    const int U = scan_sh[6];
 
     // thread (group g, chunk cc): rows g, g + NG, ... of the list, 16 bytes each
     const int NG = kDecThreads / cps;
@@ -571,7 +757,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     for (int t = 0; t < NT; ++t)
 #pragma unroll
         for (int e = 0; e < V / 2; ++e) acc[t][e] = make_float2(0.f, 0.f);
-    constexpr int UB = 8;
+    constexpr int UB = NT == 1 ? 16 : 8;                  // a group's rows in flight: usually all of them
     for (int i0 = g; i0 < U; i0 += UB * NG) {
         uint4 w[UB];
         float hv[UB][NT];

@@ -15,24 +15,30 @@
 // selected are loaded once and shared by the tokens that selected them; a
 // token that did not select a channel gets a zero activation for it.
 //
-// Rows are skipped at the granularity of 128-channel blocks: the up and down
-// passes read every block holding at least one channel that some token of the
-// batch selected (each CTA finds them from the gate's union bitmap) (a channel of such a block that a token did not select gets
-// g = 0 for it).  With several independent tokens nearly every block holds one
-// (a block is skipped only if all its 128 channels stay inactive for every
-// token), so the batched passes read what a per-channel gather would, in whole
-// tiles the TMA engine moves with one instruction.
+// The up and down passes read either whole 128-channel blocks or exactly the
+// union's rows.  Blocks: every block holding a channel that some token of the
+// batch selected (each CTA finds them from the gate's union bitmap; a channel
+// of such a block that no token selected gets g = 0), in tiles the TMA engine
+// moves with one instruction.  With several independent tokens nearly every
+// block holds one.  Gathered rows: a one-CTA kernel lists the union's channels
+// in ascending order, the A tiles are assembled four rows per TMA copy
+// (tile::gather4 with a one-row box, landing in the same 128-byte-swizzled
+// layout), h is kept in list order, and the down pass reduces over list
+// positions.  A gathered row moves at about half the rate of a block tile, so
+// a launch gathers only when the union holds under half of the channels
+// (batches of a few tokens at high sparsity), decided on the device from the
+// union's size.
 //
-// Kernel structure (one CTA per SM, 224 threads):
-//   warp 0     one thread: TMA 2-D tile copies (cp.async.bulk.tensor, 128-byte
-//              swizzle, no multicast) of the A and B tiles of the even 64-wide
-//              k-blocks into a ring of stages on mbarriers;
+// Kernel structure (one CTA per SM, 288 threads):
+//   warps 0, 6, 7, 8  one thread each: the TMA producers.  Producer p fills
+//              the ring stages of the k-blocks g with g % 4 == p: 2-D tile
+//              copies (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
+//              of the A and B tiles, or four-row gathers of A, on mbarriers;
 //   warp 1     allocates tensor memory; one thread issues tcgen05.mma (M = 128,
 //              N = token columns, K = 16 per instruction, bf16 in, fp32
 //              accumulate in tensor memory) and tcgen05.commit;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
-//              lanes), the mode's epilogue, stores;
-//   warp 6     one thread: the second TMA producer (the odd k-blocks).
+//              lanes), the mode's epilogue, stores.
 // Work is split stream-K: the (tile, k-block) iterations are cut into one
 // contiguous range per CTA, so every SM streams the same number of weight
 // bytes.  A tile cut between CTAs is finished by the CTA holding its first
@@ -58,9 +64,9 @@ constexpr int kProdWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;        // epilogue warps 2..5
 constexpr int kEpi = 4;
-constexpr int kProdWarp2 = kEpiWarp0 + kEpi;   // second TMA producer (warp 6)
-constexpr int kProducers = 2;
-constexpr int kTcThreads = (kProdWarp2 + 1) * 32;
+constexpr int kProdWarp2 = kEpiWarp0 + kEpi;   // further TMA producers: warps 6, 7, ...
+constexpr int kProducers = 4;
+constexpr int kTcThreads = (kProdWarp2 + kProducers - 1) * 32;
 constexpr uint32_t kTileA = kBM * kBK * 2;   // 16 KB
 constexpr int kMaxStages = 12;
 constexpr int kMaxBlocks = 1024;    // 128-channel blocks (d_ff <= 131072)
@@ -81,6 +87,7 @@ struct TcShared {
     int reducer;
     int wcount[kTcThreads / 32];
     int ucount;             // gather: the union's size
+    int gmode;              // this launch gathers rows (the union is under half the channels)
     int blk[kMaxBlocks];    // up/down: the active 128-channel blocks
     uint64_t ibar[kIdxSlots];
     alignas(16) int idx[kIdxSlots][kBM];   // gather: channel indices of one k-block's rows
@@ -221,16 +228,16 @@ struct Problem {
     long long I, it0, it1;
 };
 
-// nblk: the active 128-channel blocks, or with gather the union's size.
-__device__ __forceinline__ Problem make_problem(const TcParams& p, int nblk) {
+// nblk: the active 128-channel blocks, or when gathering the union's size.
+__device__ __forceinline__ Problem make_problem(const TcParams& p, int nblk, bool gmode = false) {
     Problem q;
     q.nblk = nblk;
     if (p.mode == kTcUp) {
-        q.T = p.gather ? (nblk + kBM - 1) / kBM : q.nblk;
+        q.T = gmode ? (nblk + kBM - 1) / kBM : q.nblk;
         q.KB = (p.k_total + kBK - 1) / kBK;
     } else if (p.mode == kTcDown) {
         q.T = (p.m_total + kBM - 1) / kBM;
-        q.KB = p.gather ? (nblk + kBK - 1) / kBK : 2 * q.nblk;
+        q.KB = gmode ? (nblk + kBK - 1) / kBK : 2 * q.nblk;
     } else {
         q.T = (p.m_total + kBM - 1) / kBM;
         q.KB = (p.k_total + kBK - 1) / kBK;
@@ -284,9 +291,10 @@ __device__ void prefetch_first_tiles(const TcParams& p, int count) {
 
 // Producer `pr` of kProducers fills the stages of the k-blocks g with
 // g % kProducers == pr.  One thread issuing every copy of an SM's stream keeps
-// only about three quarters of HBM bandwidth busy; two threads in different
-// warps, taking alternate k-blocks of the same ring, reach the copy peak.  The
-// ring stays one sequence for the MMA issuer.  (A producer waits for stage
+// only about three quarters of HBM bandwidth busy; threads in different warps,
+// taking turns over the k-blocks of the same ring, reach the copy peak, and
+// four of them keep the 32 gathers of a gathered stage coming.  The ring stays
+// one sequence for the MMA issuer.  (A producer waits for stage
 // g - S to be consumed; with kProducers <= S the parity wait cannot be a phase
 // behind.)
 // Gather: k-block g of the CTA's range is iteration it0 + g, i.e. tile
@@ -341,15 +349,15 @@ __device__ void run_producer_gather(const TcParams& p, const Problem& q, unsigne
 #pragma unroll 4
             for (int i = 0; i < kBK / 4; ++i) {
                 const int4 r = rows[i];
-                tma_gather4(sA + i * 512, &p.ta, m0, r, &sh->full[st], pol_w);
-                if (hi) tma_gather4(sA + 8192 + i * 512, &p.ta, m0 + 64, r, &sh->full[st], pol_w);
+                tma_gather4(sA + i * 512, &p.tg, m0, r, &sh->full[st], pol_w);
+                if (hi) tma_gather4(sA + 8192 + i * 512, &p.tg, m0 + 64, r, &sh->full[st], pol_w);
             }
             tma_tile(sB, &p.tb, kb * kBK, 0, &sh->full[st], pol_b);   // h, compacted by list position
         } else {
             // K-major A: the tile's 128 channels (rows of W_up) x 64 k
             mbar_expect_tx(&sh->full[st], tx);
 #pragma unroll 4
-            for (int i = 0; i < kBM / 4; ++i) tma_gather4(sA + i * 512, &p.ta, kb * kBK, rows[i], &sh->full[st], pol_w);
+            for (int i = 0; i < kBM / 4; ++i) tma_gather4(sA + i * 512, &p.tg, kb * kBK, rows[i], &sh->full[st], pol_w);
             tma_tile(sB, &p.tb, kb * kBK, 0, &sh->full[st], pol_b);
         }
         // this thread's reads of the index block come before the async copy that refills it
@@ -361,7 +369,7 @@ __device__ void run_producer_gather(const TcParams& p, const Problem& q, unsigne
 
 __device__ void run_producer(const TcParams& p, const Problem& q, unsigned char* stages, uint32_t stage_bytes,
                              TcShared* sh, int pr) {
-    if (p.gather) {
+    if (sh->gmode) {
         run_producer_gather(p, q, stages, stage_bytes, sh, pr);
         return;
     }
@@ -625,9 +633,9 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
         // up: output row `row` of the tile is channel m, written at column mo
         // (gather: list position mo = the tile's first position + row, whose
         // channel is the list entry, none past the union's size)
-        const int m0 = p.mode == kTcUp ? (p.gather ? s.t * kBM : sh->blk[s.t] * kBM) : s.t * kBM;
+        const int m0 = p.mode == kTcUp ? (sh->gmode ? s.t * kBM : sh->blk[s.t] * kBM) : s.t * kBM;
         const int mo = m0 + row;
-        const int m = (p.mode == kTcUp && p.gather) ? (mo < sh->ucount ? __ldcg(p.ulist + mo) : -1) : mo;
+        const int m = (p.mode == kTcUp && sh->gmode) ? (mo < sh->ucount ? __ldcg(p.ulist + mo) : -1) : mo;
         UpG g;
         if (p.mode == kTcUp && owner) up_g_load(p, m, cols, g);   // in flight during the mainloop
         if (owner && !whole && !wait_parts(p, s.t, (unsigned)(c_last - c_first))) {
@@ -771,15 +779,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
 
-    if (warp == kProdWarp && (threadIdx.x & 31) == 0 && !p.gather) prefetch_first_tiles(p, p.stages);
+    if (warp == kProdWarp && (threadIdx.x & 31) == 0) prefetch_first_tiles(p, p.stages);
     griddep_launch_dependents();
     griddep_wait();
     int nblk = 0;
-    if (p.gather) {
-        // the union's size (its list was built by the previous kernel)
-        nblk = __ldcg(p.ucount);
-        if (threadIdx.x == 0) sh->ucount = nblk;
-        __syncthreads();
+    // Gathering the union's rows moves fewer bytes but at about half the rate
+    // of whole-block tiles (four rows per copy instead of 128), so it is taken
+    // only when the union holds under half of the channels.
+    const int U = p.gather ? __ldcg(p.ucount) : 0;
+    const bool gmode = p.gather && 2 * U < p.d_ff;
+    if (threadIdx.x == 0) {
+        sh->ucount = U;
+        sh->gmode = gmode ? 1 : 0;
+    }
+    __syncthreads();
+    if (gmode) {
+        nblk = U;                                      // its list was built by the previous kernel
     } else if (p.mode == kTcUp || p.mode == kTcDown) {
         // the 128-channel blocks holding a channel some token selected, from the union bitmap
         const int nbk = (p.d_ff + 127) / 128, nwords = (p.d_ff + 31) >> 5;
@@ -808,7 +823,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
             __syncthreads();
         }
     }
-    const Problem q = make_problem(p, nblk);
+    const Problem q = make_problem(p, nblk, gmode);
     if (p.mode == kTcDown && q.KB == 0) {
         // no channel is active for any token: y = 0
         bf16* y = static_cast<bf16*>(p.out);
@@ -820,8 +835,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
         }
     }
 
-    if (warp == kProdWarp || warp == kProdWarp2) {
-        if ((threadIdx.x & 31) == 0) run_producer(p, q, stages, stage_bytes, sh, warp == kProdWarp ? 0 : 1);
+    if (warp == kProdWarp || warp >= kProdWarp2) {
+        if ((threadIdx.x & 31) == 0)
+            run_producer(p, q, stages, stage_bytes, sh, warp == kProdWarp ? 0 : warp - kProdWarp2 + 1);
     } else if (warp == kMmaWarp) {
         if ((threadIdx.x & 31) == 0) run_mma(p, q, stages, stage_bytes, sh, tmem);
     } else {
@@ -897,8 +913,7 @@ cudaError_t launch_union_list(const uint32_t* ubits, int d_ff, int* list, int* c
 cudaError_t launch_tc(const TcParams& p_in, int grid, cudaStream_t s, bool pdl) {
     TcParams p = p_in;
     if (p.nb < 16 || p.nb > 256 || p.nb % 16 || (p.paired && 2 * p.npad != p.nb)) return cudaErrorInvalidValue;
-    if ((p.mode == kTcUp || p.mode == kTcDown) && !p.gather &&
-        ((p.d_ff + 127) / 128 > kMaxBlocks || (!p.ubits && !p.force_all)))
+    if ((p.mode == kTcUp || p.mode == kTcDown) && ((p.d_ff + 127) / 128 > kMaxBlocks || (!p.ubits && !p.force_all)))
         return cudaErrorInvalidValue;
     if (p.gather && (!p.ulist || !p.ucount || (p.mode != kTcUp && p.mode != kTcDown))) return cudaErrorInvalidValue;
     int st = 0;

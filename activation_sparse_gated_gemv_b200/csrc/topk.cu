@@ -233,202 +233,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const TopkParams p) {
     }
 }
 
-// Rows of at most KPT x 1024 channels: each thread keeps the keys of channels
-// tid, tid + 1024, ... in registers, so each pass of the same radix select
-// reads no memory.  A pass builds one shared 256-bin histogram: for top-K the
-// lanes of a warp holding the same digit are merged (__match_any_sync) and
-// their leader adds their count, so a warp issues one atomic per distinct
-// digit; top-p adds each key's integer mass.  One warp scans the bins (8 per
-// lane, descending) and picks the bin holding the boundary.  Ties at the
-// boundary key are taken from the lowest channel up, as in k_topk.
-template <int KPT>
-__global__ void __launch_bounds__(kTopkThreads) k_topk_fast(const TopkParams p) {
-    __shared__ unsigned hist[256];
-    __shared__ int sh[40];
-    __shared__ uint32_t s_prefix;
-    __shared__ unsigned s_remaining, s_binw;
-    __shared__ unsigned s_red[33];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const size_t row = (size_t)blockIdx.x * p.d_ff;
-    const float* z = p.zbuf + row;
-    const bool topp = p.mode == 1;
-
-    griddep_wait();
-    griddep_launch_dependents();
-    uint32_t key[KPT];
-    float zv[KPT];
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) {
-        const int k = threadIdx.x + i * kTopkThreads;
-        zv[i] = k < p.d_ff ? __ldcg(z + k) : 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) key[i] = order_key(topp ? zv[i] : silu_f(zv[i]));
-    auto valid = [&](int i) { return (int)threadIdx.x + i * kTopkThreads < p.d_ff; };
-
-    // top-p: the largest gate value and the total integer mass
-    float zmax = 0.f, scale = 0.f;
-    unsigned target = (unsigned)p.k;
-    if (topp) {
-        uint32_t mk = 0u;
-#pragma unroll
-        for (int i = 0; i < KPT; ++i)
-            if (valid(i)) mk = max(mk, key[i]);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) mk = max(mk, __shfl_xor_sync(0xffffffffu, mk, o));
-        if (lane == 0) s_red[warp] = mk;
-        __syncthreads();
-        if (warp == 0) {
-            uint32_t v = s_red[lane];
-#pragma unroll
-            for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (lane == 0) s_red[32] = v;
-        }
-        __syncthreads();
-        zmax = key_value(s_red[32]);
-        scale = (float)(1 << topp_scale_bits(p.d_ff));
-        __syncthreads();
-    }
-    auto mass_of = [&](uint32_t k) -> unsigned { return __float2uint_rn(expf(key_value(k) - zmax) * scale); };
-    if (topp) {
-        unsigned tm = 0u;
-#pragma unroll
-        for (int i = 0; i < KPT; ++i)
-            if (valid(i)) tm += mass_of(key[i]);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) tm += __shfl_xor_sync(0xffffffffu, tm, o);
-        if (lane == 0) s_red[warp] = tm;
-        __syncthreads();
-        if (warp == 0) {
-            unsigned v = s_red[lane];
-#pragma unroll
-            for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) s_red[32] = v;
-        }
-        __syncthreads();
-        const unsigned total = s_red[32];
-        target = (unsigned)min((double)total, ceil((double)p.p * (double)total));
-        __syncthreads();
-    }
-    const bool partial = topp ? target > 0u : (target > 0u && (int)target < p.d_ff);
-    uint32_t prefix = 0u, pmask = 0u;
-    unsigned remaining = target;
-    if (partial) {
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            if (threadIdx.x < 256) hist[threadIdx.x] = 0u;
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < KPT; ++i) {
-                const bool in = valid(i) && (key[i] & pmask) == prefix;
-                const unsigned dg = (key[i] >> shift) & 0xFFu;
-                if (topp) {
-                    if (in) {
-                        const unsigned m = mass_of(key[i]);
-                        if (m) atomicAdd(&hist[dg], m);
-                    }
-                } else {
-                    const unsigned grp = __match_any_sync(0xffffffffu, in ? dg : 256u + lane);
-                    if (in && lane == __ffs(grp) - 1) atomicAdd(&hist[dg], (unsigned)__popc(grp));
-                }
-            }
-            __syncthreads();
-            if (warp == 0) {
-                // lane l takes bins 255 - 8l .. 248 - 8l (descending), then an inclusive scan
-                unsigned c[8], tot = 0u;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    c[j] = hist[255 - (8 * lane + j)];
-                    tot += c[j];
-                }
-                unsigned incl = tot;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                unsigned before = incl - tot;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (c[j] > 0u && before < remaining && before + c[j] >= remaining) {
-                        s_prefix = prefix | ((uint32_t)(255 - (8 * lane + j)) << shift);
-                        s_remaining = remaining - before;
-                        s_binw = c[j];
-                    }
-                    before += c[j];
-                }
-            }
-            __syncthreads();
-            prefix = s_prefix;
-            remaining = s_remaining;
-            pmask |= 0xFFu << shift;
-        }
-    }
-    // Keys above `prefix` are all selected; of the keys equal to it, taken in
-    // ascending channel order: `remaining` (top-K) or enough to cover the
-    // remaining mass (top-p: equal keys weigh the same).  The last pass's bin
-    // holds exactly the keys equal to the boundary, so its weight gives their
-    // number.
-    unsigned take = remaining;
-    int nties = 0;
-    if (partial) {
-        const unsigned m_tie = topp ? mass_of(prefix) : 1u;
-        if (topp) take = m_tie ? (remaining + m_tie - 1u) / m_tie : 0u;
-        if (m_tie) {
-            nties = (int)(s_binw / m_tie);
-        } else {
-            int c = 0;
-#pragma unroll
-            for (int i = 0; i < KPT; ++i) c += valid(i) && key[i] == prefix;
-            int tot0 = 0;
-            block_exclusive_scan(c, &tot0, sh);
-            nties = tot0;
-        }
-    }
-    if (!partial || nties <= (int)take) {
-#pragma unroll
-        for (int i = 0; i < KPT; ++i) {
-            const int k = threadIdx.x + i * kTopkThreads;
-            bool sel = false;
-            if (k < p.d_ff) {
-                sel = partial ? key[i] >= prefix : (!topp && target > 0u);
-                const float gv = topp ? silu_f(key_value(key[i])) : key_value(key[i]);
-                p.sel[row + k] = sel ? 1 : 0;
-                p.gbuf[row + k] = sel ? gv : 0.f;
-            }
-            // a warp's 32 lanes hold 32 consecutive channels: one bitmap word
-            const unsigned m = __ballot_sync(0xffffffffu, sel);
-            if (lane == 0 && m && p.ubits) atomicOr(&p.ubits[(warp * 32 + i * kTopkThreads) >> 5], m);
-        }
-        return;
-    }
-    // More ties than places: rank them in channel order over contiguous runs
-    // of channels (keys recomputed from z for the run).
-    auto key_of = [&](int k) { return order_key(topp ? z[k] : silu_f(z[k])); };
-    const int per = (p.d_ff + kTopkThreads - 1) / kTopkThreads;
-    const int k0 = min(p.d_ff, (int)threadIdx.x * per), k1 = min(p.d_ff, k0 + per);
-    int ties = 0;
-    for (int k = k0; k < k1; ++k) ties += key_of(k) == prefix;
-    int tot = 0;
-    int rank = block_exclusive_scan(ties, &tot, sh);
-    for (int k = k0; k < k1; ++k) {
-        const uint32_t kk = key_of(k);
-        bool sel = kk > prefix;
-        if (kk == prefix) sel = rank++ < (int)take;
-        p.sel[row + k] = sel ? 1 : 0;
-        p.gbuf[row + k] = sel ? (topp ? silu_f(key_value(kk)) : key_value(kk)) : 0.f;
-        if (sel && p.ubits) atomicOr(&p.ubits[k >> 5], 1u << (k & 31));
-    }
-}
-
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s, bool pdl) {
-    if (p.d_ff <= 8 * kTopkThreads) {
-        const int kpt = (p.d_ff + kTopkThreads - 1) / kTopkThreads;
-        if (kpt <= 1) return launch_ex(k_topk_fast<1>, dim3(p.n), dim3(kTopkThreads), 0, s, pdl, p);
-        if (kpt <= 2) return launch_ex(k_topk_fast<2>, dim3(p.n), dim3(kTopkThreads), 0, s, pdl, p);
-        if (kpt <= 4) return launch_ex(k_topk_fast<4>, dim3(p.n), dim3(kTopkThreads), 0, s, pdl, p);
-        return launch_ex(k_topk_fast<8>, dim3(p.n), dim3(kTopkThreads), 0, s, pdl, p);
-    }
     const size_t whist = 32 * 256 * sizeof(unsigned);
     const size_t keys = (size_t)p.d_ff * sizeof(uint32_t);
     if (keys <= kTopkSmemKeys) {
