@@ -114,82 +114,6 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
     return v;
 }
 
-// One warp, once the CTA's selection is final: publish the CTA's union mask
-// (one bit per slot some token selected), arrive at the mask barrier, wait for
-// every CTA's mask (bounded), and write the union's channels in ascending
-// order to `list` (word order of the masks is channel order); scan_sh[6]
-// receives the union's size, or -1 if the wait gave up.
-__device__ __forceinline__ void build_union_list(uint32_t* umask, int cpb, unsigned long long wait_ns, int* status,
-                                                 int* hstatus, unsigned long long* bar, const uint8_t* flag,
-                                                 int nslots, int* list, uint32_t* gm, int* scan_sh) {
-    const int lane = threadIdx.x & 31;
-    const int G = gridDim.x, mwc = decode_mask_words(cpb);
-    for (int w = lane; w < mwc; w += 32) {
-        uint32_t m = 0u;
-        for (int i = 0; i < 32; ++i) {
-            const int sl = 32 * w + i;
-            if (sl < nslots && flag[sl]) m |= 1u << i;
-        }
-        umask[(size_t)blockIdx.x * mwc + w] = m;
-    }
-    __syncwarp();
-    int ok = 1;
-    if (lane == 0) {
-        __threadfence();                                  // release: the mask first
-        const unsigned long long target = grid_arrive(bar + 2, G);
-        const unsigned long long t0 = globaltimer_ns();
-        unsigned backoff = 32;
-        while (ld_acquire_u64(bar + 2) < target) {
-            if (globaltimer_ns() - t0 > wait_ns) {
-                raise_status(status, hstatus, kStatusWaitTimeout);
-                ok = 0;
-                break;
-            }
-            __nanosleep(backoff);
-            if (backoff < 256) backoff <<= 1;
-        }
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) {
-        if (lane == 0) scan_sh[6] = -1;
-        return;
-    }
-    __threadfence();
-    const int nw = G * mwc;
-    // every CTA's mask words: 16 loads in flight per lane before any store
-    for (int i0 = lane; i0 < nw; i0 += 32 * 16) {
-        uint32_t v[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] = i0 + 32 * u < nw ? __ldcg(umask + i0 + 32 * u) : 0u;
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-            if (i0 + 32 * u < nw) gm[i0 + 32 * u] = v[u];
-    }
-    __syncwarp();
-    const int per = (nw + 31) / 32;
-    const int wa = min(nw, lane * per), wb = min(nw, wa + per);
-    int c = 0;
-    for (int i = wa; i < wb; ++i) c += __popc(gm[i]);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    int pos = incl - c;
-    for (int i = wa; i < wb; ++i) {
-        uint32_t m = gm[i];
-        const int b = i / mwc, base = b * cpb + 32 * (i - b * mwc);
-        while (m) {
-            list[pos++] = base + __ffs(m) - 1;
-            m &= m - 1u;
-        }
-    }
-    const int U = __shfl_sync(0xffffffffu, incl, 31);
-    __syncwarp();
-    if (lane == 0) scan_sh[6] = U;
-}
-
 template <class T, int NT, int GATE>
 __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p) {
     constexpr int V = Elem<T>::kVec;
@@ -214,7 +138,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     float* hu = reinterpret_cast<float*>(smem + L.hu);           // hot channels' up dots
     uint8_t* hrdy = reinterpret_cast<uint8_t*>(smem + L.hrdy);   // ... and whether each is in
     int* scan_sh = reinterpret_cast<int*>(smem + L.scan);
-    // grid-barrier arrival counters: [0] h published, [1] LoPA's stage 1, [2] union masks published
+    // grid-barrier arrival counters: [0] masks and h published, [1] LoPA's stage 1
     unsigned long long* bar = reinterpret_cast<unsigned long long*>(p.tickets);
     const bool streamer = warp < kDecStreamWarps;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + (streamer ? warp : 0) * p.nb;
@@ -391,10 +315,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         } else if (tokmask) {
             flag[s] = 1;
             smask[s * p.mw] = tokmask;                   // n <= 4: tokens sit in mask word 0
-            // both rows of the channel start towards L2 now: the up dot of a
-            // channel queued behind others then reads its W_up row from L2
-            const bool hot = p.hot && ((__ldg(p.hot + ((c0 + s) >> 5)) >> ((c0 + s) & 31)) & 1u);
-            if (!hot) bulk_prefetch_l2(wup + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
             bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
             const int slot = atomicAdd(ctr + kQueueTail, 1);
             __threadfence_block();
@@ -471,19 +391,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                 mbar_wait_warp(bars + (q % p.nb), (uint32_t)((q / p.nb) & 1));
         }
         __syncwarp();
-        int last = 0;
         if (lane == 0) {
             __threadfence_block();
-            last = atomicAdd(ctr + kGateDone, 1) == kDecStreamWarps - 1;
-        }
-        if (!dense && __shfl_sync(0xffffffffu, last, 0)) {
-            // The CTA's selection is final: publish its union mask, arrive at
-            // the mask barrier, and build the union's ascending channel list
-            // while the other warps finish the up dots.
-            __threadfence_block();
-            build_union_list(p.umask, p.cpb, p.wait_ns, p.status, p.hstatus, bar, flag, nslots,
-                             reinterpret_cast<int*>(smem + L.bufs + TLd.list),
-                             reinterpret_cast<uint32_t*>(smem + L.bufs + TLd.masks), scan_sh);
+            atomicAdd(ctr + kGateDone, 1);
         }
     }
 
@@ -680,17 +590,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         return;
     }
 
-    // ---- publish h for this CTA's union slots (every token; 0 for a token
-    // that did not select the channel); the union mask went out, and the
-    // union's list was built, when the CTA's selection became final
+    // ---- publish this CTA's part of the union: one mask bit per slot that
+    // some token selected, and h for those slots (every token; 0 for a token
+    // that did not select the channel)
+    const int mwc = decode_mask_words(p.cpb);
+    for (int w = threadIdx.x; w < mwc; w += kDecThreads) {
+        uint32_t m = 0u;
+        for (int i = 0; i < 32; ++i) {
+            const int sl = 32 * w + i;
+            if (sl < nslots && flag[sl]) m |= 1u << i;
+        }
+        p.umask[(size_t)blockIdx.x * mwc + w] = m;
+    }
     for (int i = threadIdx.x; i < nslots * n; i += kDecThreads) {
         const int sl = i / n, t = i - sl * n;
         if (flag[sl]) p.lst_h[(size_t)(c0 + sl) * n + t] = hs[sl * NT + t];
     }
 
-    // ---- grid barrier: every CTA's h is out.  All CTAs are resident (a
-    // cooperative launch of one CTA per SM), so the wait ends; it is bounded
-    // all the same.  A CTA without a column slice of y only arrives.
+    // ---- grid barrier: every CTA's mask and h are out.  All CTAs are
+    // resident (a cooperative launch of one CTA per SM), so the wait ends; it
+    // is bounded all the same.  A CTA without a column slice of y only arrives.
     const int G = gridDim.x;
     const int cps = decode_slice_chunks(p.d, V, G);       // 16-byte chunks per column slice
     const int col0 = blockIdx.x * cps * V;
@@ -733,7 +652,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
                 if (backoff < 256) backoff <<= 1;
             }
         }
-        scan_sh[2] = ok && scan_sh[6] >= 0;
+        scan_sh[2] = ok;
     }
     __syncthreads();
     if (!scan_sh[2] || col0 >= p.d) return;
@@ -742,10 +661,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     // ---- y[:, col0 : col0 + cps V] = sum over the union, in ascending channel
     // order, of h[k] W_down[k, slice].  The W_down rows were pulled into L2
     // when their channels were selected, so the slices come from L2.
-    const int* list = reinterpret_cast<const int*>(smem + L.bufs + TLd.list);   // [U], ascending
+    uint32_t* gm = reinterpret_cast<uint32_t*>(smem + L.bufs + TLd.masks);     // [G][mwc]
+    int* list = reinterpret_cast<int*>(smem + L.bufs + TLd.list);             // [<= G cpb], ascending
     float* red = reinterpret_cast<float*>(smem + L.bufs + TLd.red);            // [groups][NT][slice]
     float* red2 = reinterpret_cast<float*>(smem + L.bufs + TLd.red2);          // [kDecThreads]
-    const int U = scan_sh[6];
+    // every CTA's union mask, all loads in flight before any store
+    const int nw = G * mwc;
+    {
+        constexpr int UM = 4;
+        uint32_t v[UM];
+#pragma unroll
+        for (int u = 0; u < UM; ++u) {
+            const int i = (int)threadIdx.x + u * kDecThreads;
+            v[u] = i < nw ? __ldcg(p.umask + i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < UM; ++u) {
+            const int i = (int)threadIdx.x + u * kDecThreads;
+            if (i < nw) gm[i] = v[u];
+        }
+        for (int i = (int)threadIdx.x + UM * kDecThreads; i < nw; i += kDecThreads) gm[i] = __ldcg(p.umask + i);
+    }
+    __syncthreads();
+    // the union's channels in ascending order: word i is CTA i / mwc's slots
+    // 32 (i % mwc) .. + 31, so word order is channel order
+    const int per = (nw + kDecThreads - 1) / kDecThreads;
+    const int wa = min(nw, (int)threadIdx.x * per), wb = min(nw, wa + per);
+    int cw = 0;
+    for (int i = wa; i < wb; ++i) cw += __popc(gm[i]);
+    int U = 0;
+    int pos = block_exclusive_scan(cw, &U, scan_sh + 48);
+    for (int i = wa; i < wb; ++i) {
+        uint32_t m = gm[i];
+        const int b = i / mwc, base = b * p.cpb + 32 * (i - b * mwc);
+        while (m) {
+            list[pos++] = base + __ffs(m) - 1;
+            m &= m - 1u;
+        }
+    }
+    __syncthreads();
 
     // thread (group g, chunk cc): rows g, g + NG, ... of the list, 16 bytes each
     const int NG = kDecThreads / cps;

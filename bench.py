@@ -70,7 +70,12 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--dense-step", action="store_true",
+                    help="time the library's dense FFN as the step (the comparator on its own, e.g. for ncu)")
     ap.add_argument("--no-hot", action="store_true", help="heavy7b: run without the heavy-hitter set")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="weight copies rotated across steps (0: enough to exceed 3x the L2); 1 keeps ncu "
+                         "captures small (ncu flushes the caches between its passes anyway)")
     ap.add_argument("--json-out", default="")
     return ap.parse_args()
 
@@ -352,9 +357,9 @@ def main():
         unions.append(probe.active(wl.n)[1])
     probe.close()
     union = statistics.mean(unions)
-    fwd_bytes = algorithmic_bytes(wl, union)
+    fwd_bytes = dense_bytes(wl) if a.dense_step else algorithmic_bytes(wl, union)
     R = max(2, math.ceil(3 * l2 / fwd_bytes))
-    R = min(R, 64)
+    R = min(R, 64) if a.replicas <= 0 else a.replicas
     ffns = []
     for i in range(R):
         f = sffn.SparseFFN(wl.d, wl.d_ff, wl.r, wl.n, wl.dtype, device=local)
@@ -366,7 +371,8 @@ def main():
     stream = torch.cuda.Stream(dev)
 
     def step(i, dense=False):
-        ffns[i % R].forward(xs[i % P], gate=wl.gate, out=ys[i % P], dense=dense, stream=stream, **sel)
+        ffns[i % R].forward(xs[i % P], gate=wl.gate, out=ys[i % P], dense=dense or a.dense_step, stream=stream,
+                            **sel)
 
     def capture(first, count, dense=False):
         g = torch.cuda.CUDAGraph()
@@ -496,7 +502,9 @@ def main():
     dom_name = max(per_name, key=per_name.get)
     peaks, peak_kind = measured_peaks()
     w = bytes_per_elem(wl.dtype)
-    if dom_name == "decode_fused":
+    if dom_name == "decode_dense":
+        dom_bytes = dense_bytes(wl)
+    elif dom_name == "decode_fused":
         # everything (LoPA's stage 1 runs inside the same launch)
         dom_bytes = algorithmic_bytes(wl, union) - (
             wl.d * wl.r * bytes_per_elem(wl.dtype) if "lopa_u" in kernel_names else 0)
@@ -518,6 +526,8 @@ def main():
         dom_bytes = wl.n * wl.d_ff * 4                     # z read (the masks written are overhead)
     elif dom_name == "tc_lopa_u":
         dom_bytes = wl.d * wl.r * w + wl.n * wl.d * w
+    elif dom_name == "union_list":
+        dom_bytes = wl.d_ff // 8 + 4 * union                # union bitmap read, list written
     else:
         dom_bytes = wl.d * wl.r * w + wl.n * wl.d * w
     # Stage events put an event node between kernels, which stops the next
@@ -624,10 +634,14 @@ def main():
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": wl.describe() + (" (hot set off)" if wl.hot_frac > 0.0 and hot is None else ""),
+            "config": {"workload": wl.describe() + (" (hot set off)" if wl.hot_frac > 0.0 and hot is None else "")
+                       + (" -- DENSE FFN comparator as the step" if a.dense_step else ""),
                        "tokens_per_step": wl.n, "parallelism": f"replicas x{world}",
-                       "l2": f"{R} weight replicas rotated ({R * dense_bytes(wl) / 1e9:.2f} GB > L2 "
-                             f"{l2 / 2**20:.0f} MiB), no step reuses L2-resident weights",
+                       "l2": (f"{R} weight replicas rotated ({R * dense_bytes(wl) / 1e9:.2f} GB > L2 "
+                              f"{l2 / 2**20:.0f} MiB), no step reuses L2-resident weights"
+                              if R * fwd_bytes >= 3 * l2 else
+                              f"{R} weight replica(s) only ({R * fwd_bytes / 1e6:.0f} MB touched per cycle, "
+                              f"L2 {l2 / 2**20:.0f} MiB): steps may reuse L2-resident weights (profiling runs)"),
                        "mean_union": union, "timed_with": "CUDA graphs of "
                        f"{G} steps, CUDA events on the launch stream, after one untimed replay of each graph "
                        f"and {pre_replays} untimed pre-roll replays (>= 50 ms) queued straight ahead of it"},

@@ -313,6 +313,43 @@ def test_moc_shape_topp(sffn, p):
     ffn.close()
 
 
+@pytest.mark.parametrize("n,d_ff", [(1, 1000), (6, 1000), (6, 5632)])
+def test_topk_and_topp_ties_go_to_the_lower_channel(sffn, n, d_ff):
+    """W_gate with every column equal gives every channel the same z (each dot
+    product is summed in the same order), so the whole row ties: top-K must
+    keep channels 0..K-1 and top-p the first ceil(p d_ff) channels (equal
+    masses).  Then half the columns equal: the ties at the boundary are ranked
+    by channel index."""
+    d = 64
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=71)
+    col = w["w_gate"][:, :1].clone()
+    w["w_gate"] = col.expand(d, d_ff).contiguous()
+    ffn = sffn.SparseFFN(d, d_ff, 0, n, "bf16")
+    ffn.set_weights(**w)
+    x = workloads.tokens(n, d, "bf16", seed=72)
+    k = d_ff * 3 // 10 + 1
+    ffn.forward(x.cuda(), select="topk", k=k)
+    sets, _ = ffn.active(n)
+    assert all(np.array_equal(s, np.arange(k)) for s in sets)
+    ffn.forward(x.cuda(), select="topp", p=0.25)
+    sets, _ = ffn.active(n)
+    m = math.ceil(0.25 * d_ff)
+    assert all(abs(len(s) - m) <= 1 and np.array_equal(s, np.arange(len(s))) for s in sets)
+    # half the channels tie (equal columns at the odd channels), the rest are distinct
+    wg = workloads.ffn_weights(d, d_ff, "bf16", seed=73)["w_gate"].clone()
+    wg[:, 1::2] = wg[:, 1:2]
+    w["w_gate"] = wg.contiguous()
+    ffn.set_weights(**w)
+    check_forward(ffn, w, x, "dense", "topk", k=k)
+    sets, _ = ffn.active(n)
+    tied = np.arange(1, d_ff, 2)
+    for t in range(n):
+        got = np.intersect1d(sets[t], tied)
+        # which tied channels are kept is fixed: the lowest ones
+        assert np.array_equal(got, tied[:len(got)])
+    ffn.close()
+
+
 def test_k_equals_d_ff_is_dense_swiglu(sffn):
     ffn, w, x = _small(sffn, d_ff=300)
     y = ffn.forward(x.cuda(), gate="dense", select="topk", k=300)
