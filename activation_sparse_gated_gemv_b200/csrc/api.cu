@@ -441,6 +441,10 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         h->inj_wait_ns = 0;
         dp.tickets = h->dbar; dp.y = out; dp.hot = h->hot_on && !dense ? h->hot : nullptr;
         dp.dense = dense ? 1 : 0;
+        // The sparse forward's down projection: each CTA's own rows into a
+        // partial of y (measured faster up to d = 4096), or the union gather by
+        // column slice (faster on the 70B shape, d = 8192).
+        dp.own_rows = c.d <= 4096 ? 1 : 0;
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
         set_name(h, launches, dense ? "decode_dense" : "decode_fused");
         record(h, ++launches, s);

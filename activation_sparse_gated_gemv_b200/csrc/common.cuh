@@ -283,6 +283,7 @@ struct DecodeParams {
     void* y;                // [n][d] T
     const uint32_t* hot;    // [ceil(d_ff / 32)] heavy-hitter channel bits, or NULL
     int dense;              // dense FFN (dense gate): every channel, W_up rows streamed with the gate's
+    int own_rows;           // sparse: reduce through per-CTA partials of y instead of the union gather
 };
 
 // Batched tensor-core GEMM (tcgen05): modes and parameters.

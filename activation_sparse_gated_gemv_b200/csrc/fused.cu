@@ -466,12 +466,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     }
     __syncthreads();
 
-    if (dense) {
-        // ---- dense FFN: every slot, in ascending order.  Each thread adds, for
-        // its 16-byte column chunks, h_k W_down[k, :] over the CTA's rows (read
-        // straight from HBM with 8 rows in flight), stores the CTA's fp32
-        // partial of y, and after a grid barrier every CTA sums one column
+    if (dense || p.own_rows) {
+        // ---- own rows: the CTA's kept slots in ascending order (every slot in
+        // the dense FFN).  Each thread adds, for its 16-byte column chunks,
+        // h_k W_down[k, :] over those rows (8 rows in flight), stores the CTA's
+        // fp32 partial of y, and after a grid barrier every CTA sums one column
         // slice of y over the partials in CTA order.
+        int tot = nslots;
+        if (!dense) {
+            if (warp == 0) {
+                int cnt = 0;
+                for (int base = 0; base < nslots; base += 32) {
+                    const int sl = base + lane;
+                    const bool f = sl < nslots && flag[sl];
+                    const unsigned m = __ballot_sync(0xffffffffu, f);
+                    if (f) wl[cnt + __popc(m & ((1u << lane) - 1u))] = sl;
+                    cnt += __popc(m);
+                }
+                if (lane == 0) scan_sh[0] = cnt;
+            }
+            __syncthreads();
+            tot = scan_sh[0];
+        }
+        auto slot_of = [&](int i) { return dense ? i : wl[i]; };
         constexpr int UBD = 8;
         const int cpd = p.d / V;                          // 16-byte chunks per output row
         for (int cch = threadIdx.x; cch < cpd; cch += kDecThreads) {
@@ -480,20 +497,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             for (int t = 0; t < NT; ++t)
 #pragma unroll
                 for (int e = 0; e < V / 2; ++e) acc[t][e] = make_float2(0.f, 0.f);
-            for (int s0 = 0; s0 < nslots; s0 += UBD) {
+            for (int s0 = 0; s0 < tot; s0 += UBD) {
                 uint4 w[UBD];
 #pragma unroll
                 for (int u2 = 0; u2 < UBD; ++u2)
-                    w[u2] = s0 + u2 < nslots ? ld_stream(wdn + (size_t)(c0 + s0 + u2) * p.d + (size_t)cch * V)
-                                             : make_uint4(0u, 0u, 0u, 0u);
+                    w[u2] = s0 + u2 < tot ? ld_stream(wdn + (size_t)(c0 + slot_of(s0 + u2)) * p.d + (size_t)cch * V)
+                                          : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int u2 = 0; u2 < UBD; ++u2) {
-                    if (s0 + u2 < nslots) {
+                    if (s0 + u2 < tot) {
                         float wf[V];
                         unpack<T>(w[u2], wf);
 #pragma unroll
                         for (int t = 0; t < NT; ++t) {
-                            const float h = hs[(s0 + u2) * NT + t];
+                            const float h = hs[slot_of(s0 + u2) * NT + t];
                             const float2 hh = make_float2(h, h);
 #pragma unroll
                             for (int e = 0; e < V / 2; ++e)
@@ -520,13 +537,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             if (col0 < p.d) target = grid_arrive(bar, G) + (unsigned long long)p.bar_extra;
             else atomicAdd(bar, 1ull);
         }
-        // every slot is listed, for sffn_get_active only
-        for (int i = threadIdx.x; i < nslots; i += kDecThreads) {
-            p.lst_idx[c0 + i] = c0 + i;
-            for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + i) * p.mw + w] = smask[i * p.mw + w];
+        // the CTA's list, for sffn_get_active only: off the path to the barrier
+        for (int i = threadIdx.x; i < tot; i += kDecThreads) {
+            const int sl = slot_of(i);
+            p.lst_idx[c0 + i] = c0 + sl;
+            for (int w = 0; w < p.mw; ++w) p.lst_mask[(size_t)(c0 + sl) * p.mw + w] = smask[sl * p.mw + w];
         }
         if (threadIdx.x == 0) {
-            p.seg_count[blockIdx.x] = nslots;
+            p.seg_count[blockIdx.x] = tot;
             int ok = 1;
             if (col0 < p.d) {
                 const unsigned long long t0 = globaltimer_ns();
