@@ -138,8 +138,8 @@ struct sffn_ctx {
     uint32_t* selbits = nullptr; // [max_tokens][ceil(d_ff / 32)] per-token selection bits of the tensor-core gate
     int selw = 0;
 
-    void* h2 = nullptr;          // [2 npad][tc_ldh] bf16: h as hi/lo rows
-    void* u2 = nullptr;          // [2 npad][r] bf16: LoPA x A as hi/lo rows
+    void* h2 = nullptr;          // [npad][tc_ldh] bf16: h, one row per token
+    void* u2 = nullptr;          // [2 npad][r] bf16: LoPA x A as hi/lo rows (passes of up to 128 tokens)
     float* tc_part = nullptr;    // [sms][2][128][256] floats: room for one parked part per CTA at any N
     unsigned* tc_tickets = nullptr;
     bool maps_ok = false;        // weight tensor maps encoded
@@ -280,7 +280,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     if (!h->maps_ok || (lopa && c.lopa_rank < 64)) return SFFN_ERR_UNSUPPORTED;
     CUtensorMap map_x{}, map_u2{}, map_h2{};
     if (encode_tile_map(&map_x, x, c.d, n, (uint64_t)c.d * 2, 64, npad) != cudaSuccess ||
-        encode_tile_map(&map_h2, h->h2, h->tc_ldh, 2 * npad, (uint64_t)h->tc_ldh * 2, 64, 2 * npad) != cudaSuccess ||
+        encode_tile_map(&map_h2, h->h2, h->tc_ldh, npad, (uint64_t)h->tc_ldh * 2, 64, npad) != cudaSuccess ||
         (lopa && encode_tile_map(&map_u2, h->u2, c.lopa_rank, 2 * npad, (uint64_t)c.lopa_rank * 2, 64, 2 * npad) !=
                      cudaSuccess))
         return SFFN_ERR_UNSUPPORTED;
@@ -352,7 +352,9 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     w.gather = gather ? 1 : 0; w.ulist = h->ulist; w.ucount = h->ucount;
     w.ubits = h->ubits; w.d_ff = c.d_ff; w.force_all = dense ? 1 : 0;
     w.m_total = c.d_ff; w.k_total = c.d; w.nb = npad;
-    w.out = h->h2; w.ldo = h->tc_ldh; w.h_pairs = 1;
+    // h goes to the down pass as one bf16 row per token: its rounding moves y by
+    // about 2^-9 relative (LoPA's u, which decides selections, keeps hi/lo pairs)
+    w.out = h->h2; w.ldo = h->tc_ldh; w.h_pairs = 0;
     w.zsel = zrows; w.gsel = grows; w.ldsel = c.d_ff;
     SFFN_CUDA(launch_tc(w, h->sms, s, true), "tensor-core up launch");
     set_name(h, launches, "tc_up");
@@ -363,7 +365,7 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     dn.ta = h->map_wdn; dn.tg = h->map_wdn_g; dn.tb = map_h2;
     dn.gather = gather ? 1 : 0; dn.ulist = h->ulist; dn.ucount = h->ucount;
     dn.ubits = h->ubits; dn.d_ff = c.d_ff; dn.force_all = dense ? 1 : 0;
-    dn.m_total = c.d; dn.nb = 2 * npad; dn.paired = 1;
+    dn.m_total = c.d; dn.nb = npad; dn.paired = 0;
     dn.out = out; dn.ldo = c.d;
     SFFN_CUDA(launch_tc(dn, h->sms, s, true), "tensor-core down launch");
     set_name(h, launches, "tc_down");
@@ -405,12 +407,13 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
     // decode kernel, or the tensor-core path for two tokens where the decode
     // kernel's shared memory does not fit.
     if (h->tc && (n > kFusedMaxTokens || (n > 1 && !fused))) {
-        // More than kTcMaxTokens tokens: one tensor-core pass per block of
-        // kTcMaxTokens tokens (each pass streams the weights again, which still
-        // beats the CUDA-core path's fp32 arithmetic at such batches).
+        // More tokens than one pass takes (256, or 128 with LoPA): one
+        // tensor-core pass per block of tokens (each pass streams the weights
+        // again, which still beats the CUDA-core path's fp32 arithmetic).
+        const int pass = lopa ? kTcMaxTokensLopa : kTcMaxTokens;
         int rc = SFFN_OK;
-        for (int t0 = 0; t0 < n && rc == SFFN_OK; t0 += kTcMaxTokens) {
-            const int nc = n - t0 < kTcMaxTokens ? n - t0 : kTcMaxTokens;
+        for (int t0 = 0; t0 < n && rc == SFFN_OK; t0 += pass) {
+            const int nc = n - t0 < pass ? n - t0 : pass;
             rc = run_tc(h, static_cast<const char*>(x) + (size_t)t0 * c.d * h->esz, nc, lopa, sel,
                         static_cast<char*>(out) + (size_t)t0 * c.d * h->esz, s, dense, launches, t0);
             if (rc == SFFN_ERR_UNSUPPORTED && t0 > 0) rc = fail(SFFN_ERR_CUDA, "tensor-core pass failed mid-batch");
@@ -622,7 +625,8 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     const size_t o_ub = take(h->tc ? tiles * 4 * 4 : 0);
     h->selw = (int)((F + 31) / 32);
     const size_t o_sb = take(h->tc ? T * (size_t)h->selw * 4 : 0);
-    const size_t o_h2 = take(2 * NP * (size_t)h->tc_ldh * 2), o_u2 = take(2 * NP * R * 2);
+    const size_t NPL = NP < (size_t)kTcMaxTokensLopa ? NP : (size_t)kTcMaxTokensLopa;
+    const size_t o_h2 = take(NP * (size_t)h->tc_ldh * 2), o_u2 = take(2 * NPL * R * 2);
     const size_t o_ul = take(h->tc ? (size_t)h->tc_ldh * 4 : 0), o_uc = take(h->tc ? 16 : 0);
     // stream-K partial tiles: two slots per CTA of up to 256 accumulator columns x 128 rows
     const size_t o_tp = take(h->tc ? (size_t)h->sms * 2 * 256 * 128 * 4 : 0), o_tt = take(h->tc ? tiles * 8 : 0);

@@ -427,6 +427,7 @@ cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s, bool pdl);
 // padded with channel 0 to a multiple of 128, and its size.
 cudaError_t launch_union_list(const uint32_t* ubits, int d_ff, int* list, int* count, cudaStream_t s, bool pdl);
 constexpr int kTcGatherMaxTokens = 8;  // batches up to this size may gather the union's rows
-constexpr int kTcMaxTokens = 128;     // token columns of one tensor-core pass (hi/lo pairs fill N = 256)
+constexpr int kTcMaxTokens = 256;     // token columns of one tensor-core pass (MMA N <= 256)
+constexpr int kTcMaxTokensLopa = 128; // ... with LoPA, whose u enters the gate as hi/lo pairs (2 x 128 columns)
 
 }  // namespace sffn

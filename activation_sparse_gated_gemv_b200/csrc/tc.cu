@@ -495,43 +495,49 @@ __device__ __forceinline__ void emit16(const TcParams& p, int m, int c0, const f
 // ---- up epilogue ---------------------------------------------------------------
 // h(token, m) = g(token, m) * acc, g the gate activation of channel m for the
 // token (ReLU(z - tau), or the selected SiLU value; zero past n and d_ff).
-// The gate values of a tile are loaded into registers before its accumulator
-// is ready, so their latency hides behind the mainloop instead of costing one
-// round trip per 16 tokens after it.
+// The gate values of a tile's first kUpChunks x 16 tokens are loaded into
+// registers before its accumulator is ready, so their latency hides behind
+// the mainloop; the values of later tokens (passes of up to 256) are loaded
+// one chunk ahead of their use.
 
-constexpr int kUpChunks = kTcMaxTokens / 16;
+constexpr int kUpChunks = 4;
 
 struct UpG {
     float raw[kUpChunks * 16];
 };
 
-// Issue the loads of the gate source (z or the selected g) of channel m (m < 0:
-// none, a padding row of a gathered tile) for the first `cols` token columns.
-__device__ __forceinline__ void up_g_load(const TcParams& p, int m, int cols, UpG& g) {
+// The 16 gate values of channel m (m < 0: none, a padding row of a gathered
+// tile) for token columns 16j .. 16j + 15.
+__device__ __forceinline__ void up_g_chunk(const TcParams& p, int m, int j, float* g16) {
     const float* src = p.topk ? p.gsel : p.zsel;
     const bool row_ok = m >= 0 && m < p.m_total;
 #pragma unroll
-    for (int j = 0; j < kUpChunks; ++j) {
-        if (16 * j < cols) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int tok = 16 * j + i;
-                g.raw[16 * j + i] = (row_ok && tok < p.n) ? __ldcg(src + (long long)tok * p.ldsel + m) : 0.f;
-            }
-        }
+    for (int i = 0; i < 16; ++i) {
+        const int tok = 16 * j + i;
+        g16[i] = (row_ok && tok < p.n) ? __ldcg(src + (long long)tok * p.ldsel + m) : 0.f;
     }
 }
 
+// Issue the loads of the gate values of channel m for the first `cols` token
+// columns (at most kUpChunks x 16).
+__device__ __forceinline__ void up_g_load(const TcParams& p, int m, int cols, UpG& g) {
+#pragma unroll
+    for (int j = 0; j < kUpChunks; ++j)
+        if (16 * j < cols) up_g_chunk(p, m, j, g.raw + 16 * j);
+}
+
 // Columns 16j..16j+15 of channel m (m < 0: a padding row, h = 0): h = g * v,
-// written as bf16 hi (and lo) rows at output column mo (the channel, or with
-// gather its list position).
-__device__ __forceinline__ void up_emit16(const TcParams& p, int m, int mo, int j, const float* v, const UpG& g) {
+// written as bf16 rows (and, for a paired consumer, the rounding remainder as
+// lo rows) at output column mo (the channel, or with gather its list
+// position).  g16: the 16 gate values of those columns.
+__device__ __forceinline__ void up_emit16(const TcParams& p, int m, int mo, int j, const float* v,
+                                          const float* g16) {
     bf16* o = static_cast<bf16*>(p.out);
     const bool row_ok = m >= 0 && m < p.m_total;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int tok = 16 * j + i;
-        const float raw = g.raw[16 * j + i];
+        const float raw = g16[i];
         const float gv = (row_ok && tok < p.n) ? (p.topk ? raw : fmaxf(raw - p.tau, 0.f)) : 0.f;
         const float h = row_ok ? gv * v[i] : 0.f;
         const bf16 hi = __float2bfloat16_rn(h);
@@ -684,7 +690,23 @@ __device__ void run_epilogue(const TcParams& p, const Problem& q, TcShared* sh, 
                     float v[16];
                     tmem_ld16(taddr + 16 * j, v);
                     add_parts16(p, pbase, slot_floats, np, row, 16 * j, pglobal, v);
-                    up_emit16(p, m, mo, j, v, g);
+                    up_emit16(p, m, mo, j, v, g.raw + 16 * j);
+                }
+                if (cols > 16 * kUpChunks) {
+                    // tokens past the preloaded ones: each chunk's gate values load
+                    // while the previous chunk's accumulator is read and emitted
+                    float gn[16];
+                    up_g_chunk(p, m, kUpChunks, gn);
+                    for (int j = kUpChunks; 16 * j < cols; ++j) {
+                        float gc[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) gc[i] = gn[i];
+                        if (16 * (j + 1) < cols) up_g_chunk(p, m, j + 1, gn);
+                        float v[16];
+                        tmem_ld16(taddr + 16 * j, v);
+                        add_parts16(p, pbase, slot_floats, np, row, 16 * j, pglobal, v);
+                        up_emit16(p, m, mo, j, v, gc);
+                    }
                 }
             } else {
                 for (int c0 = 0; c0 < cols; c0 += 16) {
