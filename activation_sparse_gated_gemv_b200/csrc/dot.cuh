@@ -137,6 +137,52 @@ __device__ __forceinline__ void piece_dot(const unsigned char* piece, int nch, i
     }
 }
 
+// Per-lane partials of R short rows at once: rows q < cnt of a shared-memory
+// piece, rb bytes apart, cpr 16-byte chunks each.  Every lane loads its chunk
+// of all R rows before the arithmetic, and the x chunk once for all of them.
+template <class WT, int NT, int R>
+__device__ __forceinline__ void rows_dot(const unsigned char* piece, int rb, int cnt, int cpr, const float* xs,
+                                         int len, float2 (&acc)[R][NT]) {
+    const int lane = threadIdx.x & 31;
+    for (int c = lane; c < cpr; c += 32) {
+        uint4 w[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q)
+            w[q] = q < cnt ? *reinterpret_cast<const uint4*>(piece + (size_t)q * rb + (size_t)c * 16)
+                           : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int q = 0; q < R; ++q)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) chunk_dot<WT>(w[q], xs + t * len, len, c, acc[q][t]);
+    }
+}
+
+// Warp sums of R values per lane (R = 1, 2, 4 or 8) in log2(R) halving
+// exchanges plus 5 - log2(R) plain butterfly steps: the lanes of group
+// lane >> (5 - log2 R) end with the sum of v[lane >> (5 - log2 R)].  The
+// order of the additions is fixed, so the sums are reproducible.
+template <int R>
+__device__ __forceinline__ float warp_sum_scatter(const float (&v)[R]) {
+    const int lane = threadIdx.x & 31;
+    float w[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) w[q] = v[q];
+    int bit = 16;
+#pragma unroll
+    for (int m = R; m > 1; m >>= 1, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int i = 0; i < m / 2; ++i) {
+            const float send = up ? w[i] : w[i + m / 2];
+            const float keep = up ? w[i + m / 2] : w[i];
+            w[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+        }
+    }
+    float s = w[0];
+    for (; bit > 0; bit >>= 1) s += __shfl_xor_sync(0xffffffffu, s, bit);
+    return s;
+}
+
 // Ordered compaction of the slots [0, nslots) whose `keep(s)` holds: out[] gets
 // them in ascending order; returns the count.  All threads of the block call it.
 template <class Keep>

@@ -321,6 +321,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             reinterpret_cast<volatile int*>(queue)[slot] = s + 1;
         }
     };
+    // The same for several whole rows at once (pieces of whole rows), each by
+    // the lane that has `mine` for it: the lanes select in parallel and take
+    // their queue places with one atomic.
+    auto finalize_rows = [&](int s, const float (&z)[NT], bool mine) {   // all lanes
+        uint32_t tokmask = 0u;
+        if (mine) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                zfin[s * NT + t] = z[t];
+                if (t < n && z[t] > p.tau) tokmask |= 1u << t;
+            }
+            if (tokmask) {
+                flag[s] = 1;
+                smask[s * p.mw] = tokmask;
+                bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+            }
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, tokmask != 0u);
+        if (m) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(ctr + kQueueTail, __popc(m));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (tokmask) {
+                __threadfence_block();
+                reinterpret_cast<volatile int*>(queue)[base + __popc(m & ((1u << lane) - 1u))] = s + 1;
+            }
+        }
+    };
 
     // ---- streaming warps
     if (streamer) {
@@ -340,19 +368,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             if (!abort) {
                 const unsigned char* buf = bufs + (size_t)cbuf * p.sb;
                 if (rows_mode) {
+                    // R rows at a time: the dots, one scattering warp sum
+                    // that leaves row q's z with lane group q, and the
+                    // selection by the first lane of each group
+                    constexpr int R = NT <= 2 ? 8 : 4;
+                    constexpr int GS = 32 / R;                   // lanes per row group
                     const int r0 = g * rpp, cnt = min(rpp, nslots - r0);
-                    for (int q = 0; q < cnt; ++q) {
-                        float2 v2[NT];
+                    for (int q0 = 0; q0 < cnt; q0 += R) {
+                        float2 v2[R][NT];
 #pragma unroll
-                        for (int t = 0; t < NT; ++t) v2[t] = make_float2(0.f, 0.f);
-                        piece_dot<T, NT>(buf + (size_t)q * rb, cpr, 0, gx, glen, v2);
+                        for (int q = 0; q < R; ++q)
+#pragma unroll
+                            for (int t = 0; t < NT; ++t) v2[q][t] = make_float2(0.f, 0.f);
+                        rows_dot<T, NT, R>(buf + (size_t)q0 * rb, rb, min(R, cnt - q0), cpr, gx, glen, v2);
+                        float z[NT];
 #pragma unroll
                         for (int t = 0; t < NT; ++t) {
-                            const float v = warp_sum(v2[t].x + v2[t].y);
-                            if (lane == t) zpart[(r0 + q) * NT + t] = v;
+                            float v[R];
+#pragma unroll
+                            for (int q = 0; q < R; ++q) v[q] = v2[q][t].x + v2[q][t].y;
+                            z[t] = warp_sum_scatter<R>(v);
                         }
-                        __syncwarp();
-                        if (lane == 0) finalize(r0 + q);
+                        const int q = lane / GS;
+                        finalize_rows(r0 + q0 + q, z, lane % GS == 0 && q0 + q < cnt);
                     }
                 } else {
                     const int off = (part < ppr ? part : part - ppr) * pb;
