@@ -125,6 +125,7 @@ struct sffn_ctx {
     float* fpart = nullptr;      // fused decode, dense FFN: [g1][min(max_tokens, 4)][d] partials of y
     unsigned* tickets = nullptr;
     unsigned* dbar = nullptr;    // fused decode: grid-barrier arrival counters
+    unsigned long long x_arrivals = 0;   // ... and the count its x counter has reached (host forwards)
     int* status = nullptr;
     int* hstat = nullptr;        // host-mapped mirror of the status word (host address)
     int* hstat_dev = nullptr;    // ... and its device address, given to the kernels
@@ -380,8 +381,11 @@ int run_tc(sffn_ctx* h, const void* x, int n, bool lopa, const sffn_select* sel,
     return SFFN_OK;
 }
 
+// xmapped: a forward with host buffers whose x is page-locked host memory the
+// device can address (x is then the device buffer it goes to): the fused
+// decode kernel pulls it in itself; the other paths copy it first.
 int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_select* sel, void* out,
-                cudaStream_t s, bool dense) {
+                cudaStream_t s, bool dense, const void* xmapped = nullptr) {
     const sffn_config& c = h->cfg;
     const Plan& P = h->plan;
     const bool lopa = gate_mode == SFFN_GATE_LOPA;
@@ -402,6 +406,9 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
                                        &dec_smem);
 
     h->last_tc = false;
+    if (xmapped && !fused)
+        SFFN_CUDA(cudaMemcpyAsync(const_cast<void*>(x), xmapped, (size_t)n * c.d * h->esz, cudaMemcpyDefault, s),
+                  "x host-to-device copy");
     // Three or more tokens: the tensor-core path (measured faster than the fused
     // decode kernel from n = 3 on every shape but one); one or two: the fused
     // decode kernel, or the tensor-core path for two tokens where the decode
@@ -448,7 +455,13 @@ int run_forward(sffn_ctx* h, const void* x, int n, int gate_mode, const sffn_sel
         // partial of y (measured faster up to d = 4096), or the union gather by
         // column slice (faster on the 70B shape, d = 8192).
         dp.own_rows = c.d <= 4096 ? 1 : 0;
+        if (xmapped) {
+            dp.xh = xmapped;
+            dp.xld = (int)(((size_t)n * c.d * h->esz + 8191) / 8192);
+            dp.xtarget = h->x_arrivals + (unsigned long long)dp.xld;
+        }
         SFFN_CUDA(launch_decode(c.wdtype, dp, dec_nt, gk, P.g1, dec_smem, s, pdl), "fused decode launch");
+        if (xmapped) h->x_arrivals = dp.xtarget;          // counted only once the launch is in
         set_name(h, launches, dense ? "decode_dense" : "decode_fused");
         record(h, ++launches, s);
         h->last_n = n;
@@ -810,8 +823,20 @@ int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_
             ydst = pa.devicePointer;
         cudaGetLastError();
     }
-    SFFN_CUDA(cudaMemcpyAsync(h->xdev, x_host, bytes, cudaMemcpyHostToDevice, s), "x host-to-device copy");
-    rc = run_forward(h, h->xdev, n_tokens, gate_mode, sel, ydst, s, false);
+    // x: page-locked host memory the device can address is pulled in by the
+    // fused decode kernel itself (no copy-engine round trip); other memory is
+    // copied first.
+    const void* xmapped = nullptr;
+    if (n_tokens <= kFusedMaxTokens && (bytes & 15) == 0) {
+        cudaPointerAttributes pa{};
+        if (cudaPointerGetAttributes(&pa, x_host) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
+            pa.devicePointer && aligned16(pa.devicePointer))
+            xmapped = pa.devicePointer;
+        cudaGetLastError();
+    }
+    if (!xmapped)
+        SFFN_CUDA(cudaMemcpyAsync(h->xdev, x_host, bytes, cudaMemcpyHostToDevice, s), "x host-to-device copy");
+    rc = run_forward(h, h->xdev, n_tokens, gate_mode, sel, ydst, s, false, xmapped);
     if (rc) return rc;
     if (ydst == h->ydev)
         SFFN_CUDA(cudaMemcpyAsync(out_host, h->ydev, bytes, cudaMemcpyDeviceToHost, s), "y device-to-host copy");

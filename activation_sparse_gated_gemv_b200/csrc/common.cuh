@@ -279,11 +279,15 @@ struct DecodeParams {
     int* hstatus;           // host-mapped mirror of the status word, or NULL
     unsigned long long wait_ns;   // limit of the grid-barrier waits
     int bar_extra;          // arrivals the final grid barrier expects beyond the grid (0; 1 makes it time out)
-    unsigned* tickets;      // 64-bit grid-barrier arrival counters (h, LoPA's u, the union masks), zero at creation
+    unsigned* tickets;      // 64-bit arrival counters (h, LoPA's u, the union masks, x), zero at creation
     void* y;                // [n][d] T
     const uint32_t* hot;    // [ceil(d_ff / 32)] heavy-hitter channel bits, or NULL
     int dense;              // dense FFN (dense gate): every channel, W_up rows streamed with the gate's
     int own_rows;           // sparse: reduce through per-CTA partials of y instead of the union gather
+    const void* xh;         // forward with host buffers: device address of the page-locked host copy of x,
+                            // pulled into x (device memory) inside the launch; NULL when x is already there
+    int xld;                // CTAs that pull x (the first xld)
+    unsigned long long xtarget;   // arrivals the x counter (tickets' fourth word) reaches once x is in
 };
 
 // Batched tensor-core GEMM (tcgen05): modes and parameters.

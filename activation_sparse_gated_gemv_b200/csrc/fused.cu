@@ -226,6 +226,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
 
     griddep_wait();
     griddep_launch_dependents();
+    // Host buffers: the first xld CTAs pull x from page-locked host memory into
+    // the device buffer (16-byte loads, all in flight) and count themselves in
+    // on the x counter; every CTA waits for the count before it stages x.
+    if (p.xh && (int)blockIdx.x < p.xld) {
+        const int n16 = p.n * p.d * (int)sizeof(T) / 16;
+        const int per = (n16 + p.xld - 1) / p.xld;
+        const int i0 = blockIdx.x * per, i1 = min(n16, i0 + per);
+        for (int i = i0 + threadIdx.x; i < i1; i += kDecThreads)
+            reinterpret_cast<uint4*>(const_cast<void*>(p.x))[i] = reinterpret_cast<const uint4*>(p.xh)[i];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(bar + 3, 1ull);
+        }
+    }
 
     for (int i = threadIdx.x; i < p.cpb; i += kDecThreads) {
         flag[i] = 0;
@@ -250,7 +265,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     }
     for (int i = threadIdx.x; i < p.cpb * p.mw; i += kDecThreads) smask[i] = 0u;
     if (threadIdx.x < 4) ctr[threadIdx.x] = 0;
-    stage_rows<T, T, NT>(xs, static_cast<const T*>(p.x), p.d, 0, n);
+    if (p.xh) {
+        if (threadIdx.x == 0) {
+            const unsigned long long t0 = globaltimer_ns();
+            while (ld_acquire_u64(bar + 3) < p.xtarget) {
+                if (globaltimer_ns() - t0 > p.wait_ns) {
+                    raise_status(p.status, p.hstatus, kStatusWaitTimeout);
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        __syncthreads();
+        __threadfence();
+    }
+    stage_rows<T, T, NT>(xs, static_cast<const T*>(p.x), p.d, 0, n, p.xh != nullptr);
     if (streamer) {
         while (issued < min(p.nb, wcount)) issue_next();
         __syncwarp();
@@ -291,6 +320,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         __syncthreads();
     }
 
+    // A selected channel's W_down row goes to L2 at once when the gate is
+    // dense and the CTA sums its own rows (measured: 0.5 us faster on the
+    // 7B shape; slower with LoPA's short gate stream and with the union
+    // gather, whose reads are column slices).
+    const bool dn_prefetch = GATE == kGateDense && p.own_rows;
     // Row s is complete: z from its parts in order, select, queue it.  Dense
     // mode: the up dot is complete too (parts ppr ..), so h is formed here
     // and every channel is kept (with h = 0 for a token whose z <= tau).
@@ -315,7 +349,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         } else if (tokmask) {
             flag[s] = 1;
             smask[s * p.mw] = tokmask;                   // n <= 4: tokens sit in mask word 0
-            bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+            if (dn_prefetch) bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
             const int slot = atomicAdd(ctr + kQueueTail, 1);
             __threadfence_block();
             reinterpret_cast<volatile int*>(queue)[slot] = s + 1;
@@ -335,7 +369,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             if (tokmask) {
                 flag[s] = 1;
                 smask[s * p.mw] = tokmask;
-                bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+                if (dn_prefetch) bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
             }
         }
         const unsigned m = __ballot_sync(0xffffffffu, tokmask != 0u);

@@ -135,11 +135,12 @@ int sffn_forward_dense(sffn_handle h, const void* x, int n_tokens, int gate_mode
 
 /* sffn_forward with HOST buffers: copies x_host to the device, runs the
  * forward and delivers the result into out_host, all on `stream`, then
- * synchronises it.  Pinned host memory gives asynchronous copies; with one or
- * two tokens and a page-locked out_host that the device can address (memory
- * from cudaHostAlloc / cudaMallocHost or cudaHostRegister under unified
- * addressing), the decode kernel stores y there directly instead of copying
- * it back.  Errors: as sffn_forward. */
+ * synchronises it.  Pinned host memory gives asynchronous copies.  With one or
+ * two tokens, page-locked buffers that the device can address (memory from
+ * cudaHostAlloc / cudaMallocHost or cudaHostRegister under unified
+ * addressing) are read and written by the fused decode kernel itself: it
+ * pulls x_host in at its start and stores y into out_host, so neither takes a
+ * copy-engine round trip.  Errors: as sffn_forward. */
 int sffn_forward_host(sffn_handle h, const void* x_host, int n_tokens, int gate_mode,
                       const sffn_select* sel, void* out_host, void* stream);
 

@@ -416,25 +416,48 @@ def test_forward_host_matches_device_forward(sffn):
     ffn.close()
 
 
-@pytest.mark.parametrize("n,pinned_out", [(1, True), (1, False), (2, True), (5, True)])
-def test_forward_host_output_kinds(sffn, n, pinned_out):
-    """One or two tokens into a page-locked output: the decode kernel stores y
-    in host memory itself; a pageable output, or a batch, goes through a copy.
-    Either way y is bitwise the device forward's."""
+@pytest.mark.parametrize("n,pinned_x,pinned_out", [(1, True, True), (1, False, True), (1, True, False),
+                                                   (2, True, True), (2, False, False), (5, True, True)])
+def test_forward_host_buffer_kinds(sffn, n, pinned_x, pinned_out):
+    """One or two tokens with page-locked buffers: the decode kernel pulls x in
+    from host memory and stores y there itself; pageable buffers, or a batch,
+    go through copies.  Either way y is bitwise the device forward's, call
+    after call (the kernel's x arrival counter never resets)."""
     d, d_ff = 512, 3000
     w = workloads.ffn_weights(d, d_ff, "bf16", seed=91)
     ffn = sffn.SparseFFN(d, d_ff, 0, 8, "bf16")
     ffn.set_weights(**w)
-    x = workloads.tokens(n, d, "bf16", seed=92)
     tau = workloads.tau_for_sparsity(0.9)
-    yd = ffn.forward(x.cuda(), tau=tau).cpu()
     out = torch.full((n, d), float("nan"), dtype=torch.bfloat16)
     if pinned_out:
         out = out.pin_memory()
-    for _ in range(2):
-        yh = ffn.forward_host(x.pin_memory(), tau=tau, out=out)
-        assert torch.equal(yd, yh)
+    for i in range(3):
+        x = workloads.tokens(n, d, "bf16", seed=92 + i)
+        yd = ffn.forward(x.cuda(), tau=tau).cpu()
+        xh = x.pin_memory() if pinned_x else x.clone()
+        yh = ffn.forward_host(xh, tau=tau, out=out)
+        assert torch.equal(yd, yh), i
         out.fill_(float("nan"))
+    ffn.check_status()
+    ffn.close()
+
+
+def test_forward_host_mixed_calls(sffn):
+    """Host forwards of every kind in one handle, interleaved with device
+    forwards and LoPA: each matches the device forward bitwise, and the status
+    stays clean (a miscounted x arrival would time out)."""
+    d, d_ff, r = 512, 3000, 64
+    w = workloads.ffn_weights(d, d_ff, "bf16", seed=93, gate="both", r=r)
+    ffn = sffn.SparseFFN(d, d_ff, r, 8, "bf16")
+    ffn.set_weights(**w)
+    tau = workloads.tau_for_sparsity(0.9)
+    for i, (n, gate, pinned) in enumerate([(1, "dense", True), (2, "lopa", True), (1, "dense", False), (4, "dense", True),
+                                           (1, "lopa", True), (2, "dense", True), (1, "dense", True)]):
+        x = workloads.tokens(n, d, "bf16", seed=94 + i)
+        yd = ffn.forward(x.cuda(), gate=gate, tau=tau).cpu()
+        yh = ffn.forward_host(x.pin_memory() if pinned else x.clone(), gate=gate, tau=tau)
+        assert torch.equal(yd, yh), (i, n, gate, pinned)
+    ffn.check_status()
     ffn.close()
 
 
