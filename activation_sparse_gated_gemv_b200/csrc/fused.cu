@@ -637,16 +637,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         if (!scan_sh[2] || col0 >= p.d) return;
         __threadfence();
         // y[:, col0 : col0 + cps V] = sum over the G partials: thread (g, item)
-        // adds partials g, g + GR, ... in order, then the GR sums in order
+        // adds partials g, g + GR, ... in order (up to UBS loads in flight),
+        // then the GR sums in order; GR is as small as one round of loads
+        // allows, so that the serial second sum is short
+        constexpr int UBS = 16;
         const int q4 = min(cps * V, p.d - col0) / 4;      // float4 per token
         const int items = n * q4;
-        const int GR = max(1, kDecThreads / items);
+        const int GR = max(1, min(kDecThreads / items, (G + UBS - 1) / UBS));
         float4* red4 = reinterpret_cast<float4*>(smem + L.bufs);          // the idle ring
         const int g = (int)threadIdx.x / items, item = (int)threadIdx.x - g * items;
         if (g < GR) {
             const int t = item / q4, c = col0 + (item - t * q4) * 4;
             float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-            constexpr int UBS = 16;
             for (int b0 = g; b0 < G; b0 += UBS * GR) {
                 float4 v[UBS];
 #pragma unroll
