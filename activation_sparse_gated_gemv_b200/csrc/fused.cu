@@ -320,11 +320,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         __syncthreads();
     }
 
-    // A selected channel's W_down row goes to L2 at once when the gate is
-    // dense and the CTA sums its own rows (measured: 0.5 us faster on the
+    // A selected channel's W_up and W_down rows go to L2 at once when the gate
+    // is dense and the CTA sums its own rows (measured: 0.7 us faster on the
     // 7B shape; slower with LoPA's short gate stream and with the union
     // gather, whose reads are column slices).
-    const bool dn_prefetch = GATE == kGateDense && p.own_rows;
+    const bool l2_prefetch = GATE == kGateDense && p.own_rows;
     // Row s is complete: z from its parts in order, select, queue it.  Dense
     // mode: the up dot is complete too (parts ppr ..), so h is formed here
     // and every channel is kept (with h = 0 for a token whose z <= tau).
@@ -349,7 +349,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         } else if (tokmask) {
             flag[s] = 1;
             smask[s * p.mw] = tokmask;                   // n <= 4: tokens sit in mask word 0
-            if (dn_prefetch) bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+            if (l2_prefetch) {
+                bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+                bulk_prefetch_l2(wup + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+            }
             const int slot = atomicAdd(ctr + kQueueTail, 1);
             __threadfence_block();
             reinterpret_cast<volatile int*>(queue)[slot] = s + 1;
@@ -369,7 +372,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             if (tokmask) {
                 flag[s] = 1;
                 smask[s * p.mw] = tokmask;
-                if (dn_prefetch) bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+                if (l2_prefetch) {
+                    bulk_prefetch_l2(wdn + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+                    bulk_prefetch_l2(wup + (size_t)(c0 + s) * p.d, (uint32_t)(p.d * sizeof(T)));
+                }
             }
         }
         const unsigned m = __ballot_sync(0xffffffffu, tokmask != 0u);

@@ -29,11 +29,12 @@
 // (batches of a few tokens at high sparsity), decided on the device from the
 // union's size.
 //
-// Kernel structure (one CTA per SM, 288 threads):
-//   warps 0, 6, 7, 8  one thread each: the TMA producers.  Producer p fills
-//              the ring stages of the k-blocks g with g % 4 == p: 2-D tile
-//              copies (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
-//              of the A and B tiles, or four-row gathers of A, on mbarriers;
+// Kernel structure (one CTA per SM, 416 threads):
+//   warps 0, 6 .. 12  one thread each: the TMA producers, P of them (4 for
+//              tile passes, 8 for gathered ones).  Producer p fills the ring
+//              stages of the k-blocks g with g % P == p: 2-D tile copies
+//              (cp.async.bulk.tensor, 128-byte swizzle, no multicast) of the
+//              A and B tiles, or four-row gathers of A, on mbarriers;
 //   warp 1     allocates tensor memory; one thread issues tcgen05.mma (M = 128,
 //              N = token columns, K = 16 per instruction, bf16 in, fp32
 //              accumulate in tensor memory) and tcgen05.commit;
@@ -65,15 +66,15 @@ constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;        // epilogue warps 2..5
 constexpr int kEpi = 4;
 constexpr int kProdWarp2 = kEpiWarp0 + kEpi;   // further TMA producers: warps 6, 7, ...
-constexpr int kProducers = 4;
-constexpr int kTcThreads = (kProdWarp2 + kProducers - 1) * 32;
+constexpr int kMaxProducers = 8;   // gathered passes: up to 8; tile passes: 4
+constexpr int kTcThreads = (kProdWarp2 + kMaxProducers - 1) * 32;
 constexpr uint32_t kTileA = kBM * kBK * 2;   // 16 KB
 constexpr int kMaxStages = 12;
 constexpr int kMaxBlocks = 1024;    // 128-channel blocks (d_ff <= 131072)
 constexpr int kMinIters = 8;        // iterations per CTA at least
 constexpr int kMaxParts = 8;        // CTAs sharing one tile at most
-constexpr int kIdxPerProducer = 4;  // gather: channel-index blocks each producer keeps in flight
-constexpr int kIdxSlots = kProducers * kIdxPerProducer;
+constexpr int kIdxPerProducer = 2;  // gather: channel-index blocks each producer keeps in flight
+constexpr int kIdxSlots = kMaxProducers * kIdxPerProducer;
 
 struct TcShared {
     uint64_t full[kMaxStages];
@@ -88,6 +89,7 @@ struct TcShared {
     int wcount[kTcThreads / 32];
     int ucount;             // gather: the union's size
     int gmode;              // this launch gathers rows (the union is under half the channels)
+    int nprod;              // producer threads taking turns over the k-blocks (<= the stages)
     int blk[kMaxBlocks];    // up/down: the active 128-channel blocks
     uint64_t ibar[kIdxSlots];
     alignas(16) int idx[kIdxSlots][kBM];   // gather: channel indices of one k-block's rows
@@ -289,14 +291,14 @@ __device__ void prefetch_first_tiles(const TcParams& p, int count) {
 
 // ---- producer: one thread issues the TMA copies --------------------------------
 
-// Producer `pr` of kProducers fills the stages of the k-blocks g with
-// g % kProducers == pr.  One thread issuing every copy of an SM's stream keeps
-// only about three quarters of HBM bandwidth busy; threads in different warps,
-// taking turns over the k-blocks of the same ring, reach the copy peak, and
-// four of them keep the 32 gathers of a gathered stage coming.  The ring stays
-// one sequence for the MMA issuer.  (A producer waits for stage
-// g - S to be consumed; with kProducers <= S the parity wait cannot be a phase
-// behind.)
+// Producer `pr` of P = sh->nprod fills the stages of the k-blocks g with
+// g % P == pr.  One thread issuing every copy of an SM's stream keeps only
+// about three quarters of HBM bandwidth busy; threads in different warps,
+// taking turns over the k-blocks of the same ring, reach the copy peak with
+// tile copies.  A gathered stage takes 32 four-row copies, and the copy rate
+// grows with the issuing threads: about 3 TB/s with four, 4 TB/s with eight.
+// The ring stays one sequence for the MMA issuer.  (A producer waits for stage
+// g - S to be consumed; with P <= S the parity wait cannot be a phase behind.)
 // Gather: k-block g of the CTA's range is iteration it0 + g, i.e. tile
 // (it0 + g) / KB and k-block (it0 + g) % KB, so a producer knows every future
 // k-block's rows.  Their channel indices (up: the tile's 128 list entries;
@@ -304,7 +306,7 @@ __device__ void prefetch_first_tiles(const TcParams& p, int count) {
 // kIdxPerProducer k-blocks ahead of their use.
 __device__ __forceinline__ void gather_index_copy(const TcParams& p, const Problem& q, TcShared* sh, int pr,
                                                   long long g) {
-    const long long j = g / kProducers;
+    const long long j = g / sh->nprod;
     const int slot = pr * kIdxPerProducer + (int)(j % kIdxPerProducer);
     const long long it = q.it0 + g;
     const int t = (int)(it / q.KB), kb = (int)(it % q.KB);
@@ -318,14 +320,16 @@ __device__ void run_producer_gather(const TcParams& p, const Problem& q, unsigne
                                     TcShared* sh, int pr) {
     const uint64_t pol_w = l2_evict_first(), pol_b = l2_evict_last();
     const int S = p.stages;
+    const int NP = sh->nprod;
+    if (pr >= NP) return;
     const uint32_t tx = kTileA + (uint32_t)p.nb * 128u;
     const long long n_it = q.it1 - q.it0;
     for (int j = 0; j < kIdxPerProducer; ++j) {
-        const long long g = pr + (long long)kProducers * j;
+        const long long g = pr + (long long)NP * j;
         if (g < n_it) gather_index_copy(p, q, sh, pr, g);
     }
-    for (long long g = pr; g < n_it; g += kProducers) {
-        const long long j = g / kProducers;
+    for (long long g = pr; g < n_it; g += NP) {
+        const long long j = g / NP;
         const int slot = pr * kIdxPerProducer + (int)(j % kIdxPerProducer);
         const long long it = q.it0 + g;
         const int t = (int)(it / q.KB), kb = (int)(it % q.KB);
@@ -362,7 +366,7 @@ __device__ void run_producer_gather(const TcParams& p, const Problem& q, unsigne
         }
         // this thread's reads of the index block come before the async copy that refills it
         fence_proxy_async();
-        const long long gn = g + (long long)kProducers * kIdxPerProducer;
+        const long long gn = g + (long long)NP * kIdxPerProducer;
         if (gn < n_it) gather_index_copy(p, q, sh, pr, gn);
     }
 }
@@ -375,13 +379,15 @@ __device__ void run_producer(const TcParams& p, const Problem& q, unsigned char*
     }
     const uint64_t pol_w = l2_evict_first(), pol_b = l2_evict_last();
     const int S = p.stages;
+    const int NP = sh->nprod;
+    if (pr >= NP) return;
     const uint32_t tx = kTileA + (uint32_t)p.nb * 128u;
     long long it = q.it0, g = 0;
     Seg s;
     while (next_seg(q, it, s)) {
         const int m0 = p.mode == kTcUp ? sh->blk[s.t] * kBM : s.t * kBM;
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++g) {
-            if ((int)(g % kProducers) != pr) continue;
+            if ((int)(g % NP) != pr) continue;
             const int st = (int)(g % S);
             if (!mbar_wait_one(&sh->empty[st], (uint32_t)(((g / S) & 1) ^ 1))) {
                 sh->abort = 1;
@@ -813,6 +819,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     if (threadIdx.x == 0) {
         sh->ucount = U;
         sh->gmode = gmode ? 1 : 0;
+        sh->nprod = min(gmode ? kMaxProducers : 4, p.stages);
     }
     __syncthreads();
     if (gmode) {
