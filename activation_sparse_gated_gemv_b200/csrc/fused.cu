@@ -279,6 +279,71 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
         __syncthreads();
         __threadfence();
     }
+    // LoPA stage 1 inside the launch: this CTA's rows of u = x A, published,
+    // then a grid barrier, after which every CTA stages all of u.  The rows
+    // are dotted with x straight from global memory, so the barrier's arrival
+    // does not wait for x's staging (which overlaps the barrier instead); each
+    // row is split over `parts` warps, whose sums meet in shared memory (the
+    // u staging area, free until then) and are added in part order.  The wait
+    // is bounded and cannot deadlock: all CTAs are resident.
+    unsigned long long utarget = 0ull;
+    if (GATE == kGateLopa) {
+        const int nr = u1 - u0;
+        const int parts = max(1, min(kDecWarps, p.r) / max(nr, 1));
+        float* upart = us;
+        const int cpx = p.d / V, per = (cpx + parts - 1) / parts;
+        const T* xg = static_cast<const T*>(p.x);
+        constexpr int UA = NT <= 1 ? 8 : 4;
+        for (int jj = warp; jj < nr * parts; jj += kDecWarps) {
+            const int j = u0 + jj / parts, part = jj - (jj / parts) * parts;
+            const int ce = min(cpx, (part + 1) * per);
+            const T* arow = static_cast<const T*>(p.at) + (size_t)j * p.d;
+            float2 a2[NT];
+#pragma unroll
+            for (int t = 0; t < NT; ++t) a2[t] = make_float2(0.f, 0.f);
+            for (int cb = part * per + lane; cb < ce; cb += 32 * UA) {
+                uint4 wa[UA], xv[UA][NT];
+#pragma unroll
+                for (int u2 = 0; u2 < UA; ++u2) {
+                    const int c = cb + 32 * u2;
+                    wa[u2] = c < ce ? ld_stream(arow + (size_t)c * V) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t)
+                        xv[u2][t] = (c < ce && t < n) ? __ldcg(reinterpret_cast<const uint4*>(xg + (size_t)t * p.d) + c)
+                                                      : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u2 = 0; u2 < UA; ++u2) {
+                    float2 af[V / 2];
+                    unpack2<T>(wa[u2], af);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        float2 xf[V / 2];
+                        unpack2<T>(xv[u2][t], xf);
+#pragma unroll
+                        for (int e = 0; e < V / 2; ++e) a2[t] = __ffma2_rn(af[e], xf[e], a2[t]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const float v = warp_sum(a2[t].x + a2[t].y);
+                if (lane == 0) upart[jj * NT + t] = v;
+            }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < nr * n; i += kDecThreads) {
+            const int jr = i / n, t = i - jr * n;
+            float sum = 0.f;
+            for (int q = 0; q < parts; ++q) sum += upart[(jr * parts + q) * NT + t];
+            p.u[(size_t)t * p.r + u0 + jr] = sum;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            utarget = grid_arrive(bar + 1, gridDim.x);
+        }
+    }
     stage_rows<T, T, NT>(xs, static_cast<const T*>(p.x), p.d, 0, n, p.xh != nullptr);
     if (streamer) {
         while (issued < min(p.nb, wcount)) issue_next();
@@ -286,19 +351,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     }
     __syncthreads();
     if (GATE == kGateLopa) {
-        // LoPA stage 1 inside the launch: this CTA's rows of u = x A (one per
-        // warp), published; a grid barrier; then every CTA stages all of u.
-        // The wait is bounded and cannot deadlock: all CTAs are resident.
-        for (int j = u0 + warp; j < u1; j += kDecWarps) {
-            float acc[NT];
-            warp_dot_global<T, NT>(static_cast<const T*>(p.at) + (size_t)j * p.d, p.d / V, xs, p.d, acc);
-            if (lane == 0)
-                for (int t = 0; t < n; ++t) p.u[(size_t)t * p.r + j] = acc[t];
-        }
-        __syncthreads();
         if (threadIdx.x == 0) {
-            __threadfence();
-            const unsigned long long target = grid_arrive(bar + 1, gridDim.x);
+            const unsigned long long target = utarget;
             const unsigned long long t0 = globaltimer_ns();
             unsigned backoff = 32;
             int ok = 1;
