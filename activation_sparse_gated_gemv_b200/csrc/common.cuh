@@ -44,8 +44,21 @@ __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// 16-byte streaming load of read-only weights: bypasses L1 allocation.
+// 16-byte load of weights read once, cached in L2 only.  (The non-coherent
+// path, ld.global.nc, measured much slower for these row reads behind a full
+// stream of bulk copies: an 8 KB up-dot row took 3.7-4.5 us instead of
+// 2.1-2.6 us at the end of the gate stream.)
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 v;
+    asm("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+// The same through the non-coherent path without L1 allocation: faster for
+// the dense FFN's sweep of every W_down row (53.8 against 52.7 us on the 7B
+// shape).
+__device__ __forceinline__ uint4 ld_stream_nc(const void* p) {
     uint4 v;
     asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)

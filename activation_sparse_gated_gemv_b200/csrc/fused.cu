@@ -632,9 +632,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             for (int s0 = 0; s0 < tot; s0 += UBD) {
                 uint4 w[UBD];
 #pragma unroll
-                for (int u2 = 0; u2 < UBD; ++u2)
-                    w[u2] = s0 + u2 < tot ? ld_stream(wdn + (size_t)(c0 + slot_of(s0 + u2)) * p.d + (size_t)cch * V)
-                                          : make_uint4(0u, 0u, 0u, 0u);
+                for (int u2 = 0; u2 < UBD; ++u2) {
+                    if (s0 + u2 >= tot) {
+                        w[u2] = make_uint4(0u, 0u, 0u, 0u);
+                    } else {
+                        const T* src = wdn + (size_t)(c0 + slot_of(s0 + u2)) * p.d + (size_t)cch * V;
+                        w[u2] = dense ? ld_stream_nc(src) : ld_stream(src);
+                    }
+                }
 #pragma unroll
                 for (int u2 = 0; u2 < UBD; ++u2) {
                     if (s0 + u2 < tot) {
