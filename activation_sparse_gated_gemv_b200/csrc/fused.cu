@@ -1,6 +1,6 @@
 // Fused decode path (threshold selection, a few tokens): one kernel streams
-// the gate, selects, takes the up dots, adds the CTA's share of the down
-// projection and sums the per-CTA partials, one column slice per CTA.
+// the gate, selects, takes the up dots, and runs the down projection and its
+// cross-CTA reduction.
 //
 // "Model Casting and Low-Parameter Gating" (abstract): the gating matrix is
 // evaluated first and the two other matrices are touched only for channels
@@ -10,23 +10,29 @@
 // (LoPA: first each CTA computes its rows of u = x A, and a grid barrier
 // publishes u to all CTAs):
 //   * warps 0..13 stream the CTA's gate rows (dense W_gate, or LoPA's B) through
-//     per-warp rings of bulk copies (TMA engine, mbarriers) and leave per-piece
-//     dot products in shared memory.  When a row's last piece is in, the warp
-//     that finished it adds the pieces in order (z), selects (z > tau), and for
-//     an active channel pulls its W_down row into L2 and queues the channel;
+//     per-warp rings of bulk copies (TMA engine, mbarriers).  Long rows come in
+//     parts whose dot products meet in shared memory; short rows (LoPA's B)
+//     come several to a piece and are dotted and selected together.  For a
+//     complete row the warp forms z, selects (z > tau) and queues an active
+//     channel (with the dense gate and the own-row reduction below, it also
+//     pulls the channel's W_up and W_down rows into L2);
 //   * with a heavy-hitter set, warps 14 and 15 first take the up dots of the
 //     CTA's hot channels, before and independent of the gate;
 //   * warps 14 and 15 take queued channels at once and compute the up dot
 //     <x, W_up[:,k]> (a hot channel's is already in) and h = (z - tau) u (the
 //     streaming warps join them when their pieces are done), so the W_up rows
 //     are read while the gate streams;
-//   * after a barrier the active channels are compacted in ascending order
-//     and every thread adds, for its 8 (or 4) output columns, h_k W_down[k,:]
-//     over that ordered list (whole rows, mostly in L2 by now), and stores the
-//     CTA's fp32 partial of y;
-//   * a grid-wide barrier (a counter that only grows, so nothing resets it),
-//     then every CTA sums one column slice of y over all CTAs' partials (in
-//     L2) in a fixed order and stores it.
+//   * d <= 4096 (own rows): after a barrier the active channels are compacted
+//     in ascending order and every thread adds, for its 8 (or 4) output
+//     columns, h_k W_down[k,:] over that ordered list and stores the CTA's
+//     fp32 partial of y; a grid-wide barrier (a counter that only grows, so
+//     nothing resets it); then every CTA sums one column slice of y over all
+//     CTAs' partials in a fixed order and stores it;
+//   * larger d (union gather): each CTA publishes its kept-slot mask and h, a
+//     grid-wide barrier, then every CTA builds the union's ascending channel
+//     list and sums its column slice of h_k W_down[k, slice] over it.
+// A host forward with page-locked x passes its device address: the first CTA
+// copies x in and the others wait for it on an arrival counter.
 // Every sum has a fixed order, so y is bitwise reproducible.
 #include "common.cuh"
 #include "dot.cuh"

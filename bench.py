@@ -129,11 +129,38 @@ def select_args(wl):
     return dict(select="topk", k=wl.k)
 
 
+def code_only(src: str) -> str:
+    """C/C++/CUDA source without its comments and blank space, so that a change
+    to comments alone does not count as a change of the kernels (string and
+    character literals are kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_hash() -> str:
+    """Hash of the kernel sources' code (comments and layout left out)."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(KERNEL_SOURCES, "*"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode() + f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(os.path.basename(p).encode() + code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
