@@ -593,7 +593,7 @@ def main():
                 dffns.append(f)
         Rd = len(dffns)
         gate_d = "dense"
-        Kd = min(a.steps, 2000)
+        Kd = 2000                  # a comparator outside the timed region: always enough steps
         with torch.cuda.stream(stream):
             for i in range(min(a.warmup, 50)):
                 dffns[i % Rd].forward(xs[i % P], gate=gate_d, out=ys[i % P], dense=True, stream=stream, **sel)
@@ -603,6 +603,8 @@ def main():
                 dffns[i % Rd].forward(xs[i % P], gate=gate_d, out=ys[i % P], dense=True, stream=stream, **sel)
         reps = max(1, Kd // 64)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            gd.replay()                # untimed: a graph's first launch uploads it
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             e0.record(stream)
@@ -620,7 +622,7 @@ def main():
     # -- end to end through the C ABI with host buffers
     xs_host = [x.cpu().pin_memory() for x in xs]
     ys_host = [torch.empty((wl.n, wl.d), dtype=xs[0].dtype).pin_memory() for _ in range(P)]
-    Ke = max(20, min(a.e2e_steps, a.steps))
+    Ke = max(20, a.e2e_steps)     # host-timed, so not tied to the (possibly short) timed region
     # the C entry point itself, its arguments built once (what a caller with
     # its own buffers does); each call copies x in, runs the forward, copies y
     # out and synchronises
