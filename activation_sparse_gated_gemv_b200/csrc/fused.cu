@@ -382,8 +382,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
 
     // A selected channel's W_up and W_down rows go to L2 at once when the gate
     // is dense and the CTA sums its own rows (measured: 0.7 us faster on the
-    // 7B shape; slower with LoPA's short gate stream and with the union
-    // gather, whose reads are column slices).
+    // 7B shape).  With LoPA the prefetches of many channels land in one burst
+    // right after the short gate stream (1.7 us slower at 80 % sparsity), and
+    // with the union gather the W_down reads are column slices (3.2 us slower).
     const bool l2_prefetch = GATE == kGateDense && p.own_rows;
     // Row s is complete: z from its parts in order, select, queue it.  Dense
     // mode: the up dot is complete too (parts ppr ..), so h is formed here
@@ -607,7 +608,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
     if (dense || p.own_rows) {
         // ---- own rows: the CTA's kept slots in ascending order (every slot in
         // the dense FFN).  Each thread adds, for its 16-byte column chunks,
-        // h_k W_down[k, :] over those rows (8 rows in flight), stores the CTA's
+        // h_k W_down[k, :] over those rows (16 rows in flight), stores the CTA's
         // fp32 partial of y, and after a grid barrier every CTA sums one column
         // slice of y over the partials in CTA order.
         int tot = nslots;
@@ -627,7 +628,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeParams p)
             tot = scan_sh[0];
         }
         auto slot_of = [&](int i) { return dense ? i : wl[i]; };
-        constexpr int UBD = 8;
+        constexpr int UBD = 16;
         const int cpd = p.d / V;                          // 16-byte chunks per output row
         for (int cch = threadIdx.x; cch < cpd; cch += kDecThreads) {
             float2 acc[NT][V / 2];

@@ -155,18 +155,44 @@ def code_only(src: str) -> str:
     return " ".join("".join(out).split())
 
 
-def kernel_hash() -> str:
-    """Hash of the kernel sources' code (comments and layout left out)."""
+# The sources each kernel family is built from (plus the shared header and the
+# host code that sets its launch parameters).
+KERNEL_FAMILY_FILES = {
+    "decode": ["fused.cu", "dot.cuh"],
+    "tc": ["tc.cu"],
+    "topk": ["topk.cu"],
+    "gate": ["gate.cu", "dot.cuh"],
+    "down": ["down.cu"],
+}
+COMMON_KERNEL_FILES = ["common.cuh", "api.cu"]
+
+
+def kernel_family(kernel: str) -> str:
+    if kernel.startswith("decode"):
+        return "decode"
+    if kernel.startswith("tc_") or kernel == "union_list":
+        return "tc"
+    if kernel in ("topk", "topp"):
+        return "topk"
+    if kernel == "down":
+        return "down"
+    return "gate"
+
+
+def kernel_hash(family: str) -> str:
+    """Hash of the code (comments and layout left out) of one kernel family's
+    sources."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(KERNEL_SOURCES, "*"))):
-        with open(p, encoding="utf-8") as f:
-            h.update(os.path.basename(p).encode() + code_only(f.read()).encode())
+    for name in sorted(set(KERNEL_FAMILY_FILES[family] + COMMON_KERNEL_FILES)):
+        with open(os.path.join(KERNEL_SOURCES, name), encoding="utf-8") as f:
+            h.update(name.encode() + code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str, workload: str, tokens: int):
     """Per-launch DRAM bytes from a committed ncu capture, if it was taken on
-    the current kernel sources (keyed by workload and token count)."""
+    the current code of the kernel's sources (keyed by workload and token
+    count)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -175,7 +201,7 @@ def traffic_for(kernel: str, workload: str, tokens: int):
         return None
     ent = (data.get(f"{workload}:n{tokens}") or data.get(workload, {}) if tokens > 1 else
            data.get(workload, {})).get(kernel)
-    if not ent or ent.get("kernel_hash") != kernel_hash():
+    if not ent or ent.get("kernel_hash") != kernel_hash(kernel_family(kernel)):
         return None
     return ent.get("dram_bytes_per_launch")
 

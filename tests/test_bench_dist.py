@@ -74,14 +74,15 @@ def test_reference_arm_prints_only_on_rank_zero(tmp_path):
 
 
 def test_traffic_is_reported_only_for_the_current_kernel_sources(tmp_path, monkeypatch):
-    """A committed ncu traffic figure is used only while the kernel sources
-    still hash to the value it was captured on; otherwise the bench reports null."""
+    """A committed ncu traffic figure is used only while its kernel family's
+    sources still hash to the value it was captured on; otherwise the bench
+    reports null."""
     sys.path.insert(0, ROOT)
     import bench
     (tmp_path / "profiles").mkdir()
-    ent = {"dram_bytes_per_launch": 123, "kernel_hash": bench.kernel_hash()}
+    ent = {"dram_bytes_per_launch": 123, "kernel_hash": bench.kernel_hash("decode")}
     data = {"llama7b-decode": {"decode_fused": ent},
-            "llama70b:n16": {"tc_up": dict(ent, dram_bytes_per_launch=456)}}
+            "llama70b:n16": {"tc_up": {"dram_bytes_per_launch": 456, "kernel_hash": bench.kernel_hash("tc")}}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(data))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.traffic_for("decode_fused", "llama7b-decode", 1) == 123
@@ -90,3 +91,17 @@ def test_traffic_is_reported_only_for_the_current_kernel_sources(tmp_path, monke
     data["llama7b-decode"]["decode_fused"]["kernel_hash"] = "0" * 16
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(data))
     assert bench.traffic_for("decode_fused", "llama7b-decode", 1) is None
+    # a tensor-core figure keyed with the decode family's hash does not count
+    data["llama70b:n16"]["tc_up"]["kernel_hash"] = bench.kernel_hash("decode")
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(data))
+    assert bench.traffic_for("tc_up", "llama70b", 16) is None
+
+
+def test_kernel_hash_ignores_comments_and_layout():
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f(int x) { // add one\n  return x + 1; /* done */ }\n"
+    b = "int f(int x)\n{\n    return x + 1;\n}\n"
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only('const char* s = "// kept";') == 'const char* s = "// kept";'
+    assert bench.code_only("return x + 1;") != bench.code_only("return x + 2;")
