@@ -612,6 +612,10 @@ int sffn_create(sffn_handle* out, const sffn_config* cfg) {
     P.mw = (c.max_tokens + 31) / 32;
     P.down_slices = (c.d + down_slice_cols(c.wdtype) - 1) / down_slice_cols(c.wdtype);
     P.down_chunks = h->sms / P.down_slices;                 // about one down CTA per SM
+    // ... but at least 128 channels per chunk: the last CTA of a slice adds the
+    // chunks' partials one after another (a 1024-channel FFN cut into 147
+    // chunks of 7 took 138 us there for 8 tokens)
+    if (P.down_chunks > (c.d_ff + 127) / 128) P.down_chunks = (c.d_ff + 127) / 128;
     if (P.down_chunks < 1) P.down_chunks = 1;
     if (P.down_chunks > P.g1) P.down_chunks = P.g1;
 

@@ -155,8 +155,9 @@ def code_only(src: str) -> str:
     return " ".join("".join(out).split())
 
 
-# The sources each kernel family is built from (plus the shared header and the
-# host code that sets its launch parameters).
+# The device sources each kernel family is built from (plus the shared
+# header); the launch geometry of the decode and tensor-core kernels is
+# computed in their own files.
 KERNEL_FAMILY_FILES = {
     "decode": ["fused.cu", "dot.cuh"],
     "tc": ["tc.cu"],
@@ -164,7 +165,7 @@ KERNEL_FAMILY_FILES = {
     "gate": ["gate.cu", "dot.cuh"],
     "down": ["down.cu"],
 }
-COMMON_KERNEL_FILES = ["common.cuh", "api.cu"]
+COMMON_KERNEL_FILES = ["common.cuh"]
 
 
 def kernel_family(kernel: str) -> str:
