@@ -105,3 +105,19 @@ def test_kernel_hash_ignores_comments_and_layout():
     assert bench.code_only(a) == bench.code_only(b)
     assert bench.code_only('const char* s = "// kept";') == 'const char* s = "// kept";'
     assert bench.code_only("return x + 1;") != bench.code_only("return x + 2;")
+
+
+def test_bench_bytes_match_the_pinned_oracle_counter():
+    """The roofline numerator (bench.algorithmic_bytes and dense_bytes) is the
+    oracle's byte counter, which a pin checks against an enumerated read list."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    import workloads
+    for wl in (workloads.llama7b_decode(0.9), workloads.lopa7b(0.9), workloads.llama70b(4, "lopa", 0.9),
+               workloads.llama70b(16, "dense", 0.9), workloads.tiny()):
+        w = 2 if wl.dtype == "bf16" else 4
+        for union in (0, 1, 1108, wl.d_ff):
+            assert bench.algorithmic_bytes(wl, union) == oracle.bytes_moved(
+                wl.n, wl.d, wl.d_ff, union, w, w, r=wl.r if wl.gate == "lopa" else 0), (wl.name, union)
+        assert bench.dense_bytes(wl) == oracle.dense_bytes(wl.n, wl.d, wl.d_ff, w, w)
